@@ -1,0 +1,238 @@
+/*
+ * nq.h -- C ABI of the B200 (sm_100a) NanoQuant hot path.
+ *
+ * Two operations, from the NanoQuant pages (arXiv 2602.06694 summaries):
+ *
+ *   1. Calibration preconditioners.  NanoQuant summary page (paper.rainbus.top),
+ *      "Method steps" (方法步骤详情), stage one: per-linear-layer statistics z_in,
+ *      z_out collected over 128 x 2048 calibration tokens are regularised by
+ *      Ledoit-Wolf shrinkage into diagonal preconditioners D_in, D_out.  Here
+ *      z_in / z_out are the per-channel second moments of the input activations
+ *      and of the output gradients (the diagonals of the K-FAC factors, same page,
+ *      "Prerequisites" (前置知识), K-FAC paragraph).
+ *
+ *   2. LB-ADMM initialisation.  Same page, "Core method" (核心方法) and "Method
+ *      steps" stage two: the preconditioned target W~ = D_out W D_in is factorised
+ *      as diag(s1) U+-1 V+-1^T diag(s2) by an ADMM over continuous latents U, V
+ *      with (a) a Cholesky-solved regularised U (V) step, (b) an SVID projection
+ *      to a binary proxy Z, (c) a dual update; then magnitude balancing, channel
+ *      scale extraction and packing of the signs into integer words.
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major.  W is m x n (out x in features, the PyTorch layout).
+ *   - Pointers named "device" must be CUDA device (or managed) memory of the
+ *     current device; "host" pointers are ordinary host memory.
+ *   - The caller owns every buffer.  The library allocates no device memory:
+ *     all scratch lives in the caller's workspace ``ws`` (size from the matching
+ *     *_workspace_size function; 256-byte alignment required).
+ *   - All device work is enqueued on ``stream``.  Entry points that fill host
+ *     outputs synchronise ``stream`` before returning; the others return as soon
+ *     as the work is enqueued.
+ *   - Argument errors are reported before anything is launched.  Errors detected
+ *     on the device (non-finite values, a non-positive Cholesky pivot, a wait that
+ *     ran out) are reported by the next synchronising call on the same workspace.
+ *     On error, outputs are unspecified.
+ *   - Not thread-safe per workspace: two calls that share a workspace must be
+ *     ordered on the same stream.
+ */
+#ifndef NQ_H
+#define NQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nq_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    NQ_OK = 0,
+    NQ_ERR_INVALID_ARG = 1,  /* bad size, null pointer, misaligned buffer, bad dtype       */
+    NQ_ERR_WORKSPACE = 2,    /* workspace too small                                       */
+    NQ_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                          */
+    NQ_ERR_NONFINITE = 4,    /* NaN or Inf found in an input                               */
+    NQ_ERR_NOT_SPD = 5,      /* non-positive pivot in a Cholesky factorisation             */
+    NQ_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out                         */
+    NQ_ERR_UNSUPPORTED = 7   /* no sm_100a device, or a size beyond the supported range    */
+} nq_status;
+
+typedef enum { NQ_F32 = 0, NQ_BF16 = 1 } nq_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nq_status_string(nq_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t nq_version(void);
+
+/* ------------------------------------------------------------------------- */
+/* Bits-per-weight accounting.  NanoQuant summary page, "Motivation" (研究动机)  */
+/* and "Results" (实验结果): BPW counts one bit per sign of U (m x r) and V      */
+/* (n x r) and 16 bits per entry of s1 (m) and s2 (n).                         */
+/* ------------------------------------------------------------------------- */
+
+/* ((m+n) r + 16 (m+n)) / (m n).  Returns -1 for m <= 0, n <= 0 or r < 0. */
+double nq_bpw(int64_t m, int64_t n, int32_t r);
+
+/* Largest r with nq_bpw(m, n, r) <= bpw: floor((bpw m n - 16 (m+n)) / (m+n)),
+ * clamped at 0.  bpw is read as a decimal (a result within 1e-9 of an integer is
+ * taken as that integer).  Returns -1 for m <= 0 or n <= 0 or bpw < 0. */
+int32_t nq_rank_for_bpw(int64_t m, int64_t n, double bpw);
+
+/* ------------------------------------------------------------------------- */
+/* 1. Calibration preconditioners                                              */
+/* ------------------------------------------------------------------------- */
+
+/* Workspace bytes for nq_calib_stats / nq_calib_precond on streams of at most
+ * T tokens and C channels (either stream). */
+size_t nq_calib_workspace_size(int64_t T, int64_t C);
+
+/*
+ * Per-channel moments of one token-major stream X (T x C, dtype dt):
+ *     s_j = (1/T) sum_t X_tj^2,   q_j = (1/T) sum_t X_tj^4.
+ * X: device, row stride C elements.  s, q: device, C doubles each.
+ * Accumulation: FP32 within a slab of tokens, FP64 across slabs, fixed order
+ * (bit-identical from run to run).  Enqueue only.
+ */
+nq_status nq_calib_stats(const void *X, int64_t T, int64_t C, nq_dtype dt, double *s, double *q,
+                         void *ws, size_t ws_bytes, nq_stream_t stream);
+
+/*
+ * Diagonal preconditioners from the activation stream (T_in x n) and the output
+ * gradient stream (T_out x m):
+ *     mu = mean(s), delta^2 = sum_j (s_j - mu)^2, beta_bar^2 = (1/T) sum_j (q_j - s_j^2),
+ *     alpha = min(beta_bar^2, delta^2) / delta^2 (1 if delta^2 = 0),
+ *     d~ = (1 - alpha) s + alpha mu,   d = sqrt(max(d~, 1e-12 mu))
+ * (Ledoit & Wolf 2004 with target mu I, restricted to the diagonal).
+ * alpha_override >= 0 replaces alpha by that value; < 0 selects Ledoit-Wolf.
+ * acts, grads: device.  d_in (n), d_out (m): device float.
+ * alpha_out: host double[2] {alpha_in, alpha_out}, or NULL.  When non-NULL the call
+ * synchronises the stream; otherwise it only enqueues.
+ */
+nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void *grads,
+                           int64_t T_out, int64_t m, nq_dtype dt, double alpha_override,
+                           float *d_in, float *d_out, double *alpha_out, void *ws,
+                           size_t ws_bytes, nq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* 2. LB-ADMM                                                                  */
+/* ------------------------------------------------------------------------- */
+
+/* Supported sizes: 1 <= m, n <= 65536; 1 <= r <= min(m, n, 4096). */
+
+/* Workspace bytes for an m x n layer at rank r (holds the whole ADMM state). */
+size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
+
+/*
+ * Full LB-ADMM initialisation of one layer.
+ *
+ * Form of the iteration (the pages give no equations; this is the concrete form
+ * implemented, step for step the same as the library's FP64 reference):
+ *   W^ = W~ / gamma, gamma = ||W~||_F / (2 sqrt(r)), stored as BF16 (RNE);
+ *   V_0[j][k] = sqrt(2/n) * (-1 if bit 63 of SplitMix64(seed, j*r+k) else +1);
+ *   Z_U = L_U = Z_V = L_V = 0;
+ *   repeat iters times:
+ *     U = (W^ V + rho (Z_U - L_U)) (V^T V + (lambda + rho) I)^-1      (Cholesky)
+ *     S = U + L_U;  A = |S|;  b = 1;  K times { a = A b / ||A b||;  b = A^T a }
+ *     Z_U = sign(S) * a b^T;   L_U = L_U + U - Z_U
+ *     the same for V with W^^T and U
+ *     objective[t] = ||W^ - U V^T||_F^2 / ||W^||_F^2
+ *   g_k = sqrt(||V_:k|| / ||U_:k||);  U_:k *= g_k;  V_:k /= g_k
+ *   s1_i = gamma mean_k |U_ik|,  s2_j = mean_k |V_jk|
+ *   sign bit = (latent < 0), LSB-first along k, row-major uint32[rows][(r+31)/32]
+ * Tensor-core operands (W^ and the latent factor of the contraction) are BF16;
+ * accumulation and every other quantity is FP32 (reductions FP64 where noted).
+ *
+ * W: device, m x n, dtype dt.  d_in (n), d_out (m): device float, or NULL for 1.
+ * U_packed: device uint32 [m][(r+31)/32];  V_packed: device uint32 [n][(r+31)/32].
+ * s1 (m), s2 (n): device float; scales of W~ (for the raw W use s1/d_out, s2/d_in).
+ * objective: host float[iters] or NULL.  final_rel_err: host, or NULL:
+ *     ||W~ - diag(s1) U+- V+-^T diag(s2)||_F / ||W~||_F.
+ * Synchronises the stream when objective or final_rel_err is non-NULL.
+ * Requires rho > 0, lambda >= 0, iters >= 1, K >= 1.
+ */
+nq_status nq_lbadmm(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                    const float *d_out, int32_t r, float rho, float lambda, int32_t iters,
+                    int32_t K, uint64_t seed, uint32_t *U_packed, uint32_t *V_packed, float *s1,
+                    float *s2, float *objective, float *final_rel_err, void *ws,
+                    size_t ws_bytes, nq_stream_t stream);
+
+/*
+ * Reconstruction error of a packed factorisation against W~ = D_out W D_in:
+ *     ||W~ - diag(s1) U+- V+-^T diag(s2)||_F / ||W~||_F   (0 if both norms vanish).
+ * All array arguments are device pointers as in nq_lbadmm; rel_err is host.
+ * Uses a +-1 tensor-core GEMM (exact for r <= 4096) with a fused squared-error
+ * reduction.  Synchronises the stream.
+ */
+size_t nq_recon_workspace_size(int64_t m, int64_t n, int32_t r);
+nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                         const float *d_out, const uint32_t *U_packed, const uint32_t *V_packed,
+                         int32_t r, const float *s1, const float *s2, double *rel_err, void *ws,
+                         size_t ws_bytes, nq_stream_t stream);
+
+/*
+ * Sign packing alone: bits[i][k/32] bit (k%32) = (X[i][k] < 0); -0.0 packs as 0.
+ * X: device float rows x r.  bits: device uint32 rows x (r+31)/32.  Enqueue only.
+ */
+nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,
+                        nq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Step-level interface over the ADMM state held in the workspace.             */
+/* nq_lbadmm is nq_lbadmm_prepare + nq_lbadmm_iterate + nq_lbadmm_finish.      */
+/* The state fields can be read and written (checkpoint / resume, tests).      */
+/* ------------------------------------------------------------------------- */
+
+/* Form W^ (and its transpose) from W, d_in, d_out; set V = V_0(seed) and zero the
+ * dual state.  gamma_out: host double or NULL (synchronises when non-NULL). */
+nq_status nq_lbadmm_prepare(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                            const float *d_out, int32_t r, uint64_t seed, double *gamma_out,
+                            void *ws, size_t ws_bytes, nq_stream_t stream);
+
+/* Run ``iters`` full iterations (U side then V side).  objective: host float[iters]
+ * or NULL (synchronises when non-NULL). */
+nq_status nq_lbadmm_iterate(int64_t m, int64_t n, int32_t r, float rho, float lambda,
+                            int32_t iters, int32_t K, float *objective, void *ws, size_t ws_bytes,
+                            nq_stream_t stream);
+
+/* One half iteration: side 0 updates U from V, side 1 updates V from U. */
+nq_status nq_lbadmm_half_step(int64_t m, int64_t n, int32_t r, float rho, float lambda, int32_t K,
+                              int32_t side, void *ws, size_t ws_bytes, nq_stream_t stream);
+
+/* Balance, extract s1/s2, pack, and (when final_rel_err != NULL) the reconstruction
+ * error against W~ formed from W, d_in, d_out (synchronises then). */
+nq_status nq_lbadmm_finish(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                           const float *d_out, int32_t r, uint32_t *U_packed, uint32_t *V_packed,
+                           float *s1, float *s2, float *final_rel_err, void *ws, size_t ws_bytes,
+                           nq_stream_t stream);
+
+/* State fields.  X = latent after its last step (rows x r, float); S = X + L, the
+ * SVID input, from which the dual state is Z = sign(S) a b^T, L = S - Z (rows x r,
+ * float); A = a (rows, float); B = b (r, float); WHAT = W^ (m x n, bf16, row
+ * stride ld elements); GAMMA = gamma (1 double). */
+typedef enum {
+    NQ_FIELD_U = 0, NQ_FIELD_V = 1, NQ_FIELD_SU = 2, NQ_FIELD_SV = 3, NQ_FIELD_AU = 4,
+    NQ_FIELD_AV = 5, NQ_FIELD_BU = 6, NQ_FIELD_BV = 7, NQ_FIELD_WHAT = 8, NQ_FIELD_GAMMA = 9
+} nq_field;
+
+/* Device address, element count, element size and row stride (elements) of a
+ * state field inside the workspace.  The address is valid while ws is. */
+nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, void *ws,
+                                size_t ws_bytes, void **dev_ptr, int64_t *count,
+                                int32_t *elem_bytes, int64_t *ld);
+
+/* Re-derive the BF16 operand copies (transposes of U and V and W^^T) after a
+ * caller has written NQ_FIELD_U / NQ_FIELD_V / NQ_FIELD_WHAT directly. */
+nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
+                                  nq_stream_t stream);
+
+/* Device error word of a workspace: 0 if clean, else the first nq_status raised
+ * on the device since the last reset; resets it.  Synchronises the stream. */
+nq_status nq_lbadmm_check(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
+                          nq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NQ_H */

@@ -1,0 +1,80 @@
+"""ctypes binding of ``libnq.so`` (the C ABI declared in include/nq.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA library.
+Tensors are passed by ``data_ptr()``; the stream is torch's current CUDA stream.
+If the shared library is missing this module raises at import: there is no CPU
+fallback.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m rank_binary_factorization_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+c_i32, c_i64, c_u64, c_f32, c_f64 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
+                                      ctypes.c_float, ctypes.c_double)
+c_vp, c_sz = ctypes.c_void_p, ctypes.c_size_t
+
+NQ_OK, NQ_ERR_INVALID_ARG, NQ_ERR_WORKSPACE, NQ_ERR_CUDA, NQ_ERR_NONFINITE, NQ_ERR_NOT_SPD, \
+    NQ_ERR_TIMEOUT, NQ_ERR_UNSUPPORTED = range(8)
+NQ_F32, NQ_BF16 = 0, 1
+FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9)
+
+# name -> (restype, argtypes); the list is the full set of exported entry points
+SIGNATURES = {
+    "nq_status_string": (ctypes.c_char_p, [c_i32]),
+    "nq_version": (c_i32, []),
+    "nq_bpw": (c_f64, [c_i64, c_i64, c_i32]),
+    "nq_rank_for_bpw": (c_i32, [c_i64, c_i64, c_f64]),
+    "nq_calib_workspace_size": (c_sz, [c_i64, c_i64]),
+    "nq_calib_stats": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_calib_precond": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_i32, c_f64, c_vp,
+                                 c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_lbadmm_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
+    "nq_lbadmm": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_f32, c_f32, c_i32,
+                          c_i32, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_recon_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
+    "nq_recon_error": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp,
+                               c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_pack_signs": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_vp]),
+    "nq_lbadmm_prepare": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_u64, c_vp,
+                                  c_vp, c_sz, c_vp]),
+    "nq_lbadmm_iterate": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp,
+                                  c_sz, c_vp]),
+    "nq_lbadmm_half_step": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_sz,
+                                    c_vp]),
+    "nq_lbadmm_finish": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
+                                 c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_lbadmm_state_field": (c_i32, [c_i64, c_i64, c_i32, c_i32, c_vp, c_sz,
+                                      ctypes.POINTER(c_vp), ctypes.POINTER(c_i64),
+                                      ctypes.POINTER(c_i32), ctypes.POINTER(c_i64)]),
+    "nq_lbadmm_sync_operands": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
+    "nq_lbadmm_check": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
+}
+
+for _name, (_res, _args) in SIGNATURES.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class NQError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+
+
+def status_string(code):
+    return lib.nq_status_string(int(code)).decode()
+
+
+def check(fn, code):
+    if code != NQ_OK:
+        raise NQError(fn, code)
+    return code

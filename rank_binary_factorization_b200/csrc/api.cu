@@ -1,0 +1,634 @@
+// C ABI of the library (declared in include/nq.h): argument checks, workspace
+// carving and the launch sequence of each entry point.  No device allocation.
+#include <math.h>
+#include <string.h>
+
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+#include "layout.h"
+
+using namespace nq;
+
+namespace {
+
+#define NQ_CK(call)                                  \
+    do {                                             \
+        cudaError_t e_ = (call);                     \
+        if (e_ != cudaSuccess) return NQ_ERR_CUDA;   \
+    } while (0)
+
+inline cudaStream_t cs(nq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+template <class T>
+inline T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+// The library only runs on sm_100 devices (the kernels are built for sm_100a).
+nq_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NQ_ERR_CUDA;
+    static int cached[64];
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? NQ_OK : NQ_ERR_UNSUPPORTED;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return NQ_ERR_CUDA;
+    const bool ok = major == 10;
+    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? NQ_OK : NQ_ERR_UNSUPPORTED;
+}
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nq_status check_lb_args(int64_t m, int64_t n, int32_t r) {
+    if (m < 1 || n < 1 || m > kMaxDim || n > kMaxDim) return NQ_ERR_INVALID_ARG;
+    if (r < 1 || r > kMaxRank || r > m || r > n) return NQ_ERR_INVALID_ARG;
+    return NQ_OK;
+}
+
+nq_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+    if (!ws) return NQ_ERR_INVALID_ARG;
+    if (!aligned(ws, kAlign)) return NQ_ERR_INVALID_ARG;
+    if (ws_bytes < need) return NQ_ERR_WORKSPACE;
+    return NQ_OK;
+}
+
+int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
+
+nq_status read_err(int *dev_err, cudaStream_t s, bool reset) {
+    int h = 0;
+    NQ_CK(cudaMemcpyAsync(&h, dev_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    NQ_CK(cudaStreamSynchronize(s));
+    if (reset && h) NQ_CK(cudaMemsetAsync(dev_err, 0, sizeof(int), s));
+    return static_cast<nq_status>(h);
+}
+
+size_t calib_ws_bytes(int64_t C) {
+    // token slabs * channels is bounded by 6 * 148 * 256 + C + 256 (see calib_num_slabs)
+    const size_t pd = (size_t)(6 * kNumSMsB200 * 256 + C + 256);
+    return align_up(sizeof(Scalars)) + 2 * align_up(pd * 8) + 2 * align_up((size_t)C * 8);
+}
+
+struct CalibCarve {
+    Scalars *sc;
+    double *ps, *pq, *s, *q;
+};
+CalibCarve carve_calib(void *ws, int64_t C) {
+    const size_t pd = (size_t)(6 * kNumSMsB200 * 256 + C + 256);
+    size_t off = 0;
+    CalibCarve c;
+    c.sc = at<Scalars>(ws, off);
+    off += align_up(sizeof(Scalars));
+    c.ps = at<double>(ws, off);
+    off += align_up(pd * 8);
+    c.pq = at<double>(ws, off);
+    off += align_up(pd * 8);
+    c.s = at<double>(ws, off);
+    off += align_up((size_t)C * 8);
+    c.q = at<double>(ws, off);
+    return c;
+}
+
+nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s_out,
+                        double *q_out, const CalibCarve &cv, cudaStream_t st) {
+    const int nslab = calib_num_slabs(T, C);
+    NQ_CK(calib_partials(X, T, C, bf16, nslab, cv.ps, cv.pq, st));
+    NQ_CK(calib_moments(cv.ps, cv.pq, nslab, T, C, s_out, q_out, st));
+    return NQ_OK;
+}
+
+// ---- LB-ADMM internals ------------------------------------------------------------
+struct Lb {
+    LbLayout L;
+    void *ws;
+    Scalars *sc;
+    template <class T>
+    T *p(size_t off) const {
+        return at<T>(ws, off);
+    }
+};
+
+nq_status lb_open(Lb &lb, int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes) {
+    nq_status st = check_lb_args(m, n, r);
+    if (st) return st;
+    lb.L.build(m, n, r);
+    st = check_ws(ws, ws_bytes, lb.L.total);
+    if (st) return st;
+    lb.ws = ws;
+    lb.sc = at<Scalars>(ws, lb.L.scal);
+    return check_device();
+}
+
+// Gram of the operand of side ``other`` (its BF16 transpose) into g[other].
+nq_status lb_gram(const Lb &lb, int other, float diag, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    const int64_t K = L.rows(other), ld = L.ld_rows(other);
+    const __nv_bfloat16 *xt = lb.p<__nv_bfloat16>(L.xt[other]);
+    const int BN = pick_bn(L.r);
+    tc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!tc::make_map_bf16(&maps.a[0], xt, L.r, K, ld, tc::BM) ||
+        !tc::make_map_bf16(&maps.b[0], xt, L.r, K, ld, BN))
+        return NQ_ERR_CUDA;
+    tc::EpiParams ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.M = L.r;
+    ep.N = L.r;
+    ep.nseg = 1;
+    ep.kblocks[0] = (int)ceil_div(K, tc::BK);
+    ep.err = &lb.sc->err;
+    ep.out = lb.p<float>(L.g[other]);
+    ep.ldo = L.r;
+    ep.diag = diag;
+    NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
+    return NQ_OK;
+}
+
+nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    const int other = 1 - side;
+    const int64_t rows = L.rows(side), Kd = L.rows(other);
+    const int BN = pick_bn(L.r);
+    nq_status st = lb_gram(lb, other, lambda + rho, s);
+    if (st) return st;
+    NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
+                       lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.gih),
+                       lb.p<__nv_bfloat16>(L.gil), L.ldr, &lb.sc->err, lb.sc->bar, s));
+
+    // R = W^ X_other + rho (Z - L), split into hi + lo bf16
+    {
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        const void *A = side == 0 ? lb.p<void>(L.what) : lb.p<void>(L.whatT);
+        const int64_t lda = side == 0 ? L.ldn : L.ldm;
+        if (!tc::make_map_bf16(&maps.a[0], A, rows, Kd, lda, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[0], lb.p<void>(L.xt[other]), L.r, Kd, L.ld_rows(other), BN))
+            return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = (int)rows;
+        ep.N = L.r;
+        ep.nseg = 1;
+        ep.kblocks[0] = (int)ceil_div(Kd, tc::BK);
+        ep.err = &lb.sc->err;
+        ep.S = lb.p<float>(L.s[side]);
+        ep.a = lb.p<float>(L.a[side]);
+        ep.b = lb.p<float>(L.b[side]);
+        ep.ldf = L.ldr;
+        ep.rho = rho;
+        ep.Rhi = lb.p<__nv_bfloat16>(L.rhi);
+        ep.Rlo = lb.p<__nv_bfloat16>(L.rlo);
+        ep.ldr = L.ldr;
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RHS, BN, s));
+    }
+    // X = R G^-1 = [R_hi, R_lo, R_hi] [Gi_hi; Gi_hi; Gi_lo]; S <- X + L; Xt = bf16(X)^T
+    {
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        const void *rh = lb.p<void>(L.rhi), *rl = lb.p<void>(L.rlo);
+        const void *gh = lb.p<void>(L.gih), *gl = lb.p<void>(L.gil);
+        if (!tc::make_map_bf16(&maps.a[0], rh, rows, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[1], rl, rows, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[2], rh, rows, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[0], gh, L.r, L.r, L.ldr, BN) ||
+            !tc::make_map_bf16(&maps.b[1], gh, L.r, L.r, L.ldr, BN) ||
+            !tc::make_map_bf16(&maps.b[2], gl, L.r, L.r, L.ldr, BN))
+            return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = (int)rows;
+        ep.N = L.r;
+        ep.nseg = 3;
+        ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
+        ep.err = &lb.sc->err;
+        ep.S = lb.p<float>(L.s[side]);
+        ep.a = lb.p<float>(L.a[side]);
+        ep.b = lb.p<float>(L.b[side]);
+        ep.ldf = L.ldr;
+        ep.rho = rho;
+        ep.Rhi = lb.p<__nv_bfloat16>(L.rhi);
+        ep.Rlo = lb.p<__nv_bfloat16>(L.rlo);
+        ep.ldr = L.ldr;
+        ep.X = lb.p<float>(L.x[side]);
+        ep.Xt = lb.p<__nv_bfloat16>(L.xt[side]);
+        ep.ldxt = L.ld_rows(side);
+        ep.objective = side == 1;
+        ep.part = lb.p<double>(L.part);
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BN, s));
+    }
+    NQ_CK(svid(lb.p<float>(L.s[side]), rows, L.r, L.ldr, K, L.nsv, lb.p<float>(L.bcur),
+               lb.p<float>(L.tvec), lb.p<float>(L.partb), lb.p<double>(L.partn),
+               lb.p<float>(L.a[side]), lb.p<float>(L.b[side]), s));
+    return NQ_OK;
+}
+
+nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    const int npx = (int)tc::num_tiles((int)L.n, L.r, pick_bn(L.r));
+    NQ_CK(objective(lb.p<float>(L.g[0]), lb.p<float>(L.g[1]), L.r, c, lb.p<double>(L.part), npx,
+                    lb.p<double>(L.partg), lb.sc, lb.p<float>(L.obj) + slot, s));
+    return NQ_OK;
+}
+
+nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
+                     const float *d_out, uint64_t seed, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    NQ_CK(cudaMemsetAsync(lb.sc, 0, sizeof(Scalars), s));
+    NQ_CK(wt_norm_partials(W, bf16, L.m, L.n, d_in, d_out, lb.p<double>(L.part), &lb.sc->err, s));
+    NQ_CK(reduce_partials(lb.p<double>(L.part), kRedBlocks, &lb.sc->wt_norm2, &lb.sc->gamma, L.r,
+                          s));
+    NQ_CK(what_cast(W, bf16, L.m, L.n, d_in, d_out, &lb.sc->gamma, lb.p<__nv_bfloat16>(L.what),
+                    L.ldn, lb.p<__nv_bfloat16>(L.whatT), L.ldm, lb.p<double>(L.part), s));
+    NQ_CK(reduce_partials(lb.p<double>(L.part), kRedBlocks, &lb.sc->what_norm2, nullptr, L.r, s));
+    for (int sd = 0; sd < 2; ++sd) {
+        const int64_t rw = L.rows(sd);
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.s[sd]), 0, (size_t)rw * L.ldr * 4, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.a[sd]), 0, (size_t)rw * 4, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.b[sd]), 0, (size_t)L.r * 4, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.xt[sd]), 0, (size_t)L.r * L.ld_rows(sd) * 2, s));
+    }
+    NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[0]), 0, (size_t)L.m * L.ldr * 4, s));
+    NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[1]), 0, (size_t)L.n * L.ldr * 4, s));
+    NQ_CK(init_v0(L.n, L.r, seed, lb.p<float>(L.x[1]), L.ldr, lb.p<__nv_bfloat16>(L.xt[1]), L.ldn,
+                  s));
+    return NQ_OK;
+}
+
+nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, float *objective_h,
+                     cudaStream_t s) {
+    for (int t = 0; t < iters; ++t) {
+        nq_status st = lb_half_step(lb, 0, rho, lambda, K, s);
+        if (st) return st;
+        if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
+        if ((st = lb_half_step(lb, 1, rho, lambda, K, s))) return st;
+        if (objective_h && t > 0 && (t % kObjRing) == 0) {
+            // the ring holds the objectives of iterations t - kObjRing .. t - 1; the copy is
+            // stream-ordered before the next write to slot 0
+            NQ_CK(cudaMemcpyAsync(objective_h + (t - kObjRing), lb.p<float>(lb.L.obj),
+                                  (size_t)kObjRing * 4, cudaMemcpyDeviceToHost, s));
+        }
+    }
+    // objective of the last iteration needs the Gram of the last V
+    nq_status st = lb_gram(lb, 1, lambda + rho, s);
+    if (st) return st;
+    if ((st = lb_objective(lb, lambda + rho, (iters - 1) % kObjRing, s))) return st;
+    if (objective_h) {
+        const int done = (iters - 1) / kObjRing * kObjRing;
+        NQ_CK(cudaMemcpyAsync(objective_h + done, lb.p<float>(lb.L.obj),
+                              (size_t)(iters - done) * 4, cudaMemcpyDeviceToHost, s));
+    }
+    return NQ_OK;
+}
+
+nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, const float *d_out,
+                    uint32_t *Up, uint32_t *Vp, float *s1, float *s2, bool want_err,
+                    cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    float *pu = lb.p<float>(L.partb);
+    float *pv = pu + (size_t)L.nsv * L.r;
+    NQ_CK(column_sumsq(lb.p<float>(L.x[0]), L.m, L.r, L.ldr, L.nsv, pu, s));
+    NQ_CK(column_sumsq(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, L.nsv, pv, s));
+    NQ_CK(balance_gains(pu, pv, L.nsv, L.r, lb.p<float>(L.gk), s));
+    NQ_CK(extract_pack(lb.p<float>(L.x[0]), L.m, L.r, L.ldr, lb.p<float>(L.gk), 0, &lb.sc->gamma,
+                       s1, Up, lb.p<__nv_bfloat16>(L.rhi), L.ldr, s));
+    NQ_CK(extract_pack(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, lb.p<float>(L.gk), 1, nullptr, s2, Vp,
+                       lb.p<__nv_bfloat16>(L.rlo), L.ldr, s));
+    if (!want_err) return NQ_OK;
+    const int BN = pick_bn(L.n);
+    tc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!tc::make_map_bf16(&maps.a[0], lb.p<void>(L.rhi), L.m, L.r, L.ldr, tc::BM) ||
+        !tc::make_map_bf16(&maps.b[0], lb.p<void>(L.rlo), L.n, L.r, L.ldr, BN))
+        return NQ_ERR_CUDA;
+    tc::EpiParams ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.M = (int)L.m;
+    ep.N = (int)L.n;
+    ep.nseg = 1;
+    ep.kblocks[0] = (int)ceil_div(L.r, tc::BK);
+    ep.err = &lb.sc->err;
+    ep.part = lb.p<double>(L.part);
+    ep.W = W;
+    ep.w_bf16 = bf16;
+    ep.ldw = L.n;
+    ep.d_in = d_in;
+    ep.d_out = d_out;
+    ep.s1 = s1;
+    ep.s2 = s2;
+    NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RECON, BN, s));
+    NQ_CK(recon_finalize(lb.p<double>(L.part), (int)tc::num_tiles((int)L.m, (int)L.n, BN), lb.sc,
+                         &lb.sc->recon2, s));
+    return NQ_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+// Public entry points
+// =====================================================================================
+extern "C" {
+
+const char *nq_status_string(nq_status s) {
+    switch (s) {
+        case NQ_OK: return "NQ_OK";
+        case NQ_ERR_INVALID_ARG: return "NQ_ERR_INVALID_ARG";
+        case NQ_ERR_WORKSPACE: return "NQ_ERR_WORKSPACE";
+        case NQ_ERR_CUDA: return "NQ_ERR_CUDA";
+        case NQ_ERR_NONFINITE: return "NQ_ERR_NONFINITE";
+        case NQ_ERR_NOT_SPD: return "NQ_ERR_NOT_SPD";
+        case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT";
+        case NQ_ERR_UNSUPPORTED: return "NQ_ERR_UNSUPPORTED";
+        default: return "NQ_ERR_UNKNOWN";
+    }
+}
+
+int32_t nq_version(void) { return 100; }
+
+double nq_bpw(int64_t m, int64_t n, int32_t r) {
+    if (m <= 0 || n <= 0 || r < 0) return -1.0;
+    return ((double)(m + n) * r + 16.0 * (double)(m + n)) / ((double)m * (double)n);
+}
+
+int32_t nq_rank_for_bpw(int64_t m, int64_t n, double bpw) {
+    if (m <= 0 || n <= 0 || !(bpw >= 0.0)) return -1;
+    const long double x =
+        ((long double)bpw * (long double)m * (long double)n - 16.0L * (long double)(m + n)) /
+        (long double)(m + n);
+    long double f = floorl(x);
+    if (x - f > 1.0L - 1e-9L) f += 1.0L;  // a decimal bpw landing just below an integer
+    if (f < 0) return 0;
+    if (f > 2147483647.0L) return 2147483647;
+    return (int32_t)f;
+}
+
+size_t nq_calib_workspace_size(int64_t T, int64_t C) {
+    if (T < 1 || C < 1) return 0;
+    return calib_ws_bytes(C);
+}
+
+nq_status nq_calib_stats(const void *X, int64_t T, int64_t C, nq_dtype dt, double *s, double *q,
+                         void *ws, size_t ws_bytes, nq_stream_t stream) {
+    if (!X || !s || !q || T < 1 || C < 1 || (dt != NQ_F32 && dt != NQ_BF16))
+        return NQ_ERR_INVALID_ARG;
+    nq_status st = check_ws(ws, ws_bytes, calib_ws_bytes(C));
+    if (st) return st;
+    if ((st = check_device())) return st;
+    CalibCarve cv = carve_calib(ws, C);
+    return enqueue_stats(X, T, C, dt == NQ_BF16, s, q, cv, cs(stream));
+}
+
+nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void *grads,
+                           int64_t T_out, int64_t m, nq_dtype dt, double alpha_override,
+                           float *d_in, float *d_out, double *alpha_out, void *ws,
+                           size_t ws_bytes, nq_stream_t stream) {
+    if (!acts || !grads || !d_in || !d_out || T_in < 1 || T_out < 1 || n < 1 || m < 1 ||
+        (dt != NQ_F32 && dt != NQ_BF16) || !(alpha_override <= 1.0) || isnan(alpha_override))
+        return NQ_ERR_INVALID_ARG;
+    const int64_t C = n > m ? n : m;
+    nq_status st = check_ws(ws, ws_bytes, calib_ws_bytes(C));
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaStream_t s = cs(stream);
+    CalibCarve cv = carve_calib(ws, C);
+    NQ_CK(cudaMemsetAsync(cv.sc, 0, sizeof(Scalars), s));
+    const int bf16 = dt == NQ_BF16;
+    if ((st = enqueue_stats(acts, T_in, n, bf16, cv.s, cv.q, cv, s))) return st;
+    NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_in, n, alpha_override, d_in, &cv.sc->alpha[0],
+                            &cv.sc->err, s));
+    if ((st = enqueue_stats(grads, T_out, m, bf16, cv.s, cv.q, cv, s))) return st;
+    NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_out, m, alpha_override, d_out, &cv.sc->alpha[1],
+                            &cv.sc->err, s));
+    if (alpha_out) {
+        Scalars h;
+        NQ_CK(cudaMemcpyAsync(&h, cv.sc, sizeof(Scalars), cudaMemcpyDeviceToHost, s));
+        NQ_CK(cudaStreamSynchronize(s));
+        alpha_out[0] = h.alpha[0];
+        alpha_out[1] = h.alpha[1];
+        if (h.err) return static_cast<nq_status>(h.err);
+    }
+    return NQ_OK;
+}
+
+size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r) {
+    if (check_lb_args(m, n, r)) return 0;
+    LbLayout L;
+    L.build(m, n, r);
+    return L.total;
+}
+
+nq_status nq_lbadmm_prepare(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                            const float *d_out, int32_t r, uint64_t seed, double *gamma_out,
+                            void *ws, size_t ws_bytes, nq_stream_t stream) {
+    if (!W || (dt != NQ_F32 && dt != NQ_BF16)) return NQ_ERR_INVALID_ARG;
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    cudaStream_t s = cs(stream);
+    if ((st = lb_prepare(lb, W, dt == NQ_BF16, d_in, d_out, seed, s))) return st;
+    if (gamma_out) {
+        NQ_CK(cudaMemcpyAsync(gamma_out, &lb.sc->gamma, sizeof(double), cudaMemcpyDeviceToHost, s));
+        return read_err(&lb.sc->err, s, false);
+    }
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm_iterate(int64_t m, int64_t n, int32_t r, float rho, float lambda,
+                            int32_t iters, int32_t K, float *objective, void *ws, size_t ws_bytes,
+                            nq_stream_t stream) {
+    if (!(rho > 0.f) || !(lambda >= 0.f) || iters < 1 || K < 1 || !isfinite(rho) ||
+        !isfinite(lambda))
+        return NQ_ERR_INVALID_ARG;
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    cudaStream_t s = cs(stream);
+    if ((st = lb_iterate(lb, rho, lambda, iters, K, objective, s))) return st;
+    if (objective) return read_err(&lb.sc->err, s, false);
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm_half_step(int64_t m, int64_t n, int32_t r, float rho, float lambda, int32_t K,
+                              int32_t side, void *ws, size_t ws_bytes, nq_stream_t stream) {
+    if (!(rho > 0.f) || !(lambda >= 0.f) || K < 1 || (side != 0 && side != 1))
+        return NQ_ERR_INVALID_ARG;
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    return lb_half_step(lb, side, rho, lambda, K, cs(stream));
+}
+
+nq_status nq_lbadmm_finish(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                           const float *d_out, int32_t r, uint32_t *U_packed, uint32_t *V_packed,
+                           float *s1, float *s2, float *final_rel_err, void *ws, size_t ws_bytes,
+                           nq_stream_t stream) {
+    if (!U_packed || !V_packed || !s1 || !s2 || (final_rel_err && !W) ||
+        (dt != NQ_F32 && dt != NQ_BF16))
+        return NQ_ERR_INVALID_ARG;
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    cudaStream_t s = cs(stream);
+    if ((st = lb_finish(lb, W, dt == NQ_BF16, d_in, d_out, U_packed, V_packed, s1, s2,
+                        final_rel_err != nullptr, s)))
+        return st;
+    if (final_rel_err) {
+        double e = 0.0;
+        NQ_CK(cudaMemcpyAsync(&e, &lb.sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
+        st = read_err(&lb.sc->err, s, false);
+        *final_rel_err = (float)e;
+        return st;
+    }
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                    const float *d_out, int32_t r, float rho, float lambda, int32_t iters,
+                    int32_t K, uint64_t seed, uint32_t *U_packed, uint32_t *V_packed, float *s1,
+                    float *s2, float *objective, float *final_rel_err, void *ws,
+                    size_t ws_bytes, nq_stream_t stream) {
+    if (!W || !U_packed || !V_packed || !s1 || !s2 || (dt != NQ_F32 && dt != NQ_BF16) ||
+        !(rho > 0.f) || !(lambda >= 0.f) || iters < 1 || K < 1 || !isfinite(rho) ||
+        !isfinite(lambda))
+        return NQ_ERR_INVALID_ARG;
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    cudaStream_t s = cs(stream);
+    const int bf16 = dt == NQ_BF16;
+    if ((st = lb_prepare(lb, W, bf16, d_in, d_out, seed, s))) return st;
+    if ((st = lb_iterate(lb, rho, lambda, iters, K, objective, s))) return st;
+    if ((st = lb_finish(lb, W, bf16, d_in, d_out, U_packed, V_packed, s1, s2,
+                        final_rel_err != nullptr, s)))
+        return st;
+    if (final_rel_err || objective) {
+        double e = 0.0;
+        NQ_CK(cudaMemcpyAsync(&e, &lb.sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
+        st = read_err(&lb.sc->err, s, false);
+        if (final_rel_err) *final_rel_err = (float)e;
+        return st;
+    }
+    return NQ_OK;
+}
+
+size_t nq_recon_workspace_size(int64_t m, int64_t n, int32_t r) {
+    if (check_lb_args(m, n, r)) return 0;
+    ReconLayout L;
+    L.build(m, n, r);
+    return L.total;
+}
+
+nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                         const float *d_out, const uint32_t *U_packed, const uint32_t *V_packed,
+                         int32_t r, const float *s1, const float *s2, double *rel_err, void *ws,
+                         size_t ws_bytes, nq_stream_t stream) {
+    if (!W || !U_packed || !V_packed || !s1 || !s2 || !rel_err ||
+        (dt != NQ_F32 && dt != NQ_BF16))
+        return NQ_ERR_INVALID_ARG;
+    nq_status st = check_lb_args(m, n, r);
+    if (st) return st;
+    ReconLayout L;
+    L.build(m, n, r);
+    if ((st = check_ws(ws, ws_bytes, L.total))) return st;
+    if ((st = check_device())) return st;
+    cudaStream_t s = cs(stream);
+    Scalars *sc = at<Scalars>(ws, L.scal);
+    double *part = at<double>(ws, L.part);
+    __nv_bfloat16 *up = at<__nv_bfloat16>(ws, L.up), *vp = at<__nv_bfloat16>(ws, L.vp);
+    NQ_CK(cudaMemsetAsync(sc, 0, sizeof(Scalars), s));
+    NQ_CK(unpack_pm(U_packed, m, r, up, L.ldr, s));
+    NQ_CK(unpack_pm(V_packed, n, r, vp, L.ldr, s));
+    NQ_CK(wt_norm_partials(W, dt == NQ_BF16, m, n, d_in, d_out, part, &sc->err, s));
+    NQ_CK(reduce_partials(part, kRedBlocks, &sc->wt_norm2, nullptr, r, s));
+    const int BN = pick_bn(n);
+    tc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!tc::make_map_bf16(&maps.a[0], up, m, r, L.ldr, tc::BM) ||
+        !tc::make_map_bf16(&maps.b[0], vp, n, r, L.ldr, BN))
+        return NQ_ERR_CUDA;
+    tc::EpiParams ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.M = (int)m;
+    ep.N = (int)n;
+    ep.nseg = 1;
+    ep.kblocks[0] = (int)ceil_div(r, tc::BK);
+    ep.err = &sc->err;
+    ep.part = part;
+    ep.W = W;
+    ep.w_bf16 = dt == NQ_BF16;
+    ep.ldw = n;
+    ep.d_in = d_in;
+    ep.d_out = d_out;
+    ep.s1 = s1;
+    ep.s2 = s2;
+    NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RECON, BN, s));
+    NQ_CK(recon_finalize(part, (int)tc::num_tiles((int)m, (int)n, BN), sc, &sc->recon2, s));
+    NQ_CK(cudaMemcpyAsync(rel_err, &sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
+    return read_err(&sc->err, s, false);
+}
+
+nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,
+                        nq_stream_t stream) {
+    if (!X || !bits || rows < 1 || r < 1) return NQ_ERR_INVALID_ARG;
+    nq_status st = check_device();
+    if (st) return st;
+    NQ_CK(pack_signs(X, rows, r, r, bits, cs(stream)));
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, void *ws,
+                                size_t ws_bytes, void **dev_ptr, int64_t *count,
+                                int32_t *elem_bytes, int64_t *ld) {
+    if (!dev_ptr || !count || !elem_bytes || !ld) return NQ_ERR_INVALID_ARG;
+    nq_status st = check_lb_args(m, n, r);
+    if (st) return st;
+    LbLayout L;
+    L.build(m, n, r);
+    if ((st = check_ws(ws, ws_bytes, L.total))) return st;
+    size_t off = 0;
+    int64_t cnt = 0, l = 0;
+    int32_t eb = 4;
+    switch (f) {
+        case NQ_FIELD_U: off = L.x[0]; cnt = m * L.ldr; l = L.ldr; break;
+        case NQ_FIELD_V: off = L.x[1]; cnt = n * L.ldr; l = L.ldr; break;
+        case NQ_FIELD_SU: off = L.s[0]; cnt = m * L.ldr; l = L.ldr; break;
+        case NQ_FIELD_SV: off = L.s[1]; cnt = n * L.ldr; l = L.ldr; break;
+        case NQ_FIELD_AU: off = L.a[0]; cnt = m; l = 1; break;
+        case NQ_FIELD_AV: off = L.a[1]; cnt = n; l = 1; break;
+        case NQ_FIELD_BU: off = L.b[0]; cnt = r; l = 1; break;
+        case NQ_FIELD_BV: off = L.b[1]; cnt = r; l = 1; break;
+        case NQ_FIELD_WHAT: off = L.what; cnt = m * L.ldn; l = L.ldn; eb = 2; break;
+        case NQ_FIELD_GAMMA: off = L.scal + offsetof(Scalars, gamma); cnt = 1; l = 1; eb = 8; break;
+        default: return NQ_ERR_INVALID_ARG;
+    }
+    *dev_ptr = static_cast<char *>(ws) + off;
+    *count = cnt;
+    *elem_bytes = eb;
+    *ld = l;
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
+                                  nq_stream_t stream) {
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    cudaStream_t s = cs(stream);
+    const LbLayout &L = lb.L;
+    NQ_CK(transpose_to_bf16(lb.p<float>(L.x[0]), L.m, L.r, L.ldr, lb.p<__nv_bfloat16>(L.xt[0]),
+                            L.ldm, s));
+    NQ_CK(transpose_to_bf16(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, lb.p<__nv_bfloat16>(L.xt[1]),
+                            L.ldn, s));
+    NQ_CK(transpose_bf16(lb.p<__nv_bfloat16>(L.what), L.m, L.n, L.ldn,
+                         lb.p<__nv_bfloat16>(L.whatT), L.ldm, s));
+    return NQ_OK;
+}
+
+nq_status nq_lbadmm_check(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
+                          nq_stream_t stream) {
+    Lb lb;
+    nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
+    if (st) return st;
+    return read_err(&lb.sc->err, cs(stream), true);
+}
+
+}  // extern "C"

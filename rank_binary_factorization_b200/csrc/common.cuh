@@ -1,0 +1,75 @@
+// Shared device/host helpers of the sm_100a NanoQuant library.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nq.h"
+
+#define NQ_HD __host__ __device__ __forceinline__
+
+namespace nq {
+
+constexpr int kNumSMsB200 = 148;
+
+NQ_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+NQ_HD int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Device error word: the first non-OK status raised on the device wins.
+__device__ __forceinline__ void raise_error(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+// Spin budgets for every device-side wait.  A wait that runs out raises
+// NQ_ERR_TIMEOUT on the workspace's error word and returns instead of hanging.
+constexpr uint32_t kMbarSpinLimit = 1u << 26;   // polls of mbarrier.try_wait (each may suspend)
+constexpr uint32_t kGridSpinLimit = 1u << 24;   // polls of a grid-barrier flag (~50 ns apart)
+
+__device__ __forceinline__ float bf16_round(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// Warp-level sum.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Grid-wide barrier for kernels launched cooperatively (all CTAs co-resident).
+// ``bar`` points at two words: [0] arrival count, [1] generation.  Bounded: a
+// barrier that does not complete within the spin budget raises NQ_ERR_TIMEOUT and
+// lets the CTA continue (results are then garbage but nothing hangs).
+__device__ __forceinline__ void grid_barrier(unsigned int *bar, int *err) {
+    __syncthreads();
+    // after a timeout every later barrier is skipped, so at most one budget is spent
+    if (threadIdx.x == 0 && !(err && *(volatile int *)err == NQ_ERR_TIMEOUT)) {
+        volatile unsigned int *vgen = bar + 1;
+        unsigned int gen = *vgen;
+        __threadfence();
+        unsigned int arrived = atomicAdd(bar, 1u) + 1u;
+        if (arrived == gridDim.x * gridDim.y * gridDim.z) {
+            atomicExch(bar, 0u);
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            uint32_t spins = 0;
+            while (*vgen == gen) {
+                if (++spins > kGridSpinLimit) {
+                    raise_error(err, NQ_ERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+}  // namespace nq

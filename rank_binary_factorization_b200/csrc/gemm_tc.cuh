@@ -1,0 +1,76 @@
+// tcgen05 / TMEM / TMA GEMM for sm_100a with fused LB-ADMM epilogues.
+//
+// D[M x N] = sum over K-segments s of A_s[M x K_s] . B_s[N x K_s]^T, all operands BF16
+// and K-major (row-major with K contiguous), accumulation FP32 in tensor memory.
+// One CTA computes one 128 x BN tile:
+//   warp 0     one elected thread issues TMA tile loads into a STAGES-deep ring
+//   warp 1     allocates TMEM; one elected thread issues tcgen05.mma (M=128, N=BN,
+//              K=16 per instruction, 4 per 64-wide K block) and commits to mbarriers
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes
+//              32*(w%4) .. +31, i.e. those tile rows), fused element-wise work, stores
+// Every mbarrier wait is bounded; a wait that runs out raises NQ_ERR_TIMEOUT.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace nq {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 bf16 = 128 B = one 128B-swizzle atom row
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3 };
+
+struct Maps {
+    CUtensorMap a[3];
+    CUtensorMap b[3];
+};
+
+struct EpiParams {
+    int M, N;
+    int nseg;
+    int kblocks[3];
+    int *err;
+    // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
+    float *out;
+    int64_t ldo;
+    float diag;
+    // EPI_RHS / EPI_SOLVE: dual state of the side being updated
+    float *S;            // [M][ldf]
+    const float *a;      // [M]
+    const float *b;      // [N]
+    int64_t ldf;
+    float rho;
+    // EPI_RHS: R = acc + rho (2 sign(S) a b^T - S) split into hi + lo bf16
+    __nv_bfloat16 *Rhi, *Rlo;  // [M][ldr]
+    int64_t ldr;
+    // EPI_SOLVE: X = acc; S <- X + S - sign(S) a b^T; Xt[col][row] = bf16(X)
+    float *X;                  // [M][ldf]
+    __nv_bfloat16 *Xt;         // [N][ldxt]
+    int64_t ldxt;
+    int objective;             // also sum (R - rho (2Z - S_old)) . X into part[tile]
+    double *part;              // per-tile partial sums (EPI_SOLVE objective, EPI_RECON)
+    // EPI_RECON: sum_ij (d_out_i W_ij d_in_j - s1_i acc s2_j)^2
+    const void *W;
+    int w_bf16;
+    int64_t ldw;
+    const float *d_in, *d_out, *s1, *s2;
+};
+
+// Host: encode a 2-D BF16 tensor map over rows x cols (row stride ld elements) with
+// a box of 64 x box_rows and 128-byte swizzle.  Returns false on failure.
+bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                   int box_rows);
+
+// Host: launch one GEMM.  BN in {64, 128, 256}.
+cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, cudaStream_t s);
+
+// Host: number of output tiles of a launch (size of the per-tile partial array).
+inline int64_t num_tiles(int M, int N, int BN) { return ceil_div(M, BM) * ceil_div(N, BN); }
+
+}  // namespace tc
+}  // namespace nq

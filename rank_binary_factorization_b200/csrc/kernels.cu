@@ -1,0 +1,993 @@
+// SIMT kernels of the NanoQuant hot path (sm_100a): calibration reduction, target
+// preparation, V_0, blocked Cholesky + inverse, SVID power passes, objective,
+// balancing / scale extraction / sign packing.
+#include <cooperative_groups.h>
+
+#include "kernels.cuh"
+
+namespace nq {
+
+// =================================================================================
+// Calibration statistics.  NanoQuant summary page, "Method steps" (方法步骤详情),
+// stage one: per-channel statistics over the calibration tokens.
+// =================================================================================
+template <bool BF16>
+__device__ __forceinline__ void unpack16(const uint4 &raw, float (&x)[BF16 ? 8 : 4]) {
+    if constexpr (BF16) {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(h[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    } else {
+        x[0] = __uint_as_float(raw.x);
+        x[1] = __uint_as_float(raw.y);
+        x[2] = __uint_as_float(raw.z);
+        x[3] = __uint_as_float(raw.w);
+    }
+}
+
+// CTA = 8 warps over one slab of 32*VEC channels; warp w takes tokens w, w+8, ...
+// of the CTA's token slab; each lane owns VEC consecutive channels (one 16-byte load
+// per token).  FP32 sums over 16 tokens are flushed into FP64 accumulators.
+template <bool BF16>
+__global__ void __launch_bounds__(256) calib_partial_vec(const void *__restrict__ Xv, int64_t T,
+                                                         int64_t C, int64_t tok_per_slab,
+                                                         double *__restrict__ ps,
+                                                         double *__restrict__ pq) {
+    constexpr int VEC = BF16 ? 8 : 4;
+    constexpr int ESZ = BF16 ? 2 : 4;
+    __shared__ double sh_s[8][32 * VEC];
+    __shared__ double sh_q[8][32 * VEC];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t cbase = (int64_t)blockIdx.x * 32 * VEC;
+    const int64_t c0 = cbase + lane * VEC;
+    const int64_t t_begin = (int64_t)blockIdx.y * tok_per_slab;
+    const int64_t t_end = min(T, t_begin + tok_per_slab);
+    double ds[VEC], dq[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) ds[v] = dq[v] = 0.0;
+    if (c0 < C) {
+        const char *base = reinterpret_cast<const char *>(Xv) + c0 * ESZ;
+        const int64_t row_bytes = C * ESZ;
+        int64_t t = t_begin + warp;
+        while (t < t_end) {
+            float fs[VEC], fq[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) fs[v] = fq[v] = 0.f;
+            int cnt = 0;
+            for (; t + 24 < t_end && cnt < 16; t += 32, cnt += 4) {
+                uint4 raw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    raw[u] = __ldcs(reinterpret_cast<const uint4 *>(base + (t + 8 * u) * row_bytes));
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float x[VEC];
+                    unpack16<BF16>(raw[u], x);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        const float x2 = x[v] * x[v];
+                        fs[v] += x2;
+                        fq[v] = fmaf(x2, x2, fq[v]);
+                    }
+                }
+            }
+            for (; t < t_end && cnt < 16; t += 8, ++cnt) {
+                float x[VEC];
+                unpack16<BF16>(__ldcs(reinterpret_cast<const uint4 *>(base + t * row_bytes)), x);
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    const float x2 = x[v] * x[v];
+                    fs[v] += x2;
+                    fq[v] = fmaf(x2, x2, fq[v]);
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                ds[v] += fs[v];
+                dq[v] += fq[v];
+            }
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        sh_s[warp][lane * VEC + v] = ds[v];
+        sh_q[warp][lane * VEC + v] = dq[v];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < 32 * VEC; c += blockDim.x) {
+        if (cbase + c >= C) continue;
+        double a = 0.0, b = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            a += sh_s[w][c];
+            b += sh_q[w][c];
+        }
+        ps[(int64_t)blockIdx.y * C + cbase + c] = a;
+        pq[(int64_t)blockIdx.y * C + cbase + c] = b;
+    }
+}
+
+// Scalar path (C not a multiple of the vector width): thread per channel.
+template <bool BF16>
+__global__ void __launch_bounds__(256) calib_partial_scalar(const void *__restrict__ Xv, int64_t T,
+                                                            int64_t C, int64_t tok_per_slab,
+                                                            double *__restrict__ ps,
+                                                            double *__restrict__ pq) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    const int64_t t_begin = (int64_t)blockIdx.y * tok_per_slab;
+    const int64_t t_end = min(T, t_begin + tok_per_slab);
+    double ds = 0.0, dq = 0.0;
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += 16) {
+        float fs = 0.f, fq = 0.f;
+        const int64_t t1 = min(t_end, t0 + 16);
+        for (int64_t t = t0; t < t1; ++t) {
+            float x;
+            if constexpr (BF16)
+                x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(Xv)[t * C + c]);
+            else
+                x = reinterpret_cast<const float *>(Xv)[t * C + c];
+            const float x2 = x * x;
+            fs += x2;
+            fq = fmaf(x2, x2, fq);
+        }
+        ds += fs;
+        dq += fq;
+    }
+    ps[(int64_t)blockIdx.y * C + c] = ds;
+    pq[(int64_t)blockIdx.y * C + c] = dq;
+}
+
+int calib_num_slabs(int64_t T, int64_t C) {
+    const int64_t cx = ceil_div(C, 256);
+    int64_t ns = ceil_div(6 * kNumSMsB200, cx);
+    const int64_t max_by_T = ceil_div(T, 256);
+    if (ns > max_by_T) ns = max_by_T;
+    if (ns < 1) ns = 1;
+    if (ns > 4096) ns = 4096;
+    return (int)ns;
+}
+
+cudaError_t calib_partials(const void *X, int64_t T, int64_t C, int dt_bf16, int nslab,
+                           double *ps, double *pq, cudaStream_t s) {
+    const int64_t tps = ceil_div(T, nslab);
+    const int vec = dt_bf16 ? 8 : 4;
+    const bool aligned = (reinterpret_cast<uintptr_t>(X) % 16 == 0) && (C % vec == 0);
+    if (aligned) {
+        dim3 grid((unsigned)ceil_div(C, 32 * vec), (unsigned)nslab);
+        if (dt_bf16)
+            calib_partial_vec<true><<<grid, 256, 0, s>>>(X, T, C, tps, ps, pq);
+        else
+            calib_partial_vec<false><<<grid, 256, 0, s>>>(X, T, C, tps, ps, pq);
+    } else {
+        dim3 grid((unsigned)ceil_div(C, 256), (unsigned)nslab);
+        if (dt_bf16)
+            calib_partial_scalar<true><<<grid, 256, 0, s>>>(X, T, C, tps, ps, pq);
+        else
+            calib_partial_scalar<false><<<grid, 256, 0, s>>>(X, T, C, tps, ps, pq);
+    }
+    return cudaGetLastError();
+}
+
+__global__ void calib_moments_kernel(const double *__restrict__ ps, const double *__restrict__ pq,
+                                     int nslab, int64_t T, int64_t C, double *s_out,
+                                     double *q_out) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= C) return;
+    double a = 0.0, b = 0.0;
+    for (int k = 0; k < nslab; ++k) {
+        a += ps[(int64_t)k * C + c];
+        b += pq[(int64_t)k * C + c];
+    }
+    s_out[c] = a / (double)T;
+    q_out[c] = b / (double)T;
+}
+
+cudaError_t calib_moments(const double *ps, const double *pq, int nslab, int64_t T, int64_t C,
+                          double *s_out, double *q_out, cudaStream_t st) {
+    calib_moments_kernel<<<(unsigned)ceil_div(C, 256), 256, 0, st>>>(ps, pq, nslab, T, C, s_out,
+                                                                     q_out);
+    return cudaGetLastError();
+}
+
+// Deterministic block sum (fixed order) of one double per thread; blockDim = 1024.
+__device__ double block_sum_1024(double v, double *sh) {
+    sh[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 512; o > 0; o >>= 1) {
+        if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+        __syncthreads();
+    }
+    const double r = sh[0];
+    __syncthreads();
+    return r;
+}
+
+// Ledoit-Wolf 2004 with target mu I restricted to the diagonal (see nq_calib_precond).
+__global__ void __launch_bounds__(1024)
+    calib_lw_kernel(const double *__restrict__ s, const double *__restrict__ q, int64_t T,
+                    int64_t C, double alpha_override, float *d, double *alpha_out, int *err) {
+    __shared__ double sh[1024];
+    double a = 0.0;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) a += s[c];
+    const double sum_s = block_sum_1024(a, sh);
+    const double mu = sum_s / (double)C;
+    double dd = 0.0, bb = 0.0;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
+        const double e = s[c] - mu;
+        dd += e * e;
+        bb += q[c] - s[c] * s[c];
+    }
+    const double delta2 = block_sum_1024(dd, sh);
+    const double beta_bar2 = block_sum_1024(bb, sh) / (double)T;
+    if (!isfinite(sum_s) || !isfinite(beta_bar2)) {
+        if (threadIdx.x == 0) raise_error(err, NQ_ERR_NONFINITE);
+    }
+    double alpha;
+    if (alpha_override >= 0.0)
+        alpha = alpha_override;
+    else
+        alpha = delta2 == 0.0 ? 1.0 : fmin(beta_bar2, delta2) / delta2;
+    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
+        double dt = (1.0 - alpha) * s[c] + alpha * mu;
+        dt = fmax(dt, 1e-12 * mu);
+        d[c] = (float)sqrt(dt);
+    }
+    if (threadIdx.x == 0 && alpha_out) *alpha_out = alpha;
+}
+
+cudaError_t calib_ledoit_wolf(const double *s, const double *q, int64_t T, int64_t C,
+                              double alpha_override, float *d, double *alpha, int *err,
+                              cudaStream_t st) {
+    calib_lw_kernel<<<1, 1024, 0, st>>>(s, q, T, C, alpha_override, d, alpha, err);
+    return cudaGetLastError();
+}
+
+// =================================================================================
+// Preconditioned, normalised target.  Same page, "Method steps", stage two:
+// W~ = D_out W D_in.
+// =================================================================================
+__device__ __forceinline__ float load_wf(const void *W, int w_bf16, int64_t idx) {
+    return w_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(W)[idx])
+                  : reinterpret_cast<const float *>(W)[idx];
+}
+
+__device__ double block_sum_256(double v, double *sh) {
+    sh[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if (threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+        __syncthreads();
+    }
+    const double r = sh[0];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(256)
+    wt_norm_kernel(const void *__restrict__ W, int w_bf16, int64_t m, int64_t n,
+                   const float *__restrict__ d_in, const float *__restrict__ d_out, double *part,
+                   int *err) {
+    __shared__ double sh[256];
+    double acc = 0.0;
+    bool bad = false;
+    for (int64_t i = blockIdx.x; i < m; i += gridDim.x) {
+        const float dro = d_out ? d_out[i] : 1.f;
+        float f = 0.f;
+        for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
+            const float w = dro * load_wf(W, w_bf16, i * n + j) * (d_in ? d_in[j] : 1.f);
+            bad |= !isfinite(w);
+            f = fmaf(w, w, f);
+        }
+        acc += f;
+    }
+    if (bad) raise_error(err, NQ_ERR_NONFINITE);
+    const double t = block_sum_256(acc, sh);
+    if (threadIdx.x == 0) part[blockIdx.x] = t;
+}
+
+cudaError_t wt_norm_partials(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
+                             const float *d_out, double *part, int *err, cudaStream_t s) {
+    wt_norm_kernel<<<kRedBlocks, 256, 0, s>>>(W, w_bf16, m, n, d_in, d_out, part, err);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    reduce_partials_kernel(const double *part, int count, double *sum, double *gamma, int r) {
+    __shared__ double sh[256];
+    double a = 0.0;
+    for (int i = threadIdx.x; i < count; i += blockDim.x) a += part[i];
+    const double t = block_sum_256(a, sh);
+    if (threadIdx.x == 0) {
+        if (sum) *sum = t;
+        if (gamma) *gamma = sqrt(t) / (2.0 * sqrt((double)r));
+    }
+}
+
+cudaError_t reduce_partials(const double *part, int count, double *sum, double *gamma, int r,
+                            cudaStream_t s) {
+    reduce_partials_kernel<<<1, 256, 0, s>>>(part, count, sum, gamma, r);
+    return cudaGetLastError();
+}
+
+// 32 x 32 tiles, grid-stride over all tiles of the padded (ldm x ldn) index space.
+__global__ void __launch_bounds__(256)
+    what_cast_kernel(const void *__restrict__ W, int w_bf16, int64_t m, int64_t n,
+                     const float *__restrict__ d_in, const float *__restrict__ d_out,
+                     const double *__restrict__ gamma, __nv_bfloat16 *What, int64_t ldn,
+                     __nv_bfloat16 *WhatT, int64_t ldm, double *part) {
+    __shared__ __nv_bfloat16 tile[32][34];
+    __shared__ double sh[256];
+    const double g = *gamma;
+    const float inv = g > 0.0 ? (float)(1.0 / g) : 0.f;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const int64_t ntx = ceil_div(ldn, 32), nty = ceil_div(ldm, 32);
+    double acc = 0.0;
+    for (int64_t t = blockIdx.x; t < ntx * nty; t += gridDim.x) {
+        const int64_t i0 = (t / ntx) * 32, j0 = (t % ntx) * 32;
+        float f = 0.f;
+        for (int k = ty; k < 32; k += 8) {
+            const int64_t i = i0 + k, j = j0 + tx;
+            __nv_bfloat16 h = __float2bfloat16_rn(0.f);
+            if (i < m && j < n) {
+                const float w = (d_out ? d_out[i] : 1.f) * load_wf(W, w_bf16, i * n + j) *
+                                (d_in ? d_in[j] : 1.f);
+                h = __float2bfloat16_rn(w * inv);
+                const float hv = __bfloat162float(h);
+                f = fmaf(hv, hv, f);
+            }
+            if (i < m && j < ldn) What[i * ldn + j] = h;
+            tile[k][tx] = h;
+        }
+        acc += f;
+        __syncthreads();
+        for (int k = ty; k < 32; k += 8) {
+            const int64_t j = j0 + k, i = i0 + tx;
+            if (j < n && i < ldm) WhatT[j * ldm + i] = tile[tx][k];
+        }
+        __syncthreads();
+    }
+    const double s = block_sum_256(acc, sh);
+    if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+
+cudaError_t what_cast(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
+                      const float *d_out, const double *gamma, __nv_bfloat16 *What, int64_t ldn,
+                      __nv_bfloat16 *WhatT, int64_t ldm, double *part, cudaStream_t s) {
+    what_cast_kernel<<<kRedBlocks, 256, 0, s>>>(W, w_bf16, m, n, d_in, d_out, gamma, What, ldn,
+                                                WhatT, ldm, part);
+    return cudaGetLastError();
+}
+
+// SplitMix64 (Steele, Lea, Flood 2014), evaluated as a function of a counter.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t idx) {
+    uint64_t z = seed + (idx + 1ull) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__global__ void init_v0_kernel(int64_t n, int32_t r, uint64_t seed, float c, float *X,
+                               int64_t ldr, __nv_bfloat16 *Xt, int64_t ldn) {
+    const int64_t total = n * (int64_t)r;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        // row-major pass over X (k fastest)
+        const int64_t j = e / r, k = e % r;
+        const float v = (splitmix64(seed, (uint64_t)e) >> 63) ? -c : c;
+        X[j * ldr + k] = v;
+        // column-major pass over Xt (j fastest): element (k2, j2)
+        const int64_t k2 = e / n, j2 = e % n;
+        const float v2 = (splitmix64(seed, (uint64_t)(j2 * r + k2)) >> 63) ? -c : c;
+        Xt[k2 * ldn + j2] = __float2bfloat16_rn(v2);
+    }
+}
+
+cudaError_t init_v0(int64_t n, int32_t r, uint64_t seed, float *X, int64_t ldr,
+                    __nv_bfloat16 *Xt, int64_t ldn, cudaStream_t s) {
+    const float c = sqrtf(2.0f / (float)n);
+    init_v0_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(n, r, seed, c, X, ldr, Xt, ldn);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    transpose_to_bf16_kernel(const float *__restrict__ X, int64_t rows, int32_t r, int64_t ldx,
+                             __nv_bfloat16 *Xt, int64_t ldt) {
+    __shared__ float tile[32][33];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int64_t i0 = (int64_t)blockIdx.y * 32, k0 = (int64_t)blockIdx.x * 32;
+    for (int a = ty; a < 32; a += 8) {
+        const int64_t i = i0 + a, k = k0 + tx;
+        tile[a][tx] = (i < rows && k < r) ? X[i * ldx + k] : 0.f;
+    }
+    __syncthreads();
+    for (int a = ty; a < 32; a += 8) {
+        const int64_t k = k0 + a, i = i0 + tx;
+        if (k < r && i < rows) Xt[k * ldt + i] = __float2bfloat16_rn(tile[tx][a]);
+    }
+}
+
+cudaError_t transpose_to_bf16(const float *X, int64_t rows, int32_t r, int64_t ldx,
+                              __nv_bfloat16 *Xt, int64_t ldt, cudaStream_t s) {
+    dim3 grid((unsigned)ceil_div(r, 32), (unsigned)ceil_div(rows, 32));
+    transpose_to_bf16_kernel<<<grid, 256, 0, s>>>(X, rows, r, ldx, Xt, ldt);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ A, int64_t rows, int64_t cols,
+                          int64_t lda, __nv_bfloat16 *B, int64_t ldb) {
+    __shared__ __nv_bfloat16 tile[32][34];
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int64_t i0 = (int64_t)blockIdx.y * 32, j0 = (int64_t)blockIdx.x * 32;
+    for (int a = ty; a < 32; a += 8) {
+        const int64_t i = i0 + a, j = j0 + tx;
+        tile[a][tx] = (i < rows && j < cols) ? A[i * lda + j] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int a = ty; a < 32; a += 8) {
+        const int64_t j = j0 + a, i = i0 + tx;
+        if (j < cols && i < rows) B[j * ldb + i] = tile[tx][a];
+    }
+}
+
+cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, int64_t lda,
+                           __nv_bfloat16 *B, int64_t ldb, cudaStream_t s) {
+    dim3 grid((unsigned)ceil_div(cols, 32), (unsigned)ceil_div(rows, 32));
+    transpose_bf16_kernel<<<grid, 256, 0, s>>>(A, rows, cols, lda, B, ldb);
+    return cudaGetLastError();
+}
+
+// =================================================================================
+// Cholesky G = L L^T and G^-1 = L^-T L^-1 (FP32, 32 x 32 tiles, one cooperative
+// launch with bounded grid barriers).  Same page, "Core method" (核心方法), step (a):
+// the regularised linear system of the U (V) step is solved through a Cholesky
+// factorisation.
+// =================================================================================
+constexpr int CT = 32;
+
+struct CholArgs {
+    const float *G;
+    int r;
+    int64_t rp;
+    float *A;
+    float *Li;
+    __nv_bfloat16 *hi, *lo;
+    int64_t ldr;
+    int *err;
+    unsigned int *bar;
+};
+
+__device__ __forceinline__ void load_tile(float (*dst)[CT + 1], const float *M, int64_t ld,
+                                          int ti, int tj) {
+    for (int e = threadIdx.x; e < CT * CT; e += blockDim.x) {
+        const int i = e >> 5, j = e & 31;
+        // L2-coherent load: tiles are rewritten by other CTAs between grid barriers
+        dst[i][j] = __ldcg(M + ((int64_t)ti * CT + i) * ld + (int64_t)tj * CT + j);
+    }
+}
+__device__ __forceinline__ void store_tile(float *M, int64_t ld, int ti, int tj,
+                                           const float (*src)[CT + 1]) {
+    for (int e = threadIdx.x; e < CT * CT; e += blockDim.x) {
+        const int i = e >> 5, j = e & 31;
+        M[((int64_t)ti * CT + i) * ld + (int64_t)tj * CT + j] = src[i][j];
+    }
+}
+
+// acc[q] += sum_c X(a, c) Y(c, b0+q) with X(a,c) = TX ? X[c][a] : X[a][c] and
+// Y(c,b) = TY ? Y[b][c] : Y[c][b]; thread owns row a = tid/8, columns b0 = 4*(tid%8).
+template <bool TX, bool TY>
+__device__ __forceinline__ void tile_mac(float (&acc)[4], const float (*X)[CT + 1],
+                                         const float (*Y)[CT + 1], int c_begin = 0,
+                                         int c_end = CT) {
+    const int a = threadIdx.x >> 3, b0 = (threadIdx.x & 7) * 4;
+    for (int c = c_begin; c < c_end; ++c) {
+        const float x = TX ? X[c][a] : X[a][c];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = fmaf(x, TY ? Y[b0 + q][c] : Y[c][b0 + q], acc[q]);
+    }
+}
+
+__global__ void __launch_bounds__(256) chol_inv_kernel(CholArgs p) {
+    __shared__ float t0[CT][CT + 1], t1[CT][CT + 1], t2[CT][CT + 1];
+    const int nb = (int)(p.rp / CT);
+    const int64_t rp = p.rp;
+    const int a_row = threadIdx.x >> 3, b_col = (threadIdx.x & 7) * 4;
+
+    // phase 0: A = G padded with the identity, Li = 0
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rp * rp;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / rp, j = e % rp;
+        p.A[e] = (i < p.r && j < p.r) ? p.G[i * p.r + j] : (i == j ? 1.f : 0.f);
+        p.Li[e] = 0.f;
+    }
+    grid_barrier(p.bar, p.err);
+
+    for (int j = 0; j < nb; ++j) {
+        // (a) diagonal tile: L_jj (lower) and its inverse, by CTA 0 / warp 0
+        if (blockIdx.x == 0) {
+            load_tile(t0, p.A, rp, j, j);
+            __syncthreads();
+            if (threadIdx.x < 32) {
+                const int lane = threadIdx.x;
+                for (int k = 0; k < CT; ++k) {
+                    __syncwarp();
+                    float piv = t0[k][k];
+                    if (!(piv > 0.f)) {
+                        if (lane == 0) raise_error(p.err, NQ_ERR_NOT_SPD);
+                        piv = 1e-30f;
+                    }
+                    const float l = sqrtf(piv);
+                    __syncwarp();
+                    if (lane == k) t0[k][k] = l;
+                    if (lane > k) t0[lane][k] /= l;
+                    __syncwarp();
+                    if (lane > k) {
+                        const float lik = t0[lane][k];
+                        for (int jj = k + 1; jj <= lane; ++jj) t0[lane][jj] -= lik * t0[jj][k];
+                    }
+                }
+                __syncwarp();
+                // column ``lane`` of L_jj^-1 by forward substitution
+                for (int i = 0; i < CT; ++i) t1[i][lane] = 0.f;
+                t1[lane][lane] = 1.f / t0[lane][lane];
+                for (int i = lane + 1; i < CT; ++i) {
+                    float s = 0.f;
+                    for (int k = lane; k < i; ++k) s = fmaf(t0[i][k], t1[k][lane], s);
+                    t1[i][lane] = -s / t0[i][i];
+                }
+                __syncwarp();
+                for (int i = 0; i < CT; ++i)
+                    if (lane > i) t0[i][lane] = 0.f;  // clear the strict upper triangle
+            }
+            __syncthreads();
+            store_tile(p.A, rp, j, j, t0);
+            store_tile(p.Li, rp, j, j, t1);
+        }
+        grid_barrier(p.bar, p.err);
+
+        // (b) panel: L_ij = A_ij L_jj^-T
+        for (int i = j + 1 + blockIdx.x; i < nb; i += gridDim.x) {
+            load_tile(t0, p.A, rp, i, j);
+            load_tile(t1, p.Li, rp, j, j);
+            __syncthreads();
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            tile_mac<false, true>(acc, t0, t1);
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) t2[a_row][b_col + q] = acc[q];
+            __syncthreads();
+            store_tile(p.A, rp, i, j, t2);
+            __syncthreads();
+        }
+        grid_barrier(p.bar, p.err);
+
+        // (c) trailing update: A_ik -= L_ij L_kj^T for j < k <= i
+        const int T = nb - 1 - j;
+        const int64_t ntl = (int64_t)T * (T + 1) / 2;
+        for (int64_t idx = blockIdx.x; idx < ntl; idx += gridDim.x) {
+            // lower-triangular enumeration: ii >= kk
+            int ii = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
+            while ((int64_t)(ii + 1) * (ii + 2) / 2 <= idx) ++ii;
+            while ((int64_t)ii * (ii + 1) / 2 > idx) --ii;
+            const int kk = (int)(idx - (int64_t)ii * (ii + 1) / 2);
+            const int i = j + 1 + ii, k = j + 1 + kk;
+            load_tile(t0, p.A, rp, i, j);
+            load_tile(t1, p.A, rp, k, j);
+            load_tile(t2, p.A, rp, i, k);
+            __syncthreads();
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            tile_mac<false, true>(acc, t0, t1);
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) t2[a_row][b_col + q] -= acc[q];
+            __syncthreads();
+            store_tile(p.A, rp, i, k, t2);
+            __syncthreads();
+        }
+        grid_barrier(p.bar, p.err);
+    }
+
+    // Inverse of L by recursive doubling over tile blocks: for a pair of diagonal
+    // blocks [[L11, 0], [L21, L22]] with known inverses, (L^-1)_21 = -L22^-1 L21 L11^-1.
+    // T = L21 L11^-1 is kept, tile (a, b), in the unused upper tile (b, a) of Li.
+    for (int s = 1; s < nb; s *= 2) {
+        const int npairs = (int)ceil_div(nb, 2 * s);
+        // step 1: T(a, b) = sum_{c >= b} L21(a, c) Li11(c, b)
+        {
+            int64_t jobs = (int64_t)npairs * s * s;
+            for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
+                const int pr = (int)(q / (s * s));
+                const int a = 2 * pr * s + s + (int)((q % (s * s)) / s);
+                const int b = 2 * pr * s + (int)(q % s);
+                const int top_end = 2 * pr * s + s;
+                if (a >= nb) continue;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int c = b; c < top_end; ++c) {
+                    load_tile(t0, p.A, rp, a, c);
+                    load_tile(t1, p.Li, rp, c, b);
+                    __syncthreads();
+                    tile_mac<false, false>(acc, t0, t1);
+                    __syncthreads();
+                }
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) t2[a_row][b_col + qq] = acc[qq];
+                __syncthreads();
+                store_tile(p.Li, rp, b, a, t2);
+                __syncthreads();
+            }
+        }
+        grid_barrier(p.bar, p.err);
+        // step 2: Li21(a, b) = -sum_{bot0 <= c <= a} Li22(a, c) T(c, b)
+        {
+            int64_t jobs = (int64_t)npairs * s * s;
+            for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
+                const int pr = (int)(q / (s * s));
+                const int bot0 = 2 * pr * s + s;
+                const int a = bot0 + (int)((q % (s * s)) / s);
+                const int b = 2 * pr * s + (int)(q % s);
+                if (a >= nb) continue;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int c = bot0; c <= a; ++c) {
+                    load_tile(t0, p.Li, rp, a, c);
+                    load_tile(t1, p.Li, rp, b, c);  // T(c, b) lives at tile (b, c)
+                    __syncthreads();
+                    tile_mac<false, false>(acc, t0, t1);
+                    __syncthreads();
+                }
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) t2[a_row][b_col + qq] = -acc[qq];
+                __syncthreads();
+                store_tile(p.Li, rp, a, b, t2);
+                __syncthreads();
+            }
+        }
+        grid_barrier(p.bar, p.err);
+    }
+
+    // G^-1 = Li^T Li: tile (a, b), a >= b: sum_{c >= a} Li(c, a)^T Li(c, b); split into
+    // bf16 hi + lo and written to both (a, b) and (b, a).
+    const int64_t ngi = (int64_t)nb * (nb + 1) / 2;
+    for (int64_t idx = blockIdx.x; idx < ngi; idx += gridDim.x) {
+        int a = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
+        while ((int64_t)(a + 1) * (a + 2) / 2 <= idx) ++a;
+        while ((int64_t)a * (a + 1) / 2 > idx) --a;
+        const int b = (int)(idx - (int64_t)a * (a + 1) / 2);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = a; c < nb; ++c) {
+            load_tile(t0, p.Li, rp, c, a);
+            load_tile(t1, p.Li, rp, c, b);
+            __syncthreads();
+            tile_mac<true, false>(acc, t0, t1);
+            __syncthreads();
+        }
+        const int64_t gi = (int64_t)a * CT + a_row;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t gj = (int64_t)b * CT + b_col + q;
+            if (gi < p.r && gj < p.r) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(acc[q]);
+                const __nv_bfloat16 l = __float2bfloat16_rn(acc[q] - __bfloat162float(h));
+                p.hi[gi * p.ldr + gj] = h;
+                p.lo[gi * p.ldr + gj] = l;
+                p.hi[gj * p.ldr + gi] = h;
+                p.lo[gj * p.ldr + gi] = l;
+            }
+        }
+    }
+}
+
+cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
+                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr, int *err,
+                         unsigned int *bar, cudaStream_t s) {
+    static int grid = 0;
+    if (!grid) {
+        int per_sm = 0;
+        cudaError_t e =
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chol_inv_kernel, 256, 0);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        grid = sms * (per_sm < 2 ? per_sm : 2);
+        if (grid < 1) return cudaErrorLaunchOutOfResources;
+    }
+    cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
+    if (e != cudaSuccess) return e;
+    CholArgs args{G, r, rp, A, Li, Gi_hi, Gi_lo, ldr, err, bar};
+    void *params[] = {&args};
+    return cudaLaunchCooperativeKernel((const void *)chol_inv_kernel, dim3(grid), dim3(256),
+                                       params, 0, s);
+}
+
+// =================================================================================
+// SVID power steps.  Same page, "Core method", step (b): the continuous U is mapped
+// to the binary proxy Z = sign(S) * a b^T, a b^T the rank-1 fit of |S| by K power
+// steps from b = 1.  One pass over S per power step: t = |S| b row by row and
+// b' = |S|^T t / ||t|| column by column, from the same shared-memory copy of S.
+// =================================================================================
+__global__ void __launch_bounds__(256)
+    svid_pass_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
+                     const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
+                     double *partn) {
+    extern __shared__ float sm[];
+    float *sA = sm;                      // kSvidRows x r
+    float *sb = sm + kSvidRows * r;      // r
+    __shared__ float st[kSvidRows];
+    __shared__ double sn[kSvidRows];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int k = threadIdx.x; k < r; k += blockDim.x) sb[k] = b_in ? b_in[k] : 1.f;
+    float acc[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+    double nacc = 0.0;
+    const int64_t ntile = ceil_div(rows, kSvidRows);
+    for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+        const int64_t row0 = tile * kSvidRows;
+        __syncthreads();
+        for (int w = 0; w < kSvidRows; ++w) {
+            const int64_t i = row0 + w;
+            for (int k = threadIdx.x; k < r; k += blockDim.x)
+                sA[w * r + k] = i < rows ? fabsf(S[i * ldf + k]) : 0.f;
+        }
+        __syncthreads();
+        if (warp < kSvidRows) {
+            float t = 0.f;
+            for (int k = lane; k < r; k += 32) t = fmaf(sA[warp * r + k], sb[k], t);
+            t = warp_sum(t);
+            if (lane == 0) {
+                st[warp] = t;
+                nacc += (double)t * (double)t;
+                if (write_t && row0 + warp < rows) tvec[row0 + warp] = t;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int k = threadIdx.x + 256 * u;
+            if (k < r) {
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < kSvidRows; ++w) s = fmaf(sA[w * r + k], st[w], s);
+                acc[u] += s;
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int k = threadIdx.x + 256 * u;
+        if (k < r) partb[(int64_t)blockIdx.x * r + k] = acc[u];
+    }
+    if (lane == 0 && warp < kSvidRows) sn[warp] = nacc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double s = 0.0;
+        for (int w = 0; w < kSvidRows; ++w) s += sn[w];
+        partn[blockIdx.x] = s;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    svid_reduce_kernel(const float *__restrict__ partb, const double *__restrict__ partn, int nblk,
+                       int r, int64_t rows, int last, const float *__restrict__ tvec,
+                       float *b_out, float *a_out) {
+    __shared__ double s_inv;
+    if (threadIdx.x == 0) {
+        double n2 = 0.0;
+        for (int k = 0; k < nblk; ++k) n2 += partn[k];
+        const double nt = sqrt(n2);
+        s_inv = nt > 0.0 ? 1.0 / nt : 0.0;
+    }
+    __syncthreads();
+    const double inv = s_inv;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx < r) {
+        double s = 0.0;
+        for (int k = 0; k < nblk; ++k) s += partb[(int64_t)k * r + idx];
+        b_out[idx] = (float)(s * inv);
+    }
+    if (last && idx < rows) a_out[idx] = (float)((double)tvec[idx] * inv);
+}
+
+cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
+                 float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
+                 cudaStream_t s) {
+    const size_t smem = (size_t)(kSvidRows + 1) * r * sizeof(float);
+    static size_t configured = 0;
+    if (smem > 48 * 1024 && smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(svid_pass_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = smem;
+    }
+    const int64_t big = rows > r ? rows : r;
+    for (int pass = 1; pass <= K; ++pass) {
+        const float *b_in = pass == 1 ? nullptr : bcur + (size_t)((pass - 1) & 1) * r;
+        const bool last = pass == K;
+        float *b_out = last ? b : bcur + (size_t)(pass & 1) * r;
+        svid_pass_kernel<<<nsv, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec, last ? 1 : 0, partb,
+                                                partn);
+        svid_reduce_kernel<<<(unsigned)ceil_div(big, 256), 256, 0, s>>>(
+            partb, partn, nsv, r, rows, last ? 1 : 0, tvec, b_out, a);
+    }
+    return cudaGetLastError();
+}
+
+// =================================================================================
+// Objective ||W^ - U V^T||^2 / ||W^||^2 = (||W^||^2 - 2 <W^^T U, V> + <U^T U, V^T V>)
+// / ||W^||^2 from by-products: <W^^T U, V> from the V-step epilogue, the Gram
+// matrices (less the ridge) of both steps.
+// =================================================================================
+__global__ void __launch_bounds__(256)
+    gram_dot_kernel(const float *__restrict__ GU, const float *__restrict__ GV, int r, float c,
+                    double *part) {
+    __shared__ double sh[256];
+    const int64_t total = (int64_t)r * r;
+    double acc = 0.0;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const bool dg = (e / r) == (e % r);
+        acc += (double)(GU[e] - (dg ? c : 0.f)) * (double)(GV[e] - (dg ? c : 0.f));
+    }
+    const double t = block_sum_256(acc, sh);
+    if (threadIdx.x == 0) part[blockIdx.x] = t;
+}
+
+__global__ void __launch_bounds__(256)
+    objective_kernel(const double *__restrict__ px, int npx, const double *__restrict__ part,
+                     int npart, const Scalars *sc, float *obj_slot) {
+    __shared__ double sh[256];
+    double a = 0.0, b = 0.0;
+    for (int i = threadIdx.x; i < npx; i += blockDim.x) a += px[i];
+    for (int i = threadIdx.x; i < npart; i += blockDim.x) b += part[i];
+    const double spx = block_sum_256(a, sh);
+    const double sgg = block_sum_256(b, sh);
+    if (threadIdx.x == 0) {
+        const double w2 = sc->what_norm2;
+        *obj_slot = w2 > 0.0 ? (float)((w2 - 2.0 * spx + sgg) / w2) : 0.f;
+    }
+}
+
+cudaError_t objective(const float *GU, const float *GV, int32_t r, float c, const double *px,
+                      int npx, double *part, const Scalars *sc, float *obj_slot,
+                      cudaStream_t s) {
+    gram_dot_kernel<<<kRedBlocks, 256, 0, s>>>(GU, GV, r, c, part);
+    objective_kernel<<<1, 256, 0, s>>>(px, npx, part, kRedBlocks, sc, obj_slot);
+    return cudaGetLastError();
+}
+
+// =================================================================================
+// Magnitude balancing, scale extraction, sign packing.  Same page, "Method steps",
+// stage two (after convergence: balance, extract s1 and s2, pack the signs into
+// integers) and "Technical novelty" (技术新颖性).
+// =================================================================================
+__global__ void __launch_bounds__(256)
+    column_sumsq_kernel(const float *__restrict__ X, int64_t rows, int r, int64_t ldf,
+                        float *partb) {
+    float acc[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+    for (int64_t i = blockIdx.x; i < rows; i += gridDim.x) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int k = threadIdx.x + 256 * u;
+            if (k < r) {
+                const float x = X[i * ldf + k];
+                acc[u] = fmaf(x, x, acc[u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int k = threadIdx.x + 256 * u;
+        if (k < r) partb[(int64_t)blockIdx.x * r + k] = acc[u];
+    }
+}
+
+cudaError_t column_sumsq(const float *X, int64_t rows, int32_t r, int64_t ldf, int nblk,
+                         float *partb, cudaStream_t s) {
+    column_sumsq_kernel<<<nblk, 256, 0, s>>>(X, rows, r, ldf, partb);
+    return cudaGetLastError();
+}
+
+__global__ void balance_gains_kernel(const float *__restrict__ pu, const float *__restrict__ pv,
+                                     int nblk, int r, float *gk) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= r) return;
+    double su = 0.0, sv = 0.0;
+    for (int b = 0; b < nblk; ++b) {
+        su += pu[(int64_t)b * r + k];
+        sv += pv[(int64_t)b * r + k];
+    }
+    const double nu = sqrt(su), nv = sqrt(sv);
+    gk[k] = (nu > 0.0 && nv > 0.0) ? (float)sqrt(nv / nu) : 1.f;
+}
+
+cudaError_t balance_gains(const float *partU, const float *partV, int nblk, int32_t r, float *gk,
+                          cudaStream_t s) {
+    balance_gains_kernel<<<(unsigned)ceil_div(r, 256), 256, 0, s>>>(partU, partV, nblk, r, gk);
+    return cudaGetLastError();
+}
+
+// Warp per row: ballot of (x < 0) over 32 consecutive rank columns -> one word.
+__global__ void __launch_bounds__(256)
+    extract_pack_kernel(const float *__restrict__ X, int64_t rows, int r, int64_t ldf,
+                        const float *__restrict__ gk, int invert, const double *gamma,
+                        float *s_out, uint32_t *bits, __nv_bfloat16 *pm, int64_t ldpm) {
+    const int lane = threadIdx.x & 31;
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (i >= rows) return;
+    const int nw = (r + 31) / 32;
+    float sum = 0.f;
+    for (int w = 0; w < nw; ++w) {
+        const int k = 32 * w + lane;
+        const bool in = k < r;
+        const float x = in ? X[i * ldf + k] : 0.f;
+        if (in) {
+            const float g = gk ? gk[k] : 1.f;
+            sum += fabsf(invert ? x / g : x * g);
+        }
+        const unsigned word = __ballot_sync(0xffffffffu, in && x < 0.f);
+        if (lane == 0 && bits) bits[i * nw + w] = word;
+        if (in && pm) pm[i * ldpm + k] = __float2bfloat16_rn(x < 0.f ? -1.f : 1.f);
+    }
+    sum = warp_sum(sum);
+    if (lane == 0 && s_out) s_out[i] = (float)((double)sum / (double)r * (gamma ? *gamma : 1.0));
+}
+
+cudaError_t extract_pack(const float *X, int64_t rows, int32_t r, int64_t ldf, const float *gk,
+                         int invert, const double *gamma, float *s_out, uint32_t *bits,
+                         __nv_bfloat16 *pm, int64_t ldpm, cudaStream_t s) {
+    extract_pack_kernel<<<(unsigned)ceil_div(rows * 32, 256), 256, 0, s>>>(
+        X, rows, r, ldf, gk, invert, gamma, s_out, bits, pm, ldpm);
+    return cudaGetLastError();
+}
+
+cudaError_t pack_signs(const float *X, int64_t rows, int32_t r, int64_t ldx, uint32_t *bits,
+                       cudaStream_t s) {
+    return extract_pack(X, rows, r, ldx, nullptr, 0, nullptr, nullptr, bits, nullptr, 0, s);
+}
+
+__global__ void unpack_pm_kernel(const uint32_t *__restrict__ bits, int64_t rows, int r,
+                                 __nv_bfloat16 *pm, int64_t ldpm) {
+    const int nw = (r + 31) / 32;
+    const int64_t total = rows * (int64_t)r;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / r;
+        const int k = (int)(e % r);
+        const uint32_t w = bits[i * nw + k / 32];
+        pm[i * ldpm + k] = __float2bfloat16_rn(((w >> (k & 31)) & 1u) ? -1.f : 1.f);
+    }
+}
+
+cudaError_t unpack_pm(const uint32_t *bits, int64_t rows, int32_t r, __nv_bfloat16 *pm,
+                      int64_t ldpm, cudaStream_t s) {
+    unpack_pm_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(bits, rows, r, pm, ldpm);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    recon_finalize_kernel(const double *part, int count, const Scalars *sc, double *out) {
+    __shared__ double sh[256];
+    double a = 0.0;
+    for (int i = threadIdx.x; i < count; i += blockDim.x) a += part[i];
+    const double t = block_sum_256(a, sh);
+    if (threadIdx.x == 0) {
+        const double w2 = sc->wt_norm2;
+        *out = w2 > 0.0 ? sqrt(t / w2) : (t == 0.0 ? 0.0 : INFINITY);
+    }
+}
+
+cudaError_t recon_finalize(const double *part, int count, const Scalars *sc, double *out,
+                           cudaStream_t s) {
+    recon_finalize_kernel<<<1, 256, 0, s>>>(part, count, sc, out);
+    return cudaGetLastError();
+}
+
+}  // namespace nq

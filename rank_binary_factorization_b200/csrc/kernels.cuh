@@ -1,0 +1,80 @@
+// Launchers of the non-GEMM kernels (SIMT, sm_100a).
+#pragma once
+#include "common.cuh"
+#include "layout.h"
+
+namespace nq {
+
+// ---- calibration -----------------------------------------------------------------
+// Partial sums of x^2 and x^4 per (token slab, channel) in FP64.
+cudaError_t calib_partials(const void *X, int64_t T, int64_t C, int dt_bf16, int nslab,
+                           double *ps, double *pq, cudaStream_t s);
+// s_c, q_c = sum over slabs / T.
+cudaError_t calib_moments(const double *ps, const double *pq, int nslab, int64_t T, int64_t C,
+                          double *s_out, double *q_out, cudaStream_t st);
+// Ledoit-Wolf diagonal shrinkage -> d (float), alpha (double, device).
+cudaError_t calib_ledoit_wolf(const double *s, const double *q, int64_t T, int64_t C,
+                              double alpha_override, float *d, double *alpha, int *err,
+                              cudaStream_t st);
+int calib_num_slabs(int64_t T, int64_t C);
+
+// ---- preconditioned target -----------------------------------------------------
+// part[b] = partial sums of (d_out_i W_ij d_in_j)^2; non-finite -> NQ_ERR_NONFINITE.
+cudaError_t wt_norm_partials(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
+                             const float *d_out, double *part, int *err, cudaStream_t s);
+// sum of ``count`` partials in fixed order; writes *sum and, when gamma != null,
+// *gamma = sqrt(sum) / (2 sqrt(r)).
+cudaError_t reduce_partials(const double *part, int count, double *sum, double *gamma, int r,
+                            cudaStream_t s);
+// W^ = bf16(d_out W d_in / gamma) into What [m][ldn] and WhatT [n][ldm] (zero padded);
+// part[b] = partial sums of W^^2.
+cudaError_t what_cast(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
+                      const float *d_out, const double *gamma, __nv_bfloat16 *What, int64_t ldn,
+                      __nv_bfloat16 *WhatT, int64_t ldm, double *part, cudaStream_t s);
+// V_0 = sqrt(2/n) * splitmix64 signs into X [n][ldr] (float) and Xt [r][ldn] (bf16).
+cudaError_t init_v0(int64_t n, int32_t r, uint64_t seed, float *X, int64_t ldr,
+                    __nv_bfloat16 *Xt, int64_t ldn, cudaStream_t s);
+// Xt[k][i] = bf16(X[i][k]) for i < rows, k < r.
+cudaError_t transpose_to_bf16(const float *X, int64_t rows, int32_t r, int64_t ldx,
+                              __nv_bfloat16 *Xt, int64_t ldt, cudaStream_t s);
+// B[j][i] = A[i][j] (bf16), A rows x cols with row stride lda, B row stride ldb.
+cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, int64_t lda,
+                           __nv_bfloat16 *B, int64_t ldb, cudaStream_t s);
+
+// ---- Cholesky + inverse (cooperative, FP32) -------------------------------------
+// Gi = G^-1 for the SPD r x r matrix G (row stride r), written as hi + lo bf16 [r][ldr].
+cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
+                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr, int *err,
+                         unsigned int *bar, cudaStream_t s);
+
+// ---- SVID -------------------------------------------------------------------------
+// K power steps on |S| (S rows x r, row stride ldf): a = t/||t||, b = A^T t / ||t||.
+cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
+                 float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
+                 cudaStream_t s);
+
+// ---- objective --------------------------------------------------------------------
+// obj[slot] = (what_n2 - 2 sum(px) + <GU - cI, GV - cI>) / what_n2
+cudaError_t objective(const float *GU, const float *GV, int32_t r, float c, const double *px,
+                      int npx, double *part, const Scalars *sc, float *obj_slot,
+                      cudaStream_t s);
+
+// ---- balancing, scales, packing ---------------------------------------------------
+cudaError_t column_sumsq(const float *X, int64_t rows, int32_t r, int64_t ldf, int nblk,
+                         float *partb, cudaStream_t s);
+cudaError_t balance_gains(const float *partU, const float *partV, int nblk, int32_t r, float *gk,
+                          cudaStream_t s);
+// s_i = scale * mean_k |X_ik g_k^e| (e = +1 for U, -1 for V); sign bits; +-1 bf16 copy.
+cudaError_t extract_pack(const float *X, int64_t rows, int32_t r, int64_t ldf, const float *gk,
+                         int invert, const double *gamma, float *s_out, uint32_t *bits,
+                         __nv_bfloat16 *pm, int64_t ldpm, cudaStream_t s);
+cudaError_t pack_signs(const float *X, int64_t rows, int32_t r, int64_t ldx, uint32_t *bits,
+                       cudaStream_t s);
+// +-1 bf16 [rows][ldpm] from packed bits.
+cudaError_t unpack_pm(const uint32_t *bits, int64_t rows, int32_t r, __nv_bfloat16 *pm,
+                      int64_t ldpm, cudaStream_t s);
+// *out = sqrt(sum(part) / wt_norm2) (0 when both vanish)
+cudaError_t recon_finalize(const double *part, int count, const Scalars *sc, double *out,
+                           cudaStream_t s);
+
+}  // namespace nq

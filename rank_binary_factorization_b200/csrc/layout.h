@@ -1,0 +1,151 @@
+// Workspace layouts of the library (host and device visible).
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+namespace nq {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+constexpr int kSvidRows = 8;          // rows of S staged in shared memory per SVID tile
+constexpr int kRedBlocks = 592;       // CTAs of grid-stride reduction kernels (4 per SM)
+constexpr int kObjRing = 4096;        // per-iteration objective slots kept on the device
+constexpr int kMaxRank = 4096;
+constexpr int64_t kMaxDim = 65536;
+
+// Scalars block at the start of every workspace.
+struct Scalars {
+    double gamma;        // ||W~||_F / (2 sqrt r)
+    double wt_norm2;     // ||W~||_F^2 (W~ formed in FP32 from W, d_in, d_out)
+    double what_norm2;   // ||W^||_F^2 of the BF16 target
+    double alpha[2];     // Ledoit-Wolf intensities (calibration)
+    double recon2;       // sum of squared reconstruction errors
+    int err;             // first device-side error status
+    unsigned int bar[2]; // grid barrier (count, generation)
+    int pad;
+};
+
+struct LbLayout {
+    int64_t m = 0, n = 0;
+    int32_t r = 0;
+    int64_t ldr = 0;   // leading dim of every [rows][r] array (FP32 and BF16)
+    int64_t ldn = 0;   // leading dim of W^ rows (n padded) and of Vt
+    int64_t ldm = 0;   // leading dim of W^^T rows (m padded) and of Ut
+    int64_t rp = 0;    // r padded to 32 (Cholesky tiles)
+    int nsv = 0;       // CTAs of an SVID pass (rows of its partial array)
+    size_t scal = 0, what = 0, whatT = 0, x[2] = {0, 0}, s[2] = {0, 0}, a[2] = {0, 0},
+           b[2] = {0, 0}, xt[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
+           gih = 0, gil = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
+           partb = 0, obj = 0, total = 0;
+    size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
+
+    int64_t rows(int side) const { return side == 0 ? m : n; }
+    int64_t ld_rows(int side) const { return side == 0 ? ldm : ldn; }
+
+    void build(int64_t m_, int64_t n_, int32_t r_) {
+        m = m_;
+        n = n_;
+        r = r_;
+        ldr = (r + 7) / 8 * 8;
+        ldn = (n + 7) / 8 * 8;
+        ldm = (m + 7) / 8 * 8;
+        rp = (r + 31) / 32 * 32;
+        const int64_t maxrows = m > n ? m : n;
+        int64_t tiles_rows = (maxrows + kSvidRows - 1) / kSvidRows;
+        nsv = (int)(tiles_rows < 296 ? tiles_rows : 296);
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off = align_up(off + bytes);
+            return o;
+        };
+        scal = take(sizeof(Scalars));
+        what = take((size_t)m * ldn * 2);
+        whatT = take((size_t)n * ldm * 2);
+        for (int sd = 0; sd < 2; ++sd) {
+            const int64_t rw = sd == 0 ? m : n;
+            x[sd] = take((size_t)rw * ldr * 4);
+            s[sd] = take((size_t)rw * ldr * 4);
+            a[sd] = take((size_t)rw * 4);
+            b[sd] = take((size_t)r * 4);
+            xt[sd] = take((size_t)r * (sd == 0 ? ldm : ldn) * 2);
+            g[sd] = take((size_t)r * r * 4);
+        }
+        rhi = take((size_t)maxrows * ldr * 2);
+        rlo = take((size_t)maxrows * ldr * 2);
+        chA = take((size_t)rp * rp * 4);
+        chLi = take((size_t)rp * rp * 4);
+        gih = take((size_t)r * ldr * 2);
+        gil = take((size_t)r * ldr * 2);
+        tvec = take((size_t)maxrows * 4);
+        bcur = take((size_t)2 * r * 4);
+        gk = take((size_t)r * 4);
+        // per-tile partials: GEMM tiles at BN = 64 for the objective (n x r) and the
+        // reconstruction error (m x n); grid-stride reductions use kRedBlocks
+        const int64_t t_obj = ((n + 127) / 128) * ((r + 63) / 64);
+        const int64_t t_rec = ((m + 127) / 128) * ((n + 63) / 64);
+        int64_t pd = t_obj > t_rec ? t_obj : t_rec;
+        if (pd < kRedBlocks) pd = kRedBlocks;
+        part_doubles = (size_t)pd;
+        part = take(part_doubles * 8);        // per-tile partials / grid-stride partials
+        partn = take((size_t)nsv * 8);        // SVID norm partials
+        partg = take((size_t)kRedBlocks * 8); // Gram dot-product partials
+        partb = take((size_t)2 * nsv * r * 4);  // column partials (SVID; U and V norms)
+        obj = take((size_t)kObjRing * 4);
+        total = off;
+    }
+};
+
+struct CalibLayout {
+    int64_t T = 0, C = 0;
+    int nslab = 0;     // token slabs
+    size_t scal = 0, ps = 0, pq = 0, s = 0, q = 0, total = 0;
+    void build(int64_t T_, int64_t C_, int nslab_) {
+        T = T_;
+        C = C_;
+        nslab = nslab_;
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off = align_up(off + bytes);
+            return o;
+        };
+        scal = take(sizeof(Scalars));
+        ps = take((size_t)nslab * C * 8);
+        pq = take((size_t)nslab * C * 8);
+        s = take((size_t)C * 8);
+        q = take((size_t)C * 8);
+        total = off;
+    }
+};
+
+struct ReconLayout {
+    int64_t m = 0, n = 0;
+    int32_t r = 0;
+    int64_t ldr = 0;
+    size_t scal = 0, up = 0, vp = 0, part = 0, total = 0;
+    size_t part_doubles = 0;
+    void build(int64_t m_, int64_t n_, int32_t r_) {
+        m = m_;
+        n = n_;
+        r = r_;
+        ldr = (r + 7) / 8 * 8;
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off = align_up(off + bytes);
+            return o;
+        };
+        scal = take(sizeof(Scalars));
+        up = take((size_t)m * ldr * 2);
+        vp = take((size_t)n * ldr * 2);
+        int64_t t_rec = ((m + 127) / 128) * ((n + 63) / 64);
+        if (t_rec < kRedBlocks) t_rec = kRedBlocks;
+        part_doubles = (size_t)t_rec;
+        part = take(part_doubles * 8);
+        total = off;
+    }
+};
+
+}  // namespace nq
