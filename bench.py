@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the NanoQuant hot path on B200.
+
+One step = the whole hot path over one layer's synthetic inputs, resident in HBM:
+  calibration preconditioners from two 262144 x 4096 BF16 token streams
+  (nq_calib_precond), then LB-ADMM on the 4096 x 4096 BF16 q_proj-shaped layer at
+  1 BPW (r = 2032): target preparation, 100 iterations, balancing, scales, packing and
+  the reconstruction error (nq_lbadmm).
+Metric: LB-ADMM layer-iterations per second of the whole step (iterations x layers /
+step time), with 4mnr TFLOP/s, calibration GB/s and the roofline fraction of the
+dominant kernel alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+
+N > 1 runs one independent replica per GPU (the layer does not shard here): no
+collective on the data path, barrier + max-over-ranks timing, weak scaling.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LB-ADMM layer-iters/s & TFLOP/s vs roofline; calib-stats GB/s vs HBM peak"
+UNIT = "layer-iters/s"
+WORKLOAD = dict(name="llama2-7b q_proj 4096x4096 bf16, r=2032 (1.0 BPW), 100 LB-ADMM iterations, "
+                     "calibration 2 x 262144x4096 bf16 streams",
+                m=4096, n=4096, bpw=1.0, iters=100, T=128 * 2048, rho=1.0, lam=1e-4, K=4)
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+
+
+# ---------------------------------------------------------------------------------------
+# helpers shared by both arms (and tested on CPU with gloo)
+# ---------------------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def reduce_max(value, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    fp32 = NUM_SMS * FP32_LANES_PER_SM * 2 * 1.965e9 / 1e12
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    fp32_tflops=fp32, source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                fp32_tflops=fp32, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(smax) if smax else None, samples=len(sm),
+                    reasons=sorted(reasons))
+
+
+def kernel_units(cls, m, n, r, K, T):
+    """Algorithmic work of one launch scope of a kernel class: (amount, unit, bound)."""
+    if cls == "calib":
+        return T * max(m, n) * 2, "B", "hbm"                 # one BF16 stream read once
+    if cls == "rhs":
+        return 2.0 * m * n * r, "FLOP", "tensor"             # W^ X (either side)
+    if cls == "solve":
+        return 2.0 * (m + n) / 2 * r * r, "FLOP", "tensor"   # R G^-1 (mean of both sides)
+    if cls == "gram":
+        return 2.0 * (m + n) / 2 * r * r, "FLOP", "tensor"   # X^T X (full square)
+    if cls == "chol":
+        return float(r) ** 3, "FLOP", "alu"                  # Cholesky + inverse + L^-T L^-1
+    if cls == "svid":
+        return 4.0 * K * (m + n) / 2 * r, "B", "hbm"         # K reads of S (FP32)
+    return None
+
+
+def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
+    u = kernel_units(cls, m, n, r, K, T)
+    if u is None or launches == 0 or ms <= 0:
+        return None
+    amount, unit, bound = u
+    per_launch_s = ms / 1e3 / launches
+    if unit == "B":
+        achieved, peak, punit = amount / per_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    elif bound == "tensor":
+        achieved, peak, punit = amount / per_launch_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+    else:
+        achieved, peak, punit = amount / per_launch_s / 1e12, peaks["fp32_tflops"], "TFLOP/s"
+    return dict(kernel=cls, bound=bound, achieved=round(achieved, 2), peak=round(peak, 1),
+                unit=punit, frac=round(achieved / peak, 4), traffic=None,
+                launches=launches, ms_per_launch=round(ms / launches, 4),
+                share_of_step=None)
+
+
+# ---------------------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------
+def oracle_sample(W_h, acts_h, grads_h, r, iters, T):
+    """Time the oracle on a bounded sample and extrapolate one step; returns (value, info)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import calib as OC
+    from oracle import lbadmm as O
+    Ts = 16384
+    t0 = time.perf_counter()
+    d_in, d_out, _, _ = OC.calib_precond([acts_h[:Ts].float().numpy()],
+                                         [grads_h[:Ts].float().numpy()])
+    t_calib = (time.perf_counter() - t0) * (T / Ts)
+    Wd = W_h.double().numpy()
+    t0 = time.perf_counter()
+    res = O.lbadmm(Wd, d_in, d_out, r=r, iters=1)
+    t_one = time.perf_counter() - t0
+    step_s = t_calib + iters * t_one
+    cores = max([ti.get("num_threads", 1) for ti in threadpool_info()] + [1])
+    return iters / step_s, dict(
+        kind="oracle", cores=cores,
+        sample=f"calibration on {Ts} of {T} tokens per stream (time scaled by {T // Ts}); "
+               f"one full LB-ADMM iteration (with preparation, balancing, packing and the "
+               f"reconstruction error) on the whole {Wd.shape[0]}x{Wd.shape[1]} layer, time "
+               f"scaled to {iters} iterations", sample_s=round(t_calib * Ts / T + t_one, 2),
+        est_step_s=round(step_s, 2))
+
+
+def make_host_inputs(seed, m, n, T):
+    """Seeded synthetic inputs generated on the device, kept in pinned host memory too."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + seed)
+    W = torch.randn(m, n, device="cuda", generator=g) * 0.02
+    cols = torch.randperm(n, device="cuda", generator=g)[: max(1, n // 100)]
+    W[:, cols] *= 10.0
+    W = W.to(torch.bfloat16)
+
+    def stream(C):
+        scales = torch.exp(torch.randn(C, device="cuda", generator=g))
+        out = torch.empty(T, C, dtype=torch.bfloat16, device="cuda")
+        for t0 in range(0, T, 32768):
+            t1 = min(T, t0 + 32768)
+            out[t0:t1] = (torch.randn(t1 - t0, C, device="cuda", generator=g) * scales).to(
+                torch.bfloat16)
+        return out
+    acts = stream(n)
+    grads = stream(m)
+    host = [t.to("cpu", non_blocking=False).pin_memory() for t in (W, acts, grads)]
+    return (W, acts, grads), host
+
+
+# ---------------------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------------------
+def run_reference(args):
+    rank, local_rank, world = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    m, n, T, iters = WORKLOAD["m"], WORKLOAD["n"], WORKLOAD["T"], args.iters
+    from oracle.bpw import rank_for_bpw
+    r = rank_for_bpw(m, n, WORKLOAD["bpw"])
+    from synth import gaussian_weight, stream_tensor
+    W_h = gaussian_weight(0, "W", m, n, 0.02, 0.01, 10.0)
+    Ts = 16384
+    acts_h = stream_tensor(0, "acts", Ts, n)
+    grads_h = stream_tensor(0, "grads", Ts, m)
+    for _ in range(args.warmup):
+        oracle_sample(W_h, acts_h, grads_h, r, iters, T)
+    vals = []
+    info = None
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, info = oracle_sample(W_h, acts_h, grads_h, r, iters, T)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    info["value"] = value
+    info["unit"] = UNIT
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * iters / value, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=WORKLOAD["name"], m=m, n=n, r=r, iters=iters, T=T),
+                cpu_baseline=info, wall_s=round(wall, 1),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    import rank_binary_factorization_b200 as nq
+
+    m, n, T, iters = WORKLOAD["m"], WORKLOAD["n"], WORKLOAD["T"], args.iters
+    rho, lam, K = WORKLOAD["rho"], WORKLOAD["lam"], WORKLOAD["K"]
+    r = nq.nq_rank_for_bpw(m, n, WORKLOAD["bpw"])
+    (W, acts, grads), (W_h, acts_h, grads_h) = make_host_inputs(rank, m, n, T)
+    calib_ws = nq.workspace(nq.lib.nq_calib_workspace_size(T, max(m, n)))
+    lb_ws = nq.workspace(nq.lib.nq_lbadmm_workspace_size(m, n, r))
+
+    def step():
+        d_in, d_out, _, _ = nq.nq_calib_precond(acts, grads, ws=calib_ws, sync=False)
+        return nq.nq_lbadmm(W, r, d_in, d_out, rho=rho, lam=lam, iters=iters, K=K, seed=0,
+                            ws=lb_ws)
+
+    def e2e_step():
+        W.copy_(W_h, non_blocking=True)
+        acts.copy_(acts_h, non_blocking=True)
+        grads.copy_(grads_h, non_blocking=True)
+        res = step()
+        host = [res[k].to("cpu") for k in ("U_packed", "V_packed", "s1", "s2")]
+        return res, host
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 0)):
+        res = step()
+    torch.cuda.synchronize()
+
+    # device-timed region: inputs resident in HBM
+    clocks = ClockSampler(local_rank)
+    barrier(device)
+    torch.cuda.synchronize()
+    nq.nq_profile_enable(True)
+    launches0 = nq.nq_launch_count()
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        res = step()
+    ev1.record(stream)
+    ev1.synchronize()
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    barrier(device)
+    launches = nq.nq_launch_count() - launches0
+    prof = nq.nq_profile_get()
+    nq.nq_profile_enable(False)
+    t_local = ev0.elapsed_time(ev1) / 1e3
+    t = reduce_max(t_local, device)
+
+    # end-to-end through the public API with pinned host buffers
+    for _ in range(1):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(device)
+    ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev2.record(stream)
+    e2e_steps = max(1, min(args.steps, 3))
+    for _ in range(e2e_steps):
+        res_e2e, host = e2e_step()
+    ev3.record(stream)
+    ev3.synchronize()
+    t_e2e = reduce_max(ev2.elapsed_time(ev3) / 1e3, device)
+    h2d = sum(x.numel() * x.element_size() for x in (W_h, acts_h, grads_h))
+    d2h = sum(x.numel() * x.element_size() for x in host) + 4 * iters + 4
+
+    peaks = read_peaks()
+    step_ms = t / args.steps * 1e3
+    entries = {}
+    for cls, (nl, ms) in prof.items():
+        e = roofline_entry(cls, nl, ms, m, n, r, K, T, peaks)
+        if e is not None:
+            e["share_of_step"] = round(ms / (t_local * 1e3), 4)
+            entries[cls] = e
+    dominant = max(entries.values(), key=lambda e: e["launches"] * e["ms_per_launch"])
+    value = world * iters * args.steps / t
+    tflops = 4.0 * m * n * r * iters * world * args.steps / t / 1e12
+    calib = entries.get("calib")
+    line = dict(
+        metric=METRIC, value=round(value, 3), unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=round(step_ms, 3), higher_is_better=True,
+        scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+        config=dict(workload=WORKLOAD["name"], m=m, n=n, r=r, iters=iters, T=T, rho=rho,
+                    lam=lam, K=K, parallelism=f"replicas x{world}",
+                    l2="inputs larger than L2 (2 x 2.1 GB calibration streams read every step)"),
+        tflops_4mnr=round(tflops, 2),
+        lbadmm_ms_per_iter=round((step_ms - (prof["calib"][1] + prof["calib_finalize"][1])
+                                  / args.steps) / iters, 4),
+        calib_gbs=calib["achieved"] if calib else None,
+        roofline=dominant,
+        kernels=entries,
+        peaks_source=peaks["source"],
+        gpu_launches=int(launches),
+        clocks=clk,
+        e2e=dict(value=round(world * iters * e2e_steps / t_e2e, 3), unit=UNIT,
+                 h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h)),
+        rel_err=res["rel_err"])
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, info = oracle_sample(W_h, acts_h, grads_h, r, iters, T)
+        info["value"] = round(v, 5)
+        info["unit"] = UNIT
+        line["cpu_baseline"] = info
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

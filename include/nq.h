@@ -232,6 +232,37 @@ nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, void *ws, siz
 nq_status nq_lbadmm_check(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
                           nq_stream_t stream);
 
+/* ------------------------------------------------------------------------- */
+/* Measurement helpers (not steps of the method).  When enabled, the library   */
+/* records a pair of CUDA events on the launching stream around every kernel   */
+/* launch and attributes the elapsed device time to the kernel's class.        */
+/* Off by default; recording costs one event pair per launch.  Not for use     */
+/* while the stream is being captured into a CUDA graph.                       */
+/* ------------------------------------------------------------------------- */
+typedef enum {
+    NQ_K_CALIB = 0,     /* calibration moment reduction (both streams)              */
+    NQ_K_CALIB_FIN = 1, /* moments finalize + Ledoit-Wolf                            */
+    NQ_K_PREP = 2,      /* target preparation, V_0                                   */
+    NQ_K_GRAM = 3,      /* tcgen05 Gram X^T X + (lambda + rho) I                     */
+    NQ_K_CHOL = 4,      /* Cholesky + inverse                                        */
+    NQ_K_RHS = 5,       /* tcgen05 W^ X + rho (Z - L)                                */
+    NQ_K_SOLVE = 6,     /* tcgen05 R G^-1 with the dual-state epilogue               */
+    NQ_K_SVID = 7,      /* SVID power passes                                         */
+    NQ_K_OBJ = 8,       /* per-iteration objective                                   */
+    NQ_K_FINISH = 9,    /* balancing, scales, packing                                */
+    NQ_K_RECON = 10,    /* tcgen05 +-1 reconstruction error                          */
+    NQ_K_COUNT = 11
+} nq_kernel_class;
+
+/* Number of kernel launches the library has issued in this process. */
+int64_t nq_launch_count(void);
+
+/* Enable (1) or disable (0) recording; enabling also clears previous records. */
+nq_status nq_profile_enable(int32_t enable);
+/* Launch count and summed device milliseconds of one class since enabling.
+ * Synchronises with the recorded events. */
+nq_status nq_profile_get(int32_t kernel_class, int64_t *launches, double *total_ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,8 +6,14 @@ calls the library of the same name; all computation runs in the CUDA kernels of
 ``libnq.so``.  Importing this package without the built library raises ImportError.
 """
 import ctypes
+import os
 
 import torch
+
+from . import build as _build
+
+if os.environ.get("NQ_NO_AUTOBUILD") != "1":
+    _build.build()          # no-op unless libnq.so is missing or older than its sources
 
 from . import _lib
 from ._lib import FIELDS, NQ_BF16, NQ_F32, NQError, check, lib, status_string
@@ -15,6 +21,7 @@ from ._lib import FIELDS, NQ_BF16, NQ_F32, NQError, check, lib, status_string
 __all__ = [
     "nq_bpw", "nq_rank_for_bpw", "nq_calib_stats", "nq_calib_precond", "nq_lbadmm",
     "nq_recon_error", "nq_pack_signs", "LBState", "NQError", "status_string", "lib",
+    "nq_launch_count", "nq_profile_enable", "nq_profile_get",
 ]
 
 
@@ -129,6 +136,25 @@ def nq_pack_signs(X):
     bits = torch.empty(rows, (r + 31) // 32, dtype=torch.int32, device=X.device)
     check("nq_pack_signs", lib.nq_pack_signs(_ptr(X), rows, r, _ptr(bits), _stream()))
     return bits
+
+
+def nq_launch_count():
+    """Kernel launches issued by the library so far in this process."""
+    return lib.nq_launch_count()
+
+
+def nq_profile_enable(on=True):
+    check("nq_profile_enable", lib.nq_profile_enable(1 if on else 0))
+
+
+def nq_profile_get():
+    """{kernel class: (launch scopes, device ms)} recorded since nq_profile_enable(True)."""
+    out = {}
+    for i, name in enumerate(_lib.KERNEL_CLASSES):
+        n, ms = ctypes.c_int64(), ctypes.c_double()
+        check("nq_profile_get", lib.nq_profile_get(i, ctypes.byref(n), ctypes.byref(ms)))
+        out[name] = (n.value, ms.value)
+    return out
 
 
 class LBState:

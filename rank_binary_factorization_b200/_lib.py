@@ -12,8 +12,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m rank_binary_factorization_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python rank_binary_factorization_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -56,7 +56,12 @@ SIGNATURES = {
                                       ctypes.POINTER(c_i32), ctypes.POINTER(c_i64)]),
     "nq_lbadmm_sync_operands": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
     "nq_lbadmm_check": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
+    "nq_launch_count": (c_i64, []),
+    "nq_profile_enable": (c_i32, [c_i32]),
+    "nq_profile_get": (c_i32, [c_i32, ctypes.POINTER(c_i64), ctypes.POINTER(c_f64)]),
 }
+KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
+                  "objective", "finish", "recon"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

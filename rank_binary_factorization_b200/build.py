@@ -1,6 +1,6 @@
 """Build the sm_100a shared library ``libnq.so`` in-tree (nvcc, no JIT cache).
 
-    python -m rank_binary_factorization_b200.build [--force]
+    python rank_binary_factorization_b200/build.py [--force]
 """
 import os
 import subprocess

@@ -3,11 +3,20 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 #include "layout.h"
 
 using namespace nq;
+
+namespace nq {
+static std::atomic<long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace nq
 
 namespace {
 
@@ -18,6 +27,37 @@ namespace {
     } while (0)
 
 inline cudaStream_t cs(nq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---- optional per-launch device timing (nq_profile_*) ------------------------------
+struct ProfRec {
+    int cls;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::vector<ProfRec> g_prof;
+size_t g_prof_used = 0;
+bool g_prof_on = false;
+
+struct ProfScope {
+    ProfRec *rec = nullptr;
+    cudaStream_t s;
+    ProfScope(int cls, cudaStream_t st) : s(st) {
+        if (!g_prof_on) return;
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        if (g_prof_used == g_prof.size()) {
+            ProfRec r{cls, nullptr, nullptr};
+            if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess)
+                return;
+            g_prof.push_back(r);
+        }
+        rec = &g_prof[g_prof_used++];
+        rec->cls = cls;
+        cudaEventRecord(rec->a, s);
+    }
+    ~ProfScope() {
+        if (rec) cudaEventRecord(rec->b, s);
+    }
+};
 
 template <class T>
 inline T *at(void *ws, size_t off) {
@@ -92,7 +132,11 @@ CalibCarve carve_calib(void *ws, int64_t C) {
 nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s_out,
                         double *q_out, const CalibCarve &cv, cudaStream_t st) {
     const int nslab = calib_num_slabs(T, C);
-    NQ_CK(calib_partials(X, T, C, bf16, nslab, cv.ps, cv.pq, st));
+    {
+        ProfScope ps(NQ_K_CALIB, st);
+        NQ_CK(calib_partials(X, T, C, bf16, nslab, cv.ps, cv.pq, st));
+    }
+    ProfScope ps(NQ_K_CALIB_FIN, st);
     NQ_CK(calib_moments(cv.ps, cv.pq, nslab, T, C, s_out, q_out, st));
     return NQ_OK;
 }
@@ -140,6 +184,7 @@ nq_status lb_gram(const Lb &lb, int other, float diag, cudaStream_t s) {
     ep.out = lb.p<float>(L.g[other]);
     ep.ldo = L.r;
     ep.diag = diag;
+    ProfScope ps(NQ_K_GRAM, s);
     NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
     return NQ_OK;
 }
@@ -151,9 +196,12 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
     const int BN = pick_bn(L.r);
     nq_status st = lb_gram(lb, other, lambda + rho, s);
     if (st) return st;
+    {
+    ProfScope ps(NQ_K_CHOL, s);
     NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
                        lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.gih),
                        lb.p<__nv_bfloat16>(L.gil), L.ldr, &lb.sc->err, lb.sc->bar, s));
+    }
 
     // R = W^ X_other + rho (Z - L), split into hi + lo bf16
     {
@@ -179,6 +227,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
         ep.Rhi = lb.p<__nv_bfloat16>(L.rhi);
         ep.Rlo = lb.p<__nv_bfloat16>(L.rlo);
         ep.ldr = L.ldr;
+        ProfScope ps(NQ_K_RHS, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RHS, BN, s));
     }
     // X = R G^-1 = [R_hi, R_lo, R_hi] [Gi_hi; Gi_hi; Gi_lo]; S <- X + L; Xt = bf16(X)^T
@@ -214,8 +263,10 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
         ep.ldxt = L.ld_rows(side);
         ep.objective = side == 1;
         ep.part = lb.p<double>(L.part);
+        ProfScope ps(NQ_K_SOLVE, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BN, s));
     }
+    ProfScope ps(NQ_K_SVID, s);
     NQ_CK(svid(lb.p<float>(L.s[side]), rows, L.r, L.ldr, K, L.nsv, lb.p<float>(L.bcur),
                lb.p<float>(L.tvec), lb.p<float>(L.partb), lb.p<double>(L.partn),
                lb.p<float>(L.a[side]), lb.p<float>(L.b[side]), s));
@@ -225,6 +276,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
 nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
     const LbLayout &L = lb.L;
     const int npx = (int)tc::num_tiles((int)L.n, L.r, pick_bn(L.r));
+    ProfScope ps(NQ_K_OBJ, s);
     NQ_CK(objective(lb.p<float>(L.g[0]), lb.p<float>(L.g[1]), L.r, c, lb.p<double>(L.part), npx,
                     lb.p<double>(L.partg), lb.sc, lb.p<float>(L.obj) + slot, s));
     return NQ_OK;
@@ -233,6 +285,7 @@ nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
 nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
                      const float *d_out, uint64_t seed, cudaStream_t s) {
     const LbLayout &L = lb.L;
+    ProfScope ps(NQ_K_PREP, s);
     NQ_CK(cudaMemsetAsync(lb.sc, 0, sizeof(Scalars), s));
     NQ_CK(wt_norm_partials(W, bf16, L.m, L.n, d_in, d_out, lb.p<double>(L.part), &lb.sc->err, s));
     NQ_CK(reduce_partials(lb.p<double>(L.part), kRedBlocks, &lb.sc->wt_norm2, &lb.sc->gamma, L.r,
@@ -286,6 +339,8 @@ nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, co
     const LbLayout &L = lb.L;
     float *pu = lb.p<float>(L.partb);
     float *pv = pu + (size_t)L.nsv * L.r;
+    {
+    ProfScope ps(NQ_K_FINISH, s);
     NQ_CK(column_sumsq(lb.p<float>(L.x[0]), L.m, L.r, L.ldr, L.nsv, pu, s));
     NQ_CK(column_sumsq(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, L.nsv, pv, s));
     NQ_CK(balance_gains(pu, pv, L.nsv, L.r, lb.p<float>(L.gk), s));
@@ -293,7 +348,9 @@ nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, co
                        s1, Up, lb.p<__nv_bfloat16>(L.rhi), L.ldr, s));
     NQ_CK(extract_pack(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, lb.p<float>(L.gk), 1, nullptr, s2, Vp,
                        lb.p<__nv_bfloat16>(L.rlo), L.ldr, s));
+    }
     if (!want_err) return NQ_OK;
+    ProfScope ps(NQ_K_RECON, s);
     const int BN = pick_bn(L.n);
     tc::Maps maps;
     memset(&maps, 0, sizeof(maps));
@@ -393,11 +450,17 @@ nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void
     NQ_CK(cudaMemsetAsync(cv.sc, 0, sizeof(Scalars), s));
     const int bf16 = dt == NQ_BF16;
     if ((st = enqueue_stats(acts, T_in, n, bf16, cv.s, cv.q, cv, s))) return st;
-    NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_in, n, alpha_override, d_in, &cv.sc->alpha[0],
-                            &cv.sc->err, s));
+    {
+        ProfScope ps(NQ_K_CALIB_FIN, s);
+        NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_in, n, alpha_override, d_in, &cv.sc->alpha[0],
+                                &cv.sc->err, s));
+    }
     if ((st = enqueue_stats(grads, T_out, m, bf16, cv.s, cv.q, cv, s))) return st;
-    NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_out, m, alpha_override, d_out, &cv.sc->alpha[1],
-                            &cv.sc->err, s));
+    {
+        ProfScope ps(NQ_K_CALIB_FIN, s);
+        NQ_CK(calib_ledoit_wolf(cv.s, cv.q, T_out, m, alpha_override, d_out, &cv.sc->alpha[1],
+                                &cv.sc->err, s));
+    }
     if (alpha_out) {
         Scalars h;
         NQ_CK(cudaMemcpyAsync(&h, cv.sc, sizeof(Scalars), cudaMemcpyDeviceToHost, s));
@@ -629,6 +692,35 @@ nq_status nq_lbadmm_check(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_b
     nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
     if (st) return st;
     return read_err(&lb.sc->err, cs(stream), true);
+}
+
+int64_t nq_launch_count(void) { return (int64_t)nq::g_launches.load(); }
+
+nq_status nq_profile_enable(int32_t enable) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_used = 0;
+    g_prof_on = enable != 0;
+    return NQ_OK;
+}
+
+nq_status nq_profile_get(int32_t kernel_class, int64_t *launches, double *total_ms) {
+    if (!launches || !total_ms || kernel_class < 0 || kernel_class >= NQ_K_COUNT)
+        return NQ_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    int64_t n = 0;
+    double ms = 0.0;
+    for (size_t i = 0; i < g_prof_used; ++i) {
+        const ProfRec &r = g_prof[i];
+        if (r.cls != kernel_class) continue;
+        NQ_CK(cudaEventSynchronize(r.b));
+        float t = 0.f;
+        NQ_CK(cudaEventElapsedTime(&t, r.a, r.b));
+        ms += t;
+        ++n;
+    }
+    *launches = n;
+    *total_ms = ms;
+    return NQ_OK;
 }
 
 }  // extern "C"

@@ -12,6 +12,9 @@ namespace nq {
 
 constexpr int kNumSMsB200 = 148;
 
+// Host-side count of kernel launches issued by the library (nq_launch_count).
+void count_launch(int n = 1);
+
 NQ_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 NQ_HD int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 

@@ -369,6 +369,7 @@ static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s
     }
     dim3 grid((unsigned)ceil_div(p.M, BM), (unsigned)ceil_div(p.N, BN));
     kern<<<grid, kThreads, smem, s>>>(maps, p);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -170,6 +170,7 @@ cudaError_t calib_partials(const void *X, int64_t T, int64_t C, int dt_bf16, int
         else
             calib_partial_scalar<false><<<grid, 256, 0, s>>>(X, T, C, tps, ps, pq);
     }
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -191,6 +192,7 @@ cudaError_t calib_moments(const double *ps, const double *pq, int nslab, int64_t
                           double *s_out, double *q_out, cudaStream_t st) {
     calib_moments_kernel<<<(unsigned)ceil_div(C, 256), 256, 0, st>>>(ps, pq, nslab, T, C, s_out,
                                                                      q_out);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -244,6 +246,7 @@ cudaError_t calib_ledoit_wolf(const double *s, const double *q, int64_t T, int64
                               double alpha_override, float *d, double *alpha, int *err,
                               cudaStream_t st) {
     calib_lw_kernel<<<1, 1024, 0, st>>>(s, q, T, C, alpha_override, d, alpha, err);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -293,6 +296,7 @@ __global__ void __launch_bounds__(256)
 cudaError_t wt_norm_partials(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
                              const float *d_out, double *part, int *err, cudaStream_t s) {
     wt_norm_kernel<<<kRedBlocks, 256, 0, s>>>(W, w_bf16, m, n, d_in, d_out, part, err);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -311,6 +315,7 @@ __global__ void __launch_bounds__(256)
 cudaError_t reduce_partials(const double *part, int count, double *sum, double *gamma, int r,
                             cudaStream_t s) {
     reduce_partials_kernel<<<1, 256, 0, s>>>(part, count, sum, gamma, r);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -360,6 +365,7 @@ cudaError_t what_cast(const void *W, int w_bf16, int64_t m, int64_t n, const flo
                       __nv_bfloat16 *WhatT, int64_t ldm, double *part, cudaStream_t s) {
     what_cast_kernel<<<kRedBlocks, 256, 0, s>>>(W, w_bf16, m, n, d_in, d_out, gamma, What, ldn,
                                                 WhatT, ldm, part);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -391,6 +397,7 @@ cudaError_t init_v0(int64_t n, int32_t r, uint64_t seed, float *X, int64_t ldr,
                     __nv_bfloat16 *Xt, int64_t ldn, cudaStream_t s) {
     const float c = sqrtf(2.0f / (float)n);
     init_v0_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(n, r, seed, c, X, ldr, Xt, ldn);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -415,6 +422,7 @@ cudaError_t transpose_to_bf16(const float *X, int64_t rows, int32_t r, int64_t l
                               __nv_bfloat16 *Xt, int64_t ldt, cudaStream_t s) {
     dim3 grid((unsigned)ceil_div(r, 32), (unsigned)ceil_div(rows, 32));
     transpose_to_bf16_kernel<<<grid, 256, 0, s>>>(X, rows, r, ldx, Xt, ldt);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -439,6 +447,7 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
                            __nv_bfloat16 *B, int64_t ldb, cudaStream_t s) {
     dim3 grid((unsigned)ceil_div(cols, 32), (unsigned)ceil_div(rows, 32));
     transpose_bf16_kernel<<<grid, 256, 0, s>>>(A, rows, cols, lda, B, ldb);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -700,6 +709,7 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
     if (e != cudaSuccess) return e;
     CholArgs args{G, r, rp, A, Li, Gi_hi, Gi_lo, ldr, err, bar};
     void *params[] = {&args};
+    count_launch();
     return cudaLaunchCooperativeKernel((const void *)chol_inv_kernel, dim3(grid), dim3(256),
                                        params, 0, s);
 }
@@ -812,8 +822,10 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
         float *b_out = last ? b : bcur + (size_t)(pass & 1) * r;
         svid_pass_kernel<<<nsv, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec, last ? 1 : 0, partb,
                                                 partn);
+        count_launch();
         svid_reduce_kernel<<<(unsigned)ceil_div(big, 256), 256, 0, s>>>(
             partb, partn, nsv, r, rows, last ? 1 : 0, tvec, b_out, a);
+        count_launch();
     }
     return cudaGetLastError();
 }
@@ -857,7 +869,9 @@ cudaError_t objective(const float *GU, const float *GV, int32_t r, float c, cons
                       int npx, double *part, const Scalars *sc, float *obj_slot,
                       cudaStream_t s) {
     gram_dot_kernel<<<kRedBlocks, 256, 0, s>>>(GU, GV, r, c, part);
+    count_launch();
     objective_kernel<<<1, 256, 0, s>>>(px, npx, part, kRedBlocks, sc, obj_slot);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -892,6 +906,7 @@ __global__ void __launch_bounds__(256)
 cudaError_t column_sumsq(const float *X, int64_t rows, int32_t r, int64_t ldf, int nblk,
                          float *partb, cudaStream_t s) {
     column_sumsq_kernel<<<nblk, 256, 0, s>>>(X, rows, r, ldf, partb);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -911,6 +926,7 @@ __global__ void balance_gains_kernel(const float *__restrict__ pu, const float *
 cudaError_t balance_gains(const float *partU, const float *partV, int nblk, int32_t r, float *gk,
                           cudaStream_t s) {
     balance_gains_kernel<<<(unsigned)ceil_div(r, 256), 256, 0, s>>>(partU, partV, nblk, r, gk);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -945,6 +961,7 @@ cudaError_t extract_pack(const float *X, int64_t rows, int32_t r, int64_t ldf, c
                          __nv_bfloat16 *pm, int64_t ldpm, cudaStream_t s) {
     extract_pack_kernel<<<(unsigned)ceil_div(rows * 32, 256), 256, 0, s>>>(
         X, rows, r, ldf, gk, invert, gamma, s_out, bits, pm, ldpm);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -969,6 +986,7 @@ __global__ void unpack_pm_kernel(const uint32_t *__restrict__ bits, int64_t rows
 cudaError_t unpack_pm(const uint32_t *bits, int64_t rows, int32_t r, __nv_bfloat16 *pm,
                       int64_t ldpm, cudaStream_t s) {
     unpack_pm_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(bits, rows, r, pm, ldpm);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -987,6 +1005,7 @@ __global__ void __launch_bounds__(256)
 cudaError_t recon_finalize(const double *part, int count, const Scalars *sc, double *out,
                            cudaStream_t s) {
     recon_finalize_kernel<<<1, 256, 0, s>>>(part, count, sc, out);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -24,3 +24,22 @@ def read_golden(name):
             if line and not line.startswith("#"):
                 rows.append(line.split())
     return rows
+
+
+@pytest.fixture(scope="session")
+def nq():
+    """The CUDA library binding; a GPU test fails (never skips) without a device or the library."""
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("this test needs a CUDA device (B200)")
+    import rank_binary_factorization_b200 as lib
+    return lib
+
+
+def max_rel(x, ref):
+    """max |x - ref| / max |ref| (the reading of "max relative error" used for tensors)."""
+    import numpy as np
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.max(np.abs(ref))
+    return float(np.max(np.abs(x - ref)) / den) if den > 0 else float(np.max(np.abs(x)))

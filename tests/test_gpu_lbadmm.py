@@ -1,0 +1,266 @@
+"""GPU parity of LB-ADMM against the FP64 oracle (through the C ABI).
+
+Tolerances:
+  * single U (V) step on identical inputs: max|dX| / max|X_ref| <= 2e-3, same for S, a, b;
+    a sign of S may differ only where |S_ref| < 1e-3 rms(S_ref);
+  * packing on identical signs: bit-exact;
+  * end-to-end reconstruction error within 1% of the oracle's, per instance where the
+    iteration is insensitive to BF16-size perturbations, else within the range the oracle
+    itself spans under such perturbations.
+Inputs of the single-step tests are generated here (BF16-exact target and latent
+operand), imported into the GPU state, and fed unchanged to the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import max_rel
+from oracle import calib as OC
+from oracle import lbadmm as O
+from oracle.splitmix import sign_matrix
+from synth import gaussian_weight, planted_problem, stream_tensor
+
+pytestmark = pytest.mark.gpu
+TOL_STEP = 2e-3
+TOL_E2E = 0.01
+
+
+def bf16_exact(a):
+    return torch.as_tensor(np.asarray(a), dtype=torch.float32).to(torch.bfloat16).float().numpy()
+
+
+def unpack(t, r):
+    return O.unpack_signs(t.cpu().numpy().view(np.uint32), r)
+
+
+def test_v0_and_prepare_match_oracle(nq):
+    m, n, r = 300, 260, 20
+    W = gaussian_weight(3, "W", m, n, 0.02, 0.01, 10.0, torch.float32)
+    d_in = torch.exp(0.3 * torch.randn(n))
+    d_out = torch.exp(0.3 * torch.randn(m))
+    st = nq.LBState(m, n, r)
+    gamma = st.prepare(W.cuda(), d_in.cuda(), d_out.cuda(), seed=123)
+    Wt, What, g_ref = O.precondition(W.double().numpy(), d_in.double().numpy(),
+                                     d_out.double().numpy(), r)
+    assert abs(gamma - g_ref) / g_ref < 1e-6
+    V = st.field("V")[:, :r].cpu().double().numpy()
+    V0 = O.init_latent(n, r, 123)
+    np.testing.assert_array_equal(np.sign(V), np.sign(V0))
+    np.testing.assert_allclose(V, V0, rtol=1e-7)
+    Wh = st.field("WHAT")[:, :n].float().cpu().numpy()
+    ref = bf16_exact(What)
+    ulp = np.abs(ref) * 2.0 ** -7
+    assert np.all(np.abs(Wh - ref) <= ulp + 1e-30)
+    assert np.mean(Wh != ref) < 1e-3      # only rounding ties may move by one ulp
+
+
+@pytest.mark.parametrize("r", [1, 31, 32, 33, 100, 2032])
+def test_pack_signs_bit_exact(nq, r):
+    rng = np.random.default_rng(r)
+    X = rng.standard_normal((77, r)).astype(np.float32)
+    X[0, 0] = -0.0
+    X[1, :] = 0.0
+    X[2, :] = -1e-38
+    bits = nq.nq_pack_signs(torch.from_numpy(X).cuda())
+    np.testing.assert_array_equal(bits.cpu().numpy().view(np.uint32), O.pack_signs(X))
+
+
+def _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV):
+    st.field("WHAT")[:, :n].copy_(torch.from_numpy(Wh).to(torch.bfloat16).cuda())
+    for name, val in (("U", U), ("V", V), ("SU", SU), ("SV", SV)):
+        st.field(name)[:, :r].copy_(torch.from_numpy(val).float().cuda())
+    for name, val in (("AU", aU), ("BU", bU), ("AV", aV), ("BV", bV)):
+        st.field(name).copy_(torch.from_numpy(val).float().cuda())
+    st.sync_operands()
+
+
+def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4):
+    rng = np.random.default_rng(seed)
+    Wh = bf16_exact(rng.standard_normal((m, n)) * 0.1)
+    U = bf16_exact(rng.standard_normal((m, r)) * 0.2).astype(np.float64)
+    V = bf16_exact(rng.standard_normal((n, r)) * 0.2).astype(np.float64)
+    SU = rng.standard_normal((m, r)).astype(np.float32)
+    SV = rng.standard_normal((n, r)).astype(np.float32)
+    aU, aV = [np.abs(rng.standard_normal(k)).astype(np.float32) / np.sqrt(k) for k in (m, n)]
+    bU, bV = [np.abs(rng.standard_normal(r)).astype(np.float32) for _ in range(2)]
+    st = nq.LBState(m, n, r)
+    st.prepare(torch.zeros(m, n, device="cuda"), seed=0)
+    _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV)
+    st.half_step(side, rho, lam, K)
+    assert st.check_device_error() == 0
+    A = Wh.astype(np.float64) if side == 0 else Wh.astype(np.float64).T
+    Y = V if side == 0 else U
+    S0, a0, b0 = (SU, aU, bU) if side == 0 else (SV, aV, bV)
+    S0 = S0.astype(np.float64)
+    Z = O.sign_pm(S0) * np.outer(a0, b0)
+    Lam = S0 - Z
+    Xr, _, _, _ = O.latent_update(A, Y, Z, Lam, rho, lam)
+    Sr = Xr + Lam
+    _, ar, br = O.svid(Sr, K)
+    tag = "U" if side == 0 else "V"
+    X = st.field(tag)[:, :r].cpu().double().numpy()
+    S = st.field("S" + tag)[:, :r].cpu().double().numpy()
+    a = st.field("A" + tag).cpu().double().numpy()
+    b = st.field("B" + tag).cpu().double().numpy()
+    assert max_rel(X, Xr) <= TOL_STEP
+    assert max_rel(S, Sr) <= TOL_STEP
+    assert max_rel(a, ar) <= TOL_STEP
+    assert max_rel(b, br) <= TOL_STEP
+    flips = np.sign(S) != np.sign(Sr)
+    rms = np.sqrt(np.mean(Sr ** 2))
+    assert np.all(np.abs(Sr[flips]) < 1e-3 * rms)
+    # the transposed BF16 operand the other side will read
+    xt_ref = bf16_exact(Xr)
+    return max_rel(X, Xr), st, xt_ref
+
+
+@pytest.mark.parametrize("m,n,r", [(300, 200, 40), (1000, 777, 130), (520, 600, 300),
+                                   (129, 65, 1), (256, 512, 16), (700, 900, 257)])
+@pytest.mark.parametrize("side", [0, 1])
+def test_single_step_matches_oracle(nq, m, n, r, side):
+    _single_step_case(nq, m, n, r, side, seed=m + n + r + side)
+
+
+def test_single_step_full_size_q_proj(nq):
+    # Llama-2-7B q_proj shape at 1 BPW (4096 x 4096, r = 2032): both sides
+    for side in (0, 1):
+        err, _, _ = _single_step_case(nq, 4096, 4096, 2032, side, seed=7 + side)
+        assert err < TOL_STEP
+
+
+def test_planted_factors_recovered_on_gpu(nq):
+    p = planted_problem(0, noise=0.0)
+    res = nq.nq_lbadmm(p["W"].cuda(), 16, iters=100)
+    Us, Vs = unpack(res["U_packed"], 16), unpack(res["V_packed"], 16)
+    for got, planted in ((Us, p["U"].numpy()), (Vs, p["V"].numpy())):
+        M = np.abs(got.T @ planted) / got.shape[0]
+        assert np.all(M.max(axis=1) == 1.0)
+        assert len(set(M.argmax(axis=1).tolist())) == 16
+    assert res["rel_err"] <= 1e-3
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_planted_with_noise_end_to_end(nq, seed):
+    p = planted_problem(seed, noise=0.1)
+    res = nq.nq_lbadmm(p["W"].cuda(), 16, iters=30)
+    ref = O.lbadmm(p["W"].double().numpy(), r=16, iters=30)
+    assert abs(res["rel_err"] - ref.rel_err) <= TOL_E2E * ref.rel_err
+    # first objective value: identical start, differs only by arithmetic
+    assert abs(res["objective"][0] - ref.objective[0]) <= 1e-3 * ref.objective[0]
+
+
+def test_planted_config_with_preconditioners_within_oracle_spread(nq):
+    # The 256 x 512, r = 16 problem with calibration preconditioners is, at 30 iterations,
+    # sensitive to perturbations of BF16 size (the oracle itself moves by a few percent), so
+    # the GPU result is compared with the spread of oracle runs on inputs perturbed by
+    # relative noise of BF16 rounding size.
+    p = planted_problem(0, noise=0.1)
+    d_in, d_out, _, _ = nq.nq_calib_precond(p["acts"].cuda(), p["grads"].cuda())
+    res = nq.nq_lbadmm(p["W"].cuda(), 16, d_in, d_out, iters=30)
+    r_in, r_out, _, _ = OC.calib_precond([p["acts"].numpy()], [p["grads"].numpy()])
+    W = p["W"].double().numpy()
+    rng = np.random.default_rng(0)
+    ens = [O.lbadmm(W, r_in, r_out, r=16, iters=30).rel_err]
+    for _ in range(6):
+        Wp = W * (1 + 2.0 ** -9 * rng.uniform(-1, 1, W.shape))
+        Wt, _, _ = O.precondition(W, r_in, r_out, 16)
+        rp = O.lbadmm(Wp, r_in, r_out, r=16, iters=30)
+        ens.append(O.recon_error(Wt, rp.s1, O.sign_pm(rp.U), O.sign_pm(rp.V), rp.s2))
+    lo, hi = min(ens) * (1 - TOL_E2E), max(ens) * (1 + TOL_E2E)
+    assert lo <= res["rel_err"] <= hi, (res["rel_err"], ens)
+
+
+def test_random_layer_end_to_end_within_one_percent(nq):
+    # 2048 x 2048 BF16 layer with 1% outlier input columns, calibration streams of 8192
+    # tokens, 1 BPW (r = 1008), 20 iterations: large enough for the error to self-average.
+    m = n = 2048
+    r = 1008
+    W = gaussian_weight(5, "W", m, n, 0.02, 0.01, 10.0)
+    acts = stream_tensor(5, "acts", 8192, n)
+    grads = stream_tensor(5, "grads", 8192, m)
+    d_in, d_out, _, _ = nq.nq_calib_precond(acts.cuda(), grads.cuda())
+    res = nq.nq_lbadmm(W.cuda(), r, d_in, d_out, iters=20)
+    r_in, r_out, _, _ = OC.calib_precond([acts.float().numpy()], [grads.float().numpy()])
+    Wd = W.double().numpy()
+    ref = O.lbadmm(Wd, r_in, r_out, r=r, iters=20)
+    assert abs(res["rel_err"] - ref.rel_err) <= TOL_E2E * ref.rel_err, (res["rel_err"], ref.rel_err)
+    # Eckart-Young: no rank-r matrix beats the truncated SVD
+    Wt, _, _ = O.precondition(Wd, r_in, r_out, r)
+    sv = np.linalg.svd(Wt, compute_uv=False)
+    assert np.sum(sv[r:] ** 2) / np.sum(sv ** 2) <= res["rel_err"] ** 2
+    # the dedicated entry point agrees with the error nq_lbadmm reported
+    e2 = nq.nq_recon_error(W.cuda(), res["U_packed"], res["V_packed"], r, res["s1"], res["s2"],
+                           d_in, d_out)
+    assert abs(e2 - res["rel_err"]) <= 1e-5 * res["rel_err"]
+
+
+@pytest.mark.parametrize("m,n,r", [(257, 300, 33), (64, 1000, 7)])
+def test_recon_error_entry_matches_oracle(nq, m, n, r):
+    rng = np.random.default_rng(m)
+    W = rng.standard_normal((m, n)).astype(np.float32)
+    Us = sign_matrix(1, m, r)
+    Vs = sign_matrix(2, n, r)
+    s1 = np.exp(rng.standard_normal(m)).astype(np.float32)
+    s2 = np.exp(rng.standard_normal(n)).astype(np.float32) / r
+    d_in = np.exp(0.2 * rng.standard_normal(n)).astype(np.float32)
+    d_out = np.exp(0.2 * rng.standard_normal(m)).astype(np.float32)
+    Up = torch.from_numpy(O.pack_signs(Us).view(np.int32)).cuda()
+    Vp = torch.from_numpy(O.pack_signs(Vs).view(np.int32)).cuda()
+    e = nq.nq_recon_error(torch.from_numpy(W).cuda(), Up, Vp, r, torch.from_numpy(s1).cuda(),
+                          torch.from_numpy(s2).cuda(), torch.from_numpy(d_in).cuda(),
+                          torch.from_numpy(d_out).cuda())
+    Wt = (d_out[:, None].astype(np.float64) * W) * d_in[None, :]
+    ref = O.recon_error(Wt, s1.astype(np.float64), Us, Vs, s2.astype(np.float64))
+    assert abs(e - ref) <= 1e-5 * ref
+
+
+def test_zero_weight_is_a_fixed_point(nq):
+    res = nq.nq_lbadmm(torch.zeros(200, 100, device="cuda"), 8, iters=3)
+    assert res["rel_err"] == 0.0
+    assert torch.all(res["s1"] == 0) and torch.all(res["s2"] == 0)
+    assert torch.all(res["U_packed"] == 0) and torch.all(res["V_packed"] == 0)
+    assert all(o == 0.0 for o in res["objective"])
+
+
+def test_nonfinite_weight_is_reported(nq):
+    W = torch.randn(128, 96)
+    W[5, 7] = float("inf")
+    with pytest.raises(nq.NQError) as e:
+        nq.nq_lbadmm(W.cuda(), 8, iters=2)
+    assert e.value.code == 4
+
+
+def test_runs_are_bit_identical(nq):
+    W = gaussian_weight(9, "W", 640, 384, dtype=torch.bfloat16).cuda()
+    a = nq.nq_lbadmm(W, 96, iters=5)
+    b = nq.nq_lbadmm(W, 96, iters=5)
+    assert torch.equal(a["U_packed"], b["U_packed"]) and torch.equal(a["V_packed"], b["V_packed"])
+    assert torch.equal(a["s1"], b["s1"]) and torch.equal(a["s2"], b["s2"])
+    assert a["objective"] == b["objective"] and a["rel_err"] == b["rel_err"]
+
+
+def test_full_size_q_proj_pipeline_properties(nq):
+    # The bench workload: 4096 x 4096 BF16 q_proj with 1% x10 outlier columns, 262144-token
+    # act/grad streams, r = 2032 (1 BPW), 100 iterations.  The oracle cannot run 100
+    # iterations at this size within a test; checked here: Eckart-Young, agreement of the
+    # two error paths, a decreasing objective, and balanced-scale consistency.
+    m = n = 4096
+    r = nq.nq_rank_for_bpw(m, n, 1.0)
+    assert r == 2032
+    W = gaussian_weight(0, "W", m, n, 0.02, 0.01, 10.0).cuda()
+    acts = stream_tensor(0, "acts", 262144, n).cuda()
+    grads = stream_tensor(0, "grads", 262144, m).cuda()
+    d_in, d_out, _, _ = nq.nq_calib_precond(acts, grads)
+    del acts, grads
+    res = nq.nq_lbadmm(W, r, d_in, d_out, iters=100)
+    e = res["rel_err"]
+    obj = res["objective"]
+    assert np.isfinite(e) and 0 < e < 1
+    assert obj[-1] < obj[0]
+    Wt = (d_out.double()[:, None] * W.double() * d_in.double()[None, :]).cpu().numpy()
+    ev = np.linalg.eigvalsh(Wt.T @ Wt)[::-1]
+    assert np.sum(ev[r:]) / np.sum(ev) <= e ** 2
+    e2 = nq.nq_recon_error(W, res["U_packed"], res["V_packed"], r, res["s1"], res["s2"],
+                           d_in, d_out)
+    assert abs(e2 - e) <= 1e-5 * e
+    assert torch.all(res["s1"] > 0) and torch.all(res["s2"] > 0)
