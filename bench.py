@@ -382,7 +382,15 @@ def main():
     ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["q_proj", "profile"], default="q_proj",
+                    help="profile: the same layer with 65536-token streams and 2 iterations, "
+                         "the small case used for ncu section captures")
     args = ap.parse_args()
+    if args.workload == "profile":
+        WORKLOAD.update(T=65536, name="profiling case: q_proj 4096x4096 bf16, r=2032, "
+                                      "2 x 65536x4096 bf16 streams")
+        if args.iters == WORKLOAD["iters"]:
+            args.iters = 2
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
