@@ -99,6 +99,24 @@ nq_status nq_calib_stats(const void *X, int64_t T, int64_t C, nq_dtype dt, doubl
                          void *ws, size_t ws_bytes, nq_stream_t stream);
 
 /*
+ * nq_calib_stats without a workspace.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory or pass a workspace -- a plugin
+ * inside a host program that owns the device memory pool and refuses new allocations,
+ * a process whose device-memory budget is fixed at launch, or a path that must not call
+ * cudaMalloc / cudaFree because they may synchronise the device.
+ * Same arguments, arithmetic and results as nq_calib_stats.  Its scratch is a fixed
+ * 4 MiB array inside the library image, held on every GPU that loads the library until
+ * the process exits.  Limit: C <= 32768 channels (any T); larger C returns
+ * NQ_ERR_UNSUPPORTED.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before any
+ * stream capture.  All calls share the array, so calls whose GPU work may overlap
+ * (other streams, other threads) race and must be ordered by the caller.  Nothing in the
+ * array needs clearing between calls.  Allocates nothing.  Enqueue only.
+ */
+nq_status nq_calib_stats_noalloc(const void *X, int64_t T, int64_t C, nq_dtype dt, double *s,
+                                 double *q, nq_stream_t stream);
+
+/*
  * Diagonal preconditioners from the activation stream (T_in x n) and the output
  * gradient stream (T_out x m):
  *     mu = mean(s), delta^2 = sum_j (s_j - mu)^2, beta_bar^2 = (1/T) sum_j (q_j - s_j^2),

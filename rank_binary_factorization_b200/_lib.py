@@ -34,6 +34,7 @@ SIGNATURES = {
     "nq_rank_for_bpw": (c_i32, [c_i64, c_i64, c_f64]),
     "nq_calib_workspace_size": (c_sz, [c_i64, c_i64]),
     "nq_calib_stats": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "nq_calib_stats_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp]),
     "nq_calib_precond": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_i32, c_f64, c_vp,
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
