@@ -367,6 +367,7 @@ nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, co
     ep.part = lb.p<double>(L.part);
     ep.W = W;
     ep.w_bf16 = bf16;
+    ep.w_vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) && ((L.n * (bf16 ? 2 : 4)) % 16 == 0);
     ep.ldw = L.n;
     ep.d_in = d_in;
     ep.d_out = d_out;
@@ -618,6 +619,7 @@ nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const
     ep.part = part;
     ep.W = W;
     ep.w_bf16 = dt == NQ_BF16;
+    ep.w_vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) && ((n * (dt == NQ_BF16 ? 2 : 4)) % 16 == 0);
     ep.ldw = n;
     ep.d_in = d_in;
     ep.d_out = d_out;

@@ -44,30 +44,35 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Grid-wide barrier for kernels launched cooperatively (all CTAs co-resident).
 // ``bar`` points at two words: [0] arrival count, [1] generation.  Bounded: a
 // barrier that does not complete within the spin budget raises NQ_ERR_TIMEOUT and
-// lets the CTA continue (results are then garbage but nothing hangs).
+// lets the CTA continue (results are then garbage but nothing hangs); after a
+// timeout every later barrier is skipped, so at most one budget is spent.
 __device__ __forceinline__ void grid_barrier(unsigned int *bar, int *err) {
     __syncthreads();
-    // after a timeout every later barrier is skipped, so at most one budget is spent
     if (threadIdx.x == 0 && !(err && *(volatile int *)err == NQ_ERR_TIMEOUT)) {
-        volatile unsigned int *vgen = bar + 1;
-        unsigned int gen = *vgen;
+        const unsigned int gen = ld_acquire_gpu(bar + 1);
         __threadfence();
-        unsigned int arrived = atomicAdd(bar, 1u) + 1u;
+        const unsigned int arrived = atomicAdd(bar, 1u) + 1u;
         if (arrived == gridDim.x * gridDim.y * gridDim.z) {
             atomicExch(bar, 0u);
             __threadfence();
             atomicAdd(bar + 1, 1u);
         } else {
             uint32_t spins = 0;
-            while (*vgen == gen) {
+            while (ld_acquire_gpu(bar + 1) == gen) {
                 if (++spins > kGridSpinLimit) {
                     raise_error(err, NQ_ERR_TIMEOUT);
                     break;
                 }
-                __nanosleep(32);
+                if (spins > 256) __nanosleep(32);
             }
         }
         __threadfence();

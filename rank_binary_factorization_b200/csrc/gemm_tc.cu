@@ -107,6 +107,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Named barrier among the epilogue warps only (barrier 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_bar() {
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");
+}
+
 // ---------------------------------------------------------------------------------
 // Epilogues: thread owns tile row ``row`` and columns col0 .. col0+15.
 // ---------------------------------------------------------------------------------
@@ -118,15 +127,40 @@ __device__ __forceinline__ float load_w(const EpiParams &p, int64_t i, int64_t j
     return reinterpret_cast<const float *>(p.W)[i * p.ldw + j];
 }
 
+__device__ __forceinline__ void ld16(float (&d)[16], const float *src) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4 *>(&d[j]) = *reinterpret_cast<const float4 *>(src + j);
+}
+__device__ __forceinline__ void st16(float *dst, const float (&v)[16]) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4 *>(dst + j) = *reinterpret_cast<const float4 *>(&v[j]);
+}
+__device__ __forceinline__ void ld16_bf16(float (&d)[16], const __nv_bfloat16 *src) {
+    __align__(16) __nv_bfloat16 h[16];
+    reinterpret_cast<uint4 *>(h)[0] = reinterpret_cast<const uint4 *>(src)[0];
+    reinterpret_cast<uint4 *>(h)[1] = reinterpret_cast<const uint4 *>(src)[1];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) d[j] = __bfloat162float(h[j]);
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int col0,
                                                const float (&v)[16], float &acc_sum) {
     const bool full = (col0 + 16 <= p.N);
     if constexpr (EPI == EPI_GRAM) {
         float *o = p.out + (int64_t)row * p.ldo + col0;
+        float w[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (full || col0 + j < p.N) o[j] = v[j] + ((row == col0 + j) ? p.diag : 0.f);
+        for (int j = 0; j < 16; ++j) w[j] = v[j] + ((row == col0 + j) ? p.diag : 0.f);
+        if (full && (p.ldo & 3) == 0) {
+            st16(o, w);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (full || col0 + j < p.N) o[j] = w[j];
+        }
     } else if constexpr (EPI == EPI_RHS) {
         const float ai = p.a[row];
         const float *Srow = p.S + (int64_t)row * p.ldf + col0;
@@ -134,12 +168,8 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
         __nv_bfloat16 *lo = p.Rlo + (int64_t)row * p.ldr + col0;
         if (full) {
             float s[16], bb[16];
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                *reinterpret_cast<float4 *>(&s[j]) = *reinterpret_cast<const float4 *>(Srow + j);
-                *reinterpret_cast<float4 *>(&bb[j]) =
-                    *reinterpret_cast<const float4 *>(p.b + col0 + j);
-            }
+            ld16(s, Srow);
+            ld16(bb, p.b + col0);
             __align__(16) __nv_bfloat16 h[16], l[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -168,20 +198,45 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
         float *Xrow = p.X + (int64_t)row * p.ldf + col0;
         bool bad = false;
         float part = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            if (!(full || col0 + j < p.N)) continue;
-            const float x = v[j];
-            bad |= !isfinite(x);
-            const float sold = Srow[j];
-            const float z = sgn(sold) * ai * p.b[col0 + j];
-            Xrow[j] = x;
-            Srow[j] = x + sold - z;
-            p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = __float2bfloat16_rn(x);
+        if (full) {
+            float so[16], bb[16], sn[16], rr[16];
+            ld16(so, Srow);
+            ld16(bb, p.b + col0);
             if (p.objective) {
-                const int64_t o = (int64_t)row * p.ldr + col0 + j;
-                const float r = __bfloat162float(p.Rhi[o]) + __bfloat162float(p.Rlo[o]);
-                part += (r - p.rho * (2.f * z - sold)) * x;
+                float lo_[16];
+                const int64_t o = (int64_t)row * p.ldr + col0;
+                ld16_bf16(rr, p.Rhi + o);
+                ld16_bf16(lo_, p.Rlo + o);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) rr[j] += lo_[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float x = v[j];
+                bad |= !isfinite(x);
+                const float z = sgn(so[j]) * ai * bb[j];
+                sn[j] = x + so[j] - z;
+                if (p.objective) part += (rr[j] - p.rho * (2.f * z - so[j])) * x;
+            }
+            st16(Xrow, v);
+            st16(Srow, sn);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = __float2bfloat16_rn(v[j]);
+        } else {
+            for (int j = 0; j < 16 && col0 + j < p.N; ++j) {
+                const float x = v[j];
+                bad |= !isfinite(x);
+                const float sold = Srow[j];
+                const float z = sgn(sold) * ai * p.b[col0 + j];
+                Xrow[j] = x;
+                Srow[j] = x + sold - z;
+                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = __float2bfloat16_rn(x);
+                if (p.objective) {
+                    const int64_t o = (int64_t)row * p.ldr + col0 + j;
+                    const float r = __bfloat162float(p.Rhi[o]) + __bfloat162float(p.Rlo[o]);
+                    part += (r - p.rho * (2.f * z - sold)) * x;
+                }
             }
         }
         if (bad) raise_error(p.err, NQ_ERR_NONFINITE);
@@ -189,12 +244,22 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
     } else if constexpr (EPI == EPI_RECON) {
         const float dro = p.d_out ? p.d_out[row] : 1.f;
         const float s1 = p.s1[row];
+        float w[16];
+        if (full && p.w_vec) {
+            if (p.w_bf16)
+                ld16_bf16(w, reinterpret_cast<const __nv_bfloat16 *>(p.W) + (int64_t)row * p.ldw + col0);
+            else
+                ld16(w, reinterpret_cast<const float *>(p.W) + (int64_t)row * p.ldw + col0);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = (full || col0 + j < p.N) ? load_w(p, row, col0 + j) : 0.f;
+        }
         float part = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int c = col0 + j;
             if (!(full || c < p.N)) continue;
-            const float wt = dro * load_w(p, row, c) * (p.d_in ? p.d_in[c] : 1.f);
+            const float wt = dro * w[j] * (p.d_in ? p.d_in[c] : 1.f);
             const float d = wt - s1 * v[j] * p.s2[c];
             part += d * d;
         }
@@ -203,28 +268,31 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
 }
 
 // ---------------------------------------------------------------------------------
-// The kernel
+// The kernel: persistent, one CTA per SM, tiles assigned round-robin (m fastest, so
+// consecutive CTAs share the B tile).  Two TMEM accumulator stages let the epilogue
+// of one tile run while the MMAs of the next are issued.
 // ---------------------------------------------------------------------------------
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ Maps maps, const EpiParams p) {
     constexpr int B_TILE_BYTES = BN * BK * 2;
     constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
-    constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+    constexpr uint32_t TMEM_COLS = 2 * BN;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *empty_bar = full_bar + STAGES;
-    uint64_t *acc_bar = empty_bar + STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
-    __shared__ double red[kEpiWarps];
+    uint64_t *tfull = empty_bar + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    __shared__ double red[2][kEpiWarps];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BM;
-    const int n0 = blockIdx.y * BN;
+    const int num_m = (int)ceil_div(p.M, BM);
+    const int num_tiles = num_m * (int)ceil_div(p.N, BN);
     const int total_kb = p.kblocks[0] + (p.nseg > 1 ? p.kblocks[1] : 0) +
                          (p.nseg > 2 ? p.kblocks[2] : 0);
 
@@ -233,7 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(acc_bar, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&tfull[s], 1);
+            mbar_init(&tempty[s], kEpiWarps);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -251,72 +322,104 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // TMA producer
-            for (int kb = 0; kb < total_kb; ++kb) {
-                const int s = kb % STAGES;
-                if (kb >= STAGES && !mbar_wait(&empty_bar[s], ((kb / STAGES) - 1) & 1, p.err))
-                    break;
-                int seg = 0, k = kb;
-                while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
-                uint8_t *a_dst = smem + s * STAGE_BYTES;
-                uint8_t *b_dst = a_dst + A_TILE_BYTES;
-                mbar_expect_tx(&full_bar[s], STAGE_BYTES);
-                tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
-                tma_load_2d(b_dst, &maps.b[seg], k * BK, n0, &full_bar[s]);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+                for (int kb = 0; kb < total_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES &&
+                        !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    int seg = 0, k = kb;
+                    while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                    uint8_t *a_dst = smem + s * STAGE_BYTES;
+                    mbar_expect_tx(&full_bar[s], STAGE_BYTES);
+                    tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
+                    tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0, &full_bar[s]);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // MMA issuer
             constexpr uint32_t idesc = instr_desc_bf16(BM, BN);
+            uint32_t it = 0;
             bool ok = true;
-            for (int kb = 0; kb < total_kb; ++kb) {
-                const int s = kb % STAGES;
-                if (!mbar_wait(&full_bar[s], (kb / STAGES) & 1, p.err)) {
-                    ok = false;
-                    break;
-                }
+            int lt = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+                const int as = lt & 1;
+                if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, p.err)) break;
                 tc_fence_after();
-                const uint8_t *a_src = smem + s * STAGE_BYTES;
-                const uint64_t adesc = smem_desc_sw128(a_src);
-                const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
+                const uint32_t d = tmem + (uint32_t)(as * BN);
+                for (int kb = 0; kb < total_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t *a_src = smem + s * STAGE_BYTES;
+                    const uint64_t adesc = smem_desc_sw128(a_src);
+                    const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
-                    mma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
-                mma_commit(&empty_bar[s]);
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit(&empty_bar[s]);
+                }
+                if (ok) mma_commit(&tfull[as]);
             }
-            if (ok) mma_commit(acc_bar);
         }
     } else {
-        // epilogue warps
+        // epilogue warps.  Every epilogue warp walks the same tiles and reaches the same
+        // named barriers, also after a timed-out wait (then it only skips the work).
         const int q = warp & 3;
-        const int row = m0 + 32 * q + lane;
-        float acc_sum = 0.f;
-        // one lane waits; the outcome is broadcast so that the warp-collective
-        // tcgen05.ld below is executed by all 32 lanes or by none
-        int ok = 0;
-        if (lane == 0) ok = mbar_wait(acc_bar, 0, p.err) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
-            tc_fence_after();
-            const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16);
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
-                tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
-                if (row < p.M && n0 + c < p.N) epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
+        int lt = 0;
+        bool dead = false;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+            const int as = lt & 1;
+            const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+            const int row = m0 + 32 * q + lane;
+            float acc_sum = 0.f;
+            if (!dead) {
+                // one lane waits; the outcome is broadcast so that the warp-collective
+                // tcgen05.ld below is executed by all 32 lanes or by none
+                int ok = 0;
+                if (lane == 0) ok = mbar_wait(&tfull[as], (lt >> 1) & 1, p.err) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                dead = !ok;
             }
-        }
-        if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
-            double w = warp_sum((double)acc_sum);
-            if (lane == 0) red[warp - 2] = w;
+            if (!dead) {
+                tc_fence_after();
+                const uint32_t tbase = tmem + (uint32_t)(as * BN) + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
+                    if (row < p.M && n0 + c < p.N) epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[as]);
+            }
+            if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
+                if (p.part && (EPI == EPI_RECON || p.objective)) {
+                    const double w = warp_sum((double)acc_sum);
+                    if (lane == 0) red[as][warp - 2] = w;
+                    epilogue_bar();
+                    if (warp == 2 && lane == 0) {
+                        double t = 0.0;
+                        for (int e = 0; e < kEpiWarps; ++e) t += red[as][e];
+                        p.part[tile] = t;
+                    }
+                }
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
-        if (threadIdx.x == 0 && p.part && (EPI == EPI_RECON || p.objective))
-            p.part[blockIdx.y * gridDim.x + blockIdx.x] = red[0] + red[1] + red[2] + red[3];
-    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -359,7 +462,7 @@ bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t col
 
 template <int BN, int STAGES, int EPI>
 static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s) {
-    constexpr int smem = STAGES * (A_TILE_BYTES + BN * BK * 2) + 1024 + 256;
+    constexpr int smem = STAGES * (A_TILE_BYTES + BN * BK * 2) + 1024 + 256;  // + barriers
     auto kern = gemm_kernel<BN, STAGES, EPI>;
     static bool configured = false;
     if (!configured) {
@@ -367,7 +470,15 @@ static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    dim3 grid((unsigned)ceil_div(p.M, BM), (unsigned)ceil_div(p.N, BN));
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms < 1) sms = kNumSMsB200;
+    }
+    const int64_t tiles = num_tiles(p.M, p.N, BN);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     kern<<<grid, kThreads, smem, s>>>(maps, p);
     count_launch();
     return cudaGetLastError();

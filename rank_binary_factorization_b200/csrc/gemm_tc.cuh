@@ -2,10 +2,11 @@
 //
 // D[M x N] = sum over K-segments s of A_s[M x K_s] . B_s[N x K_s]^T, all operands BF16
 // and K-major (row-major with K contiguous), accumulation FP32 in tensor memory.
-// One CTA computes one 128 x BN tile:
+// Persistent: one CTA per SM walks 128 x BN output tiles round-robin.  Per CTA:
 //   warp 0     one elected thread issues TMA tile loads into a STAGES-deep ring
-//   warp 1     allocates TMEM; one elected thread issues tcgen05.mma (M=128, N=BN,
-//              K=16 per instruction, 4 per 64-wide K block) and commits to mbarriers
+//   warp 1     allocates TMEM (two accumulator stages of BN columns); one elected thread
+//              issues tcgen05.mma (M=128, N=BN, K=16 per instruction, 4 per 64-wide K
+//              block) and commits to mbarriers
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes
 //              32*(w%4) .. +31, i.e. those tile rows), fused element-wise work, stores
 // Every mbarrier wait is bounded; a wait that runs out raises NQ_ERR_TIMEOUT.
@@ -57,6 +58,7 @@ struct EpiParams {
     // EPI_RECON: sum_ij (d_out_i W_ij d_in_j - s1_i acc s2_j)^2
     const void *W;
     int w_bf16;
+    int w_vec;                 // W rows 16-byte aligned: vector loads in the epilogue
     int64_t ldw;
     const float *d_in, *d_out, *s1, *s2;
 };

@@ -1,5 +1,5 @@
 // SIMT kernels of the NanoQuant hot path (sm_100a): calibration reduction, target
-// preparation, V_0, blocked Cholesky + inverse, SVID power passes, objective,
+// preparation, V_0, SVID power passes, objective,
 // balancing / scale extraction / sign packing.
 #include <cooperative_groups.h>
 
@@ -452,281 +452,22 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 }
 
 // =================================================================================
-// Cholesky G = L L^T and G^-1 = L^-T L^-1 (FP32, 32 x 32 tiles, one cooperative
-// launch with bounded grid barriers).  Same page, "Core method" (核心方法), step (a):
-// the regularised linear system of the U (V) step is solved through a Cholesky
-// factorisation.
-// =================================================================================
-constexpr int CT = 32;
-
-struct CholArgs {
-    const float *G;
-    int r;
-    int64_t rp;
-    float *A;
-    float *Li;
-    __nv_bfloat16 *hi, *lo;
-    int64_t ldr;
-    int *err;
-    unsigned int *bar;
-};
-
-__device__ __forceinline__ void load_tile(float (*dst)[CT + 1], const float *M, int64_t ld,
-                                          int ti, int tj) {
-    for (int e = threadIdx.x; e < CT * CT; e += blockDim.x) {
-        const int i = e >> 5, j = e & 31;
-        // L2-coherent load: tiles are rewritten by other CTAs between grid barriers
-        dst[i][j] = __ldcg(M + ((int64_t)ti * CT + i) * ld + (int64_t)tj * CT + j);
-    }
-}
-__device__ __forceinline__ void store_tile(float *M, int64_t ld, int ti, int tj,
-                                           const float (*src)[CT + 1]) {
-    for (int e = threadIdx.x; e < CT * CT; e += blockDim.x) {
-        const int i = e >> 5, j = e & 31;
-        M[((int64_t)ti * CT + i) * ld + (int64_t)tj * CT + j] = src[i][j];
-    }
-}
-
-// acc[q] += sum_c X(a, c) Y(c, b0+q) with X(a,c) = TX ? X[c][a] : X[a][c] and
-// Y(c,b) = TY ? Y[b][c] : Y[c][b]; thread owns row a = tid/8, columns b0 = 4*(tid%8).
-template <bool TX, bool TY>
-__device__ __forceinline__ void tile_mac(float (&acc)[4], const float (*X)[CT + 1],
-                                         const float (*Y)[CT + 1], int c_begin = 0,
-                                         int c_end = CT) {
-    const int a = threadIdx.x >> 3, b0 = (threadIdx.x & 7) * 4;
-    for (int c = c_begin; c < c_end; ++c) {
-        const float x = TX ? X[c][a] : X[a][c];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] = fmaf(x, TY ? Y[b0 + q][c] : Y[c][b0 + q], acc[q]);
-    }
-}
-
-__global__ void __launch_bounds__(256) chol_inv_kernel(CholArgs p) {
-    __shared__ float t0[CT][CT + 1], t1[CT][CT + 1], t2[CT][CT + 1];
-    const int nb = (int)(p.rp / CT);
-    const int64_t rp = p.rp;
-    const int a_row = threadIdx.x >> 3, b_col = (threadIdx.x & 7) * 4;
-
-    // phase 0: A = G padded with the identity, Li = 0
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rp * rp;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t i = e / rp, j = e % rp;
-        p.A[e] = (i < p.r && j < p.r) ? p.G[i * p.r + j] : (i == j ? 1.f : 0.f);
-        p.Li[e] = 0.f;
-    }
-    grid_barrier(p.bar, p.err);
-
-    for (int j = 0; j < nb; ++j) {
-        // (a) diagonal tile: L_jj (lower) and its inverse, by CTA 0 / warp 0
-        if (blockIdx.x == 0) {
-            load_tile(t0, p.A, rp, j, j);
-            __syncthreads();
-            if (threadIdx.x < 32) {
-                const int lane = threadIdx.x;
-                for (int k = 0; k < CT; ++k) {
-                    __syncwarp();
-                    float piv = t0[k][k];
-                    if (!(piv > 0.f)) {
-                        if (lane == 0) raise_error(p.err, NQ_ERR_NOT_SPD);
-                        piv = 1e-30f;
-                    }
-                    const float l = sqrtf(piv);
-                    __syncwarp();
-                    if (lane == k) t0[k][k] = l;
-                    if (lane > k) t0[lane][k] /= l;
-                    __syncwarp();
-                    if (lane > k) {
-                        const float lik = t0[lane][k];
-                        for (int jj = k + 1; jj <= lane; ++jj) t0[lane][jj] -= lik * t0[jj][k];
-                    }
-                }
-                __syncwarp();
-                // column ``lane`` of L_jj^-1 by forward substitution
-                for (int i = 0; i < CT; ++i) t1[i][lane] = 0.f;
-                t1[lane][lane] = 1.f / t0[lane][lane];
-                for (int i = lane + 1; i < CT; ++i) {
-                    float s = 0.f;
-                    for (int k = lane; k < i; ++k) s = fmaf(t0[i][k], t1[k][lane], s);
-                    t1[i][lane] = -s / t0[i][i];
-                }
-                __syncwarp();
-                for (int i = 0; i < CT; ++i)
-                    if (lane > i) t0[i][lane] = 0.f;  // clear the strict upper triangle
-            }
-            __syncthreads();
-            store_tile(p.A, rp, j, j, t0);
-            store_tile(p.Li, rp, j, j, t1);
-        }
-        grid_barrier(p.bar, p.err);
-
-        // (b) panel: L_ij = A_ij L_jj^-T
-        for (int i = j + 1 + blockIdx.x; i < nb; i += gridDim.x) {
-            load_tile(t0, p.A, rp, i, j);
-            load_tile(t1, p.Li, rp, j, j);
-            __syncthreads();
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            tile_mac<false, true>(acc, t0, t1);
-            __syncthreads();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) t2[a_row][b_col + q] = acc[q];
-            __syncthreads();
-            store_tile(p.A, rp, i, j, t2);
-            __syncthreads();
-        }
-        grid_barrier(p.bar, p.err);
-
-        // (c) trailing update: A_ik -= L_ij L_kj^T for j < k <= i
-        const int T = nb - 1 - j;
-        const int64_t ntl = (int64_t)T * (T + 1) / 2;
-        for (int64_t idx = blockIdx.x; idx < ntl; idx += gridDim.x) {
-            // lower-triangular enumeration: ii >= kk
-            int ii = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
-            while ((int64_t)(ii + 1) * (ii + 2) / 2 <= idx) ++ii;
-            while ((int64_t)ii * (ii + 1) / 2 > idx) --ii;
-            const int kk = (int)(idx - (int64_t)ii * (ii + 1) / 2);
-            const int i = j + 1 + ii, k = j + 1 + kk;
-            load_tile(t0, p.A, rp, i, j);
-            load_tile(t1, p.A, rp, k, j);
-            load_tile(t2, p.A, rp, i, k);
-            __syncthreads();
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            tile_mac<false, true>(acc, t0, t1);
-            __syncthreads();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) t2[a_row][b_col + q] -= acc[q];
-            __syncthreads();
-            store_tile(p.A, rp, i, k, t2);
-            __syncthreads();
-        }
-        grid_barrier(p.bar, p.err);
-    }
-
-    // Inverse of L by recursive doubling over tile blocks: for a pair of diagonal
-    // blocks [[L11, 0], [L21, L22]] with known inverses, (L^-1)_21 = -L22^-1 L21 L11^-1.
-    // T = L21 L11^-1 is kept, tile (a, b), in the unused upper tile (b, a) of Li.
-    for (int s = 1; s < nb; s *= 2) {
-        const int npairs = (int)ceil_div(nb, 2 * s);
-        // step 1: T(a, b) = sum_{c >= b} L21(a, c) Li11(c, b)
-        {
-            int64_t jobs = (int64_t)npairs * s * s;
-            for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
-                const int pr = (int)(q / (s * s));
-                const int a = 2 * pr * s + s + (int)((q % (s * s)) / s);
-                const int b = 2 * pr * s + (int)(q % s);
-                const int top_end = 2 * pr * s + s;
-                if (a >= nb) continue;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int c = b; c < top_end; ++c) {
-                    load_tile(t0, p.A, rp, a, c);
-                    load_tile(t1, p.Li, rp, c, b);
-                    __syncthreads();
-                    tile_mac<false, false>(acc, t0, t1);
-                    __syncthreads();
-                }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) t2[a_row][b_col + qq] = acc[qq];
-                __syncthreads();
-                store_tile(p.Li, rp, b, a, t2);
-                __syncthreads();
-            }
-        }
-        grid_barrier(p.bar, p.err);
-        // step 2: Li21(a, b) = -sum_{bot0 <= c <= a} Li22(a, c) T(c, b)
-        {
-            int64_t jobs = (int64_t)npairs * s * s;
-            for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
-                const int pr = (int)(q / (s * s));
-                const int bot0 = 2 * pr * s + s;
-                const int a = bot0 + (int)((q % (s * s)) / s);
-                const int b = 2 * pr * s + (int)(q % s);
-                if (a >= nb) continue;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int c = bot0; c <= a; ++c) {
-                    load_tile(t0, p.Li, rp, a, c);
-                    load_tile(t1, p.Li, rp, b, c);  // T(c, b) lives at tile (b, c)
-                    __syncthreads();
-                    tile_mac<false, false>(acc, t0, t1);
-                    __syncthreads();
-                }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) t2[a_row][b_col + qq] = -acc[qq];
-                __syncthreads();
-                store_tile(p.Li, rp, a, b, t2);
-                __syncthreads();
-            }
-        }
-        grid_barrier(p.bar, p.err);
-    }
-
-    // G^-1 = Li^T Li: tile (a, b), a >= b: sum_{c >= a} Li(c, a)^T Li(c, b); split into
-    // bf16 hi + lo and written to both (a, b) and (b, a).
-    const int64_t ngi = (int64_t)nb * (nb + 1) / 2;
-    for (int64_t idx = blockIdx.x; idx < ngi; idx += gridDim.x) {
-        int a = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
-        while ((int64_t)(a + 1) * (a + 2) / 2 <= idx) ++a;
-        while ((int64_t)a * (a + 1) / 2 > idx) --a;
-        const int b = (int)(idx - (int64_t)a * (a + 1) / 2);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c = a; c < nb; ++c) {
-            load_tile(t0, p.Li, rp, c, a);
-            load_tile(t1, p.Li, rp, c, b);
-            __syncthreads();
-            tile_mac<true, false>(acc, t0, t1);
-            __syncthreads();
-        }
-        const int64_t gi = (int64_t)a * CT + a_row;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t gj = (int64_t)b * CT + b_col + q;
-            if (gi < p.r && gj < p.r) {
-                const __nv_bfloat16 h = __float2bfloat16_rn(acc[q]);
-                const __nv_bfloat16 l = __float2bfloat16_rn(acc[q] - __bfloat162float(h));
-                p.hi[gi * p.ldr + gj] = h;
-                p.lo[gi * p.ldr + gj] = l;
-                p.hi[gj * p.ldr + gi] = h;
-                p.lo[gj * p.ldr + gi] = l;
-            }
-        }
-    }
-}
-
-cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
-                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr, int *err,
-                         unsigned int *bar, cudaStream_t s) {
-    static int grid = 0;
-    if (!grid) {
-        int per_sm = 0;
-        cudaError_t e =
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chol_inv_kernel, 256, 0);
-        if (e != cudaSuccess) return e;
-        int dev = 0, sms = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        grid = sms * (per_sm < 2 ? per_sm : 2);
-        if (grid < 1) return cudaErrorLaunchOutOfResources;
-    }
-    cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
-    if (e != cudaSuccess) return e;
-    CholArgs args{G, r, rp, A, Li, Gi_hi, Gi_lo, ldr, err, bar};
-    void *params[] = {&args};
-    count_launch();
-    return cudaLaunchCooperativeKernel((const void *)chol_inv_kernel, dim3(grid), dim3(256),
-                                       params, 0, s);
-}
-
-// =================================================================================
 // SVID power steps.  Same page, "Core method", step (b): the continuous U is mapped
 // to the binary proxy Z = sign(S) * a b^T, a b^T the rank-1 fit of |S| by K power
 // steps from b = 1.  One pass over S per power step: t = |S| b row by row and
 // b' = |S|^T t / ||t|| column by column, from the same shared-memory copy of S.
 // =================================================================================
+// One CTA tile = kSvidRows rows of |S| staged in shared memory with 16-byte loads; warp w
+// forms the row dot t_w = |S_w.| b, then every thread accumulates its columns' share of
+// |S|^T t.  Small tiles keep several CTAs per SM in flight (the loads of one overlap the
+// arithmetic of another).  Partial sums per CTA go to partb / partn (fixed order).
 __global__ void __launch_bounds__(256)
     svid_pass_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
                      const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
                      double *partn) {
-    extern __shared__ float sm[];
-    float *sA = sm;                      // kSvidRows x r
-    float *sb = sm + kSvidRows * r;      // r
+    extern __shared__ __align__(16) float sm[];
+    float *sA = sm;                      // kSvidRows x ldf
+    float *sb = sm + kSvidRows * ldf;    // r
     __shared__ float st[kSvidRows];
     __shared__ double sn[kSvidRows];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -735,19 +476,29 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int u = 0; u < 16; ++u) acc[u] = 0.f;
     double nacc = 0.0;
+    const int r4 = r >> 2;
     const int64_t ntile = ceil_div(rows, kSvidRows);
     for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
         const int64_t row0 = tile * kSvidRows;
         __syncthreads();
-        for (int w = 0; w < kSvidRows; ++w) {
+        // rows x r4 float4 loads, then the scalar tail
+        for (int e = threadIdx.x; e < kSvidRows * r4; e += blockDim.x) {
+            const int w = e / r4, k4 = e - w * r4;
             const int64_t i = row0 + w;
-            for (int k = threadIdx.x; k < r; k += blockDim.x)
-                sA[w * r + k] = i < rows ? fabsf(S[i * ldf + k]) : 0.f;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < rows) v = __ldcg(reinterpret_cast<const float4 *>(S + i * ldf) + k4);
+            *reinterpret_cast<float4 *>(sA + w * ldf + 4 * k4) =
+                make_float4(fabsf(v.x), fabsf(v.y), fabsf(v.z), fabsf(v.w));
+        }
+        for (int e = threadIdx.x; e < kSvidRows * (r - 4 * r4); e += blockDim.x) {
+            const int w = e / (r - 4 * r4), k = 4 * r4 + e % (r - 4 * r4);
+            const int64_t i = row0 + w;
+            sA[w * ldf + k] = i < rows ? fabsf(S[i * ldf + k]) : 0.f;
         }
         __syncthreads();
         if (warp < kSvidRows) {
             float t = 0.f;
-            for (int k = lane; k < r; k += 32) t = fmaf(sA[warp * r + k], sb[k], t);
+            for (int k = lane; k < r; k += 32) t = fmaf(sA[warp * ldf + k], sb[k], t);
             t = warp_sum(t);
             if (lane == 0) {
                 st[warp] = t;
@@ -760,10 +511,10 @@ __global__ void __launch_bounds__(256)
         for (int u = 0; u < 16; ++u) {
             const int k = threadIdx.x + 256 * u;
             if (k < r) {
-                float s = 0.f;
+                float v = 0.f;
 #pragma unroll
-                for (int w = 0; w < kSvidRows; ++w) s = fmaf(sA[w * r + k], st[w], s);
-                acc[u] += s;
+                for (int w = 0; w < kSvidRows; ++w) v = fmaf(sA[w * ldf + k], st[w], v);
+                acc[u] += v;
             }
         }
     }
@@ -775,38 +526,57 @@ __global__ void __launch_bounds__(256)
     if (lane == 0 && warp < kSvidRows) sn[warp] = nacc;
     __syncthreads();
     if (threadIdx.x == 0) {
-        double s = 0.0;
-        for (int w = 0; w < kSvidRows; ++w) s += sn[w];
-        partn[blockIdx.x] = s;
+        double v = 0.0;
+        for (int w = 0; w < kSvidRows; ++w) v += sn[w];
+        partn[blockIdx.x] = v;
     }
 }
 
+// b'_k = sum over CTAs of partb[.][k] / ||t||: CTA = 32 columns x 8 groups of partial rows;
+// each group walks every 8th partial row, then the 8 group sums are combined in a fixed
+// order (deterministic).  The last pass also writes a = t / ||t||.
 __global__ void __launch_bounds__(256)
     svid_reduce_kernel(const float *__restrict__ partb, const double *__restrict__ partn, int nblk,
                        int r, int64_t rows, int last, const float *__restrict__ tvec,
                        float *b_out, float *a_out) {
     __shared__ double s_inv;
-    if (threadIdx.x == 0) {
+    __shared__ double sg[8][33];
+    if (threadIdx.x < 32) {
         double n2 = 0.0;
-        for (int k = 0; k < nblk; ++k) n2 += partn[k];
-        const double nt = sqrt(n2);
-        s_inv = nt > 0.0 ? 1.0 / nt : 0.0;
+        for (int k = threadIdx.x; k < nblk; k += 32) n2 += partn[k];
+        n2 = warp_sum(n2);
+        if (threadIdx.x == 0) {
+            const double nt = sqrt(n2);
+            s_inv = nt > 0.0 ? 1.0 / nt : 0.0;
+        }
     }
+    const int c = threadIdx.x & 31, grp = threadIdx.x >> 5;
+    const int64_t col = (int64_t)blockIdx.x * 32 + c;
+    double v = 0.0;
+    if (col < r) {
+#pragma unroll 8
+        for (int k = grp; k < nblk; k += 8) v += partb[(int64_t)k * r + col];
+    }
+    sg[grp][c] = v;
     __syncthreads();
     const double inv = s_inv;
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx < r) {
-        double s = 0.0;
-        for (int k = 0; k < nblk; ++k) s += partb[(int64_t)k * r + idx];
-        b_out[idx] = (float)(s * inv);
+    if (grp == 0 && col < r) {
+        double t = 0.0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) t += sg[g][c];
+        b_out[col] = (float)(t * inv);
     }
-    if (last && idx < rows) a_out[idx] = (float)((double)tvec[idx] * inv);
+    if (last) {
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows;
+             i += (int64_t)gridDim.x * blockDim.x)
+            a_out[i] = (float)((double)tvec[i] * inv);
+    }
 }
 
 cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
                  float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
                  cudaStream_t s) {
-    const size_t smem = (size_t)(kSvidRows + 1) * r * sizeof(float);
+    const size_t smem = (size_t)(kSvidRows * ldf + r) * sizeof(float);
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
         cudaError_t e = cudaFuncSetAttribute(svid_pass_kernel,
@@ -815,7 +585,6 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
         if (e != cudaSuccess) return e;
         configured = smem;
     }
-    const int64_t big = rows > r ? rows : r;
     for (int pass = 1; pass <= K; ++pass) {
         const float *b_in = pass == 1 ? nullptr : bcur + (size_t)((pass - 1) & 1) * r;
         const bool last = pass == K;
@@ -823,7 +592,7 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
         svid_pass_kernel<<<nsv, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec, last ? 1 : 0, partb,
                                                 partn);
         count_launch();
-        svid_reduce_kernel<<<(unsigned)ceil_div(big, 256), 256, 0, s>>>(
+        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 256, 0, s>>>(
             partb, partn, nsv, r, rows, last ? 1 : 0, tvec, b_out, a);
         count_launch();
     }

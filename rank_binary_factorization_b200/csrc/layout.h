@@ -8,7 +8,8 @@ namespace nq {
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-constexpr int kSvidRows = 8;          // rows of S staged in shared memory per SVID tile
+constexpr int kSvidRows = 4;          // rows of S staged in shared memory per SVID tile
+constexpr int kSvidCtas = 4 * 148;     // CTAs of an SVID pass (4 per SM)
 constexpr int kRedBlocks = 592;       // CTAs of grid-stride reduction kernels (4 per SM)
 constexpr int kObjRing = 4096;        // per-iteration objective slots kept on the device
 constexpr int kMaxRank = 4096;
@@ -32,7 +33,7 @@ struct LbLayout {
     int64_t ldr = 0;   // leading dim of every [rows][r] array (FP32 and BF16)
     int64_t ldn = 0;   // leading dim of W^ rows (n padded) and of Vt
     int64_t ldm = 0;   // leading dim of W^^T rows (m padded) and of Ut
-    int64_t rp = 0;    // r padded to 32 (Cholesky tiles)
+    int64_t rp = 0;    // r padded to 64 (Cholesky tiles)
     int nsv = 0;       // CTAs of an SVID pass (rows of its partial array)
     size_t scal = 0, what = 0, whatT = 0, x[2] = {0, 0}, s[2] = {0, 0}, a[2] = {0, 0},
            b[2] = {0, 0}, xt[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
@@ -50,10 +51,10 @@ struct LbLayout {
         ldr = (r + 7) / 8 * 8;
         ldn = (n + 7) / 8 * 8;
         ldm = (m + 7) / 8 * 8;
-        rp = (r + 31) / 32 * 32;
+        rp = (r + 63) / 64 * 64;
         const int64_t maxrows = m > n ? m : n;
         int64_t tiles_rows = (maxrows + kSvidRows - 1) / kSvidRows;
-        nsv = (int)(tiles_rows < 296 ? tiles_rows : 296);
+        nsv = (int)(tiles_rows < kSvidCtas ? tiles_rows : kSvidCtas);
         size_t off = 0;
         auto take = [&](size_t bytes) {
             size_t o = off;

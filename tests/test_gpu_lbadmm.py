@@ -141,9 +141,11 @@ def test_planted_factors_recovered_on_gpu(nq):
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_planted_with_noise_end_to_end(nq, seed):
+    # 60 iterations: both the oracle and the BF16-operand arithmetic have converged to the
+    # planted factors on every seed (at 30 the slowest seed is still on its way there).
     p = planted_problem(seed, noise=0.1)
-    res = nq.nq_lbadmm(p["W"].cuda(), 16, iters=30)
-    ref = O.lbadmm(p["W"].double().numpy(), r=16, iters=30)
+    res = nq.nq_lbadmm(p["W"].cuda(), 16, iters=60)
+    ref = O.lbadmm(p["W"].double().numpy(), r=16, iters=60)
     assert abs(res["rel_err"] - ref.rel_err) <= TOL_E2E * ref.rel_err
     # first objective value: identical start, differs only by arithmetic
     assert abs(res["objective"][0] - ref.objective[0]) <= 1e-3 * ref.objective[0]
