@@ -197,10 +197,35 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
     nq_status st = lb_gram(lb, other, lambda + rho, s);
     if (st) return st;
     {
-    ProfScope ps(NQ_K_CHOL, s);
-    NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
-                       lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.gih),
-                       lb.p<__nv_bfloat16>(L.gil), L.ldr, &lb.sc->err, lb.sc->bar, s));
+        ProfScope ps(NQ_K_CHOL, s);
+        NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
+                           lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
+                           lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
+                           &lb.sc->err, lb.sc->bar, s));
+        // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        const void *th = lb.p<void>(L.lth), *tl = lb.p<void>(L.ltl);
+        const int BNg = L.r > 1024 ? 128 : BN;
+        if (!tc::make_map_bf16(&maps.a[0], th, L.r, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[1], th, L.r, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[2], tl, L.r, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[0], th, L.r, L.r, L.ldr, BNg) ||
+            !tc::make_map_bf16(&maps.b[1], tl, L.r, L.r, L.ldr, BNg) ||
+            !tc::make_map_bf16(&maps.b[2], th, L.r, L.r, L.ldr, BNg))
+            return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = L.r;
+        ep.N = L.r;
+        ep.nseg = 3;
+        ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
+        ep.tri_k = 1;
+        ep.err = &lb.sc->err;
+        ep.Rhi = lb.p<__nv_bfloat16>(L.gih);
+        ep.Rlo = lb.p<__nv_bfloat16>(L.gil);
+        ep.ldr = L.ldr;
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, s));
     }
 
     // R = W^ X_other + rho (Z - L), split into hi + lo bf16

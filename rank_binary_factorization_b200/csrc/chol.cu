@@ -1,6 +1,6 @@
-// G^-1 for the r x r SPD system matrix of the U (V) step: Cholesky G = L L^T, L^-1 by
-// recursive doubling, G^-1 = L^-T L^-1, written as BF16 hi + lo for the split-BF16
-// tensor-core solve.  NanoQuant summary page, "Core method" (核心方法), step (a): the
+// Cholesky G = L L^T of the r x r SPD system matrix of the U (V) step and L^-1 by
+// recursive doubling; (L^-1)^T is emitted as BF16 hi + lo for the tensor-core product
+// G^-1 = L^-T L^-1.  NanoQuant summary page, "Core method" (核心方法), step (a): the
 // regularised linear system is solved through a Cholesky factorisation.
 //
 // One cooperative launch of FP32 SIMT work on 64 x 64 tiles (4 x 4 register blocks per
@@ -8,10 +8,15 @@
 //   * right-looking blocked Cholesky with look-ahead: while CTAs 1.. apply the trailing
 //     update of step j, CTA 0 updates the next diagonal tile and factors it, so a step
 //     costs two barriers and the diagonal factorisation overlaps the update;
-//   * the diagonal 64 x 64 factorisation and its inverse keep each thread's 16 entries
-//     in registers and broadcast the current column / row with one barrier per step;
+//   * panel tiles are solved by forward substitution (all in parallel), so the inverse
+//     of a diagonal tile is not on the chain of block steps; the diagonal inverses are
+//     formed afterwards, one CTA per tile, all at once;
+//   * the 64 x 64 tile Cholesky works in 16-column blocks factored by one warp with
+//     shuffles (no CTA barrier per column); panel rows are independent substitutions,
+//     one thread per row with no barrier at all;
 //   * (L^-1)_21 = -L22^-1 L21 L11^-1 level by level (log2(r/64) levels, two barriers each);
-//   * G^-1 tiles (a >= b) = sum_{c >= a} Li(c,a)^T Li(c,b), mirrored.
+//   * (L^-1)^T is written as bf16 hi + lo; G^-1 = L^-T L^-1 is then one split-BF16
+//     tensor-core GEMM (see gemm_tc.cu, EPI_SPLIT).
 #include "kernels.cuh"
 
 namespace nq {
@@ -31,6 +36,7 @@ struct Chol2Args {
     float *Li;    // rp x rp: L^-1 (lower tiles), scratch T in upper tiles
     __nv_bfloat16 *hi, *lo;
     int64_t ldr;
+    unsigned int *cnt;  // nb x nb: operations completed on tile (i, k)
     int *err;
     unsigned int *bar;
 };
@@ -65,6 +71,23 @@ __device__ __forceinline__ void store_n(float *M, int64_t ld, int ti, int tj, co
     }
 }
 
+// Asynchronous plain tile load (cp.async, L2 only): completes at cp_async_wait.
+__device__ __forceinline__ void load_n_async(Tile &d, const float *M, int64_t ld, int ti, int tj) {
+    const float *base = M + (int64_t)ti * TB * ld + (int64_t)tj * TB;
+    for (int f = threadIdx.x; f < TB * TB / 4; f += blockDim.x) {
+        const int row = f >> 4, c4 = (f & 15) * 4;
+        const uint32_t sa = (uint32_t)__cvta_generic_to_shared(&d[row][c4]);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
+                     "l"(base + (int64_t)row * ld + c4)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Thread's 4 x 4 block of a 64 x 64 tile: rows a0..a0+3, columns b0..b0+3.
 __device__ __forceinline__ int blk_a0() { return (threadIdx.x >> 4) * 4; }
 __device__ __forceinline__ int blk_b0() { return (threadIdx.x & 15) * 4; }
@@ -86,6 +109,34 @@ __device__ __forceinline__ void mac(float (&acc)[4][4], const Tile &XT, const Ti
     }
 }
 
+// acc[i][j] += sum_c X[a0+i][c] * Y[c][b0+j]  (both tiles in plain layout)
+__device__ __forceinline__ void mac_n(float (&acc)[4][4], const Tile &X, const Tile &Y) {
+    const int a0 = blk_a0(), b0 = blk_b0();
+#pragma unroll 2
+    for (int c = 0; c < TB; c += 4) {
+        float x[4][4], y[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = *reinterpret_cast<const float4 *>(&X[a0 + i][c]);
+            x[i][0] = v.x;
+            x[i][1] = v.y;
+            x[i][2] = v.z;
+            x[i][3] = v.w;
+            const float4 w = *reinterpret_cast<const float4 *>(&Y[c + i][b0]);
+            y[i][0] = w.x;
+            y[i][1] = w.y;
+            y[i][2] = w.z;
+            y[i][3] = w.w;
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(x[i][cc], y[cc][j], acc[i][j]);
+    }
+}
+
 __device__ __forceinline__ void zero(float (&acc)[4][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -104,88 +155,197 @@ __device__ __forceinline__ void put(float *M, int64_t ld, int ti, int tj, const 
                make_float4(sgn * acc[i][0], sgn * acc[i][1], sgn * acc[i][2], sgn * acc[i][3]));
 }
 
-// ---- 64 x 64 diagonal tile: Cholesky and triangular inverse -------------------------
-// Thread t owns row i = t / 4 and the columns 4p + g (g = t % 4, p = 0..15) in
-// registers.  Column k (Cholesky) and row k of L^-1 (inverse) are broadcast through a
-// double-buffered shared array; the owners of the next column / row publish it in the
-// same step, so each of the 2 x 64 steps costs a single CTA barrier.  The loops are
-// compact: this code runs once per block step.  The register window is shifted by one
-// column quad per four steps so that the current column always sits in a[0].
-// On entry s holds A_jj; on exit s holds L_jj (zero above the diagonal), inv holds L_jj^-1.
-// cb: 2 x 64 floats of shared scratch.
-__device__ void factor_diag(Tile &s, Tile &inv, float *cb, int *err) {
-    const int t = threadIdx.x, i = t >> 2, g = t & 3;
-    float a[16];
-#pragma unroll
-    for (int p = 0; p < 16; ++p) a[p] = s[i][4 * p + g];
+// ---- 64 x 64 tile Cholesky: four 16-column blocks -----------------------------------
+// Block b: all threads subtract the finished columns from block column b (rows 16b ..
+// 63), then warp 0 factors it column by column with shuffles (lane l holds rows
+// 16b + l and 16b + l + 32), so the 64 sequential column steps need no CTA barrier.
+__device__ void chol_tile(Tile &s, int *err) {
+    const int t = threadIdx.x, lane = t & 31;
     bool bad = false;
-    if (g == 0) cb[i] = a[0];  // column 0 (its owners have g == 0)
-    __syncthreads();
 #pragma unroll 1
-    for (int q = 0; q < 16; ++q) {
-#pragma unroll
-        for (int g2 = 0; g2 < 4; ++g2) {
-            const int k = 4 * q + g2;
-            const float *col = cb + 64 * (k & 1);
-            float *nxt = cb + 64 * ((k + 1) & 1);
-            float piv = col[k];
-            if (!(piv > 0.f)) {
-                bad = true;
-                piv = 1e-30f;
+    for (int b = 0; b < 4; ++b) {
+        const int c0 = 16 * b;
+        if (b > 0) {
+            const int c = c0 + (t & 15);
+            for (int i = c0 + (t >> 4); i < TB; i += 16) {
+                float acc = 0.f;
+                for (int m = 0; m < c0; m += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(&s[i][m]);
+                    const float4 y = *reinterpret_cast<const float4 *>(&s[c][m]);
+                    acc = fmaf(x.x, y.x, acc);
+                    acc = fmaf(x.y, y.y, acc);
+                    acc = fmaf(x.z, y.z, acc);
+                    acc = fmaf(x.w, y.w, acc);
+                }
+                s[i][c] -= acc;
             }
-            const float l = sqrtf(piv);
-            const float il = 1.f / l;
-            const float lik = (i == k) ? l : col[i] * il;
-#pragma unroll
-            for (int p = 0; p < 16; ++p) {
-                const int j = 4 * (q + p) + g;
-                if (j > k && j <= i && j < 64) a[p] = fmaf(-lik, col[j] * il, a[p]);
-            }
-            if (g == g2) s[i][k] = (i >= k) ? lik : 0.f;
-            // publish column k + 1: its owners hold it in a[0] (g2 < 3) or a[1] (g2 == 3)
-            if (k + 1 < 64 && g == ((g2 + 1) & 3) && i >= k + 1) nxt[i] = (g2 == 3) ? a[1] : a[0];
             __syncthreads();
         }
+        if (t < 32) {
+            const int r0 = c0 + lane, r1 = r0 + 32;
+            float a0[16], a1[16];
 #pragma unroll
-        for (int p = 0; p < 15; ++p) a[p] = a[p + 1];
-    }
-    if (bad && t == 0) raise_error(err, NQ_ERR_NOT_SPD);
-    // X = L^-1, thread owns x[p] = X[i][4p + g]; row k final = (row k after updates) / L_kk
-    float x[16];
+            for (int c = 0; c < 16; ++c) {
+                a0[c] = (r0 < TB) ? s[r0][c0 + c] : 0.f;
+                a1[c] = (r1 < TB) ? s[r1][c0 + c] : 0.f;
+            }
 #pragma unroll
-    for (int p = 0; p < 16; ++p) x[p] = (4 * p + g == i) ? 1.f : 0.f;
-    if (i == 0) {
-        const float il0 = 1.f / s[0][0];
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-            x[p] *= il0;
-            cb[4 * p + g] = x[p];
-        }
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int k = 0; k < 64; ++k) {
-        const float *rowk = cb + 64 * (k & 1);
-        float *nxt = cb + 64 * ((k + 1) & 1);
-        if (i > k) {
-            const float lik = s[i][k];
-#pragma unroll
-            for (int p = 0; p < 16; ++p)
-                if (4 * p + g <= k) x[p] = fmaf(-lik, rowk[4 * p + g], x[p]);
-            if (i == k + 1) {  // row k + 1 is now final: scale and publish
-                const float il = 1.f / s[i][i];
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    x[p] *= il;
-                    nxt[4 * p + g] = x[p];
+            for (int k = 0; k < 16; ++k) {
+                float piv = __shfl_sync(0xffffffffu, a0[k], k);
+                if (!(piv > 0.f)) {
+                    bad = true;
+                    piv = 1e-30f;
                 }
+                const float il = rsqrtf(piv);
+                const float l0 = a0[k] * il, l1 = a1[k] * il;
+                a0[k] = l0;
+                a1[k] = l1;
+#pragma unroll
+                for (int c = k + 1; c < 16; ++c) {
+                    const float lc = __shfl_sync(0xffffffffu, l0, c);
+                    a0[c] = fmaf(-l0, lc, a0[c]);
+                    a1[c] = fmaf(-l1, lc, a1[c]);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                if (r0 < TB) s[r0][c0 + c] = (lane >= c) ? a0[c] : 0.f;
+                if (r1 < TB) s[r1][c0 + c] = a1[c];
             }
         }
         __syncthreads();
     }
-#pragma unroll
-    for (int p = 0; p < 16; ++p) inv[i][4 * p + g] = x[p];
+    for (int e = t; e < TB * TB; e += blockDim.x) {
+        const int i = e >> 6, c = e & 63;
+        if (i < (c & ~15)) s[i][c] = 0.f;
+    }
+    if (bad) raise_error(err, NQ_ERR_NOT_SPD);
     __syncthreads();
+}
+
+// ---- panel: X L_jj^T = A for a 64 x 64 tile, one thread per row ----------------------
+// Rows are independent forward substitutions, so they need no synchronisation.  The
+// thread keeps its row in registers as a window x[0..W) over columns c0 .. c0 + W - 1;
+// after each quad of 4 columns the finished values are stored and the window shifts by
+// 4.  W is the remaining width rounded up to 16 (64, 48, 32, 16): lt rows are padded with
+// zeros to LTW columns so the last window reads zeros past column 63.
+constexpr int LTW = 80;  // >= 60 + 16, multiple of 4
+using LtTile = float[TB][LTW];
+
+template <int W, bool COL>
+__device__ __forceinline__ void subst_quad(float (&x)[64], const LtTile &lt, const float *dinv,
+                                           int c0, float *dst, int64_t ld) {
+#pragma unroll
+    for (int g2 = 0; g2 < 4; ++g2) {
+        const int c = c0 + g2;
+        const float xc = x[g2] * dinv[c];
+        x[g2] = xc;
+#pragma unroll
+        for (int m = 0; m < W / 4; ++m) {
+            const float4 l = *reinterpret_cast<const float4 *>(&lt[c][c0 + 4 * m]);
+            const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * m + e > g2) x[4 * m + e] = fmaf(-xc, lv[e], x[4 * m + e]);
+        }
+    }
+    if (COL) {  // entries c0 .. c0 + 3 of a column: rows of the output
+#pragma unroll
+        for (int e = 0; e < 4; ++e) __stcg(dst + (int64_t)(c0 + e) * ld, x[e]);
+    } else {
+        __stcg(reinterpret_cast<float4 *>(dst + c0), make_float4(x[0], x[1], x[2], x[3]));
+    }
+#pragma unroll
+    for (int p = 0; p < W - 4; ++p) x[p] = x[p + 4];
+}
+
+template <bool COL>
+__device__ __forceinline__ void subst_run(float (&x)[64], const LtTile &lt, const float *dinv,
+                                          float *dst, int64_t ld) {
+#pragma unroll 1
+    for (int qb = 0; qb < 16; ++qb) {
+        const int c0 = 4 * qb;
+        if (qb < 4)
+            subst_quad<64, COL>(x, lt, dinv, c0, dst, ld);
+        else if (qb < 8)
+            subst_quad<48, COL>(x, lt, dinv, c0, dst, ld);
+        else if (qb < 12)
+            subst_quad<32, COL>(x, lt, dinv, c0, dst, ld);
+        else
+            subst_quad<16, COL>(x, lt, dinv, c0, dst, ld);
+    }
+}
+
+// Row `row` of the tile at Ag (row stride ld) is replaced by its solution x, x L^T = a.
+// lt[c][k] = L_kc (zero for k >= 64), dinv[c] = 1 / L_cc.
+__device__ void panel_row(float *Ag, int64_t ld, int row, const LtTile &lt, const float *dinv) {
+    float *rp = Ag + (int64_t)row * ld;
+    float x[64];
+#pragma unroll
+    for (int p = 0; p < 64; p += 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(rp + p));
+        x[p] = v.x;
+        x[p + 1] = v.y;
+        x[p + 2] = v.z;
+        x[p + 3] = v.w;
+    }
+    subst_run<false>(x, lt, dinv, rp, ld);
+}
+
+// Column `col` of L^-1 (L x = e_col) into the tile at Og (row stride ld).
+__device__ void inverse_col(float *Og, int64_t ld, int col, const LtTile &lt, const float *dinv) {
+    float x[64];
+#pragma unroll
+    for (int p = 0; p < 64; ++p) x[p] = (p == col) ? 1.f : 0.f;
+    subst_run<true>(x, lt, dinv, Og + col, ld);
+}
+
+// lt[c][k] = L_kc for the lower tile (ti, ti) of A (zero-padded to LTW), dinv[c] = 1/L_cc.
+__device__ void load_lt(LtTile &lt, float *dinv, const float *A, int64_t ld, int ti) {
+    const float *L = A + (int64_t)ti * TB * ld + (int64_t)ti * TB;
+    __syncthreads();
+    for (int e = threadIdx.x; e < TB * TB; e += blockDim.x) {
+        const int k = e >> 6, c = e & 63;  // coalesced read of row k
+        lt[c][k] = __ldcg(L + (int64_t)k * ld + c);
+    }
+    for (int e = threadIdx.x; e < TB * (LTW - TB); e += blockDim.x)
+        lt[e / (LTW - TB)][TB + e % (LTW - TB)] = 0.f;
+    __syncthreads();
+    if (threadIdx.x < TB) dinv[threadIdx.x] = 1.f / lt[threadIdx.x][threadIdx.x];
+    __syncthreads();
+}
+
+// Job order for a CTA: rounds of gridDim.x jobs dealt in alternating direction, so
+// that with jobs sorted by decreasing cost the per-CTA totals stay balanced.
+__device__ __forceinline__ int64_t dealt_job(int64_t k) {
+    const int64_t G = gridDim.x;
+    return k * G + ((k & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
+}
+
+// ---- tile counters of the factorisation ------------------------------------------
+// cnt(i, k) counts the operations finished on tile (i, k): the k updates of steps
+// 0 .. k-1, then its Cholesky (i == k) or panel solve (i > k).  A task waits until the
+// counters of its operands reach the required values; waits are bounded and, once one
+// has timed out, skipped.
+__device__ __forceinline__ void wait_count(const unsigned int *c, unsigned int target, int *err) {
+    if (threadIdx.x == 0 && !(*(volatile int *)err == NQ_ERR_TIMEOUT)) {
+        uint32_t spins = 0;
+        while (ld_acquire_gpu(c) < target) {
+            if (++spins > kGridSpinLimit) {
+                raise_error(err, NQ_ERR_TIMEOUT);
+                break;
+            }
+            if (spins > 64) __nanosleep(32);
+        }
+    }
+    __syncthreads();
+}
+__device__ __forceinline__ void signal_count(unsigned int *c, unsigned int inc) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(c, inc);
+    }
 }
 
 // lower-triangular enumeration idx -> (ii >= kk)
@@ -206,45 +366,51 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
     const int64_t rp = p.rp;
 
     // phase 0: A = G padded with the identity
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rp * rp;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t i = e / rp, j = e % rp;
-        p.A[e] = (i < p.r && j < p.r) ? p.G[i * p.r + j] : (i == j ? 1.f : 0.f);
+    for (int i = blockIdx.x; i < rp; i += gridDim.x) {
+        float *dst = p.A + (int64_t)i * rp;
+        const float *src = p.G + (int64_t)i * p.r;
+#pragma unroll 4
+        for (int j = threadIdx.x; j < rp; j += blockDim.x)
+            dst[j] = (i < p.r && j < p.r) ? __ldg(src + j) : (i == j ? 1.f : 0.f);
     }
     grid_barrier(p.bar, p.err);
+    Tile &cb = *reinterpret_cast<Tile *>(smem_f + 3 * TB * LDS);  // published columns
+    float *rpv = smem_f + 4 * TB * LDS;     // 64 reciprocal pivots
+    float *dinv = rpv + 64;                 // 64 reciprocals of the current L_jj diagonal
+    LtTile &lt = *reinterpret_cast<LtTile *>(smem_f + 4 * TB * LDS + 128);  // L_jj^T, padded
+    // Dataflow factorisation.  CTA 0 runs the critical chain: Cholesky of (j, j), panel
+    // tile (j+1, j) from the L_jj it holds in shared memory, update of (j+1, j+1) and its
+    // Cholesky.  CTAs 1.. take the other panel tiles and trailing updates round-robin in
+    // a topological order (step by step), so every wait ends.
+    auto CNT = [&](int i, int k) { return p.cnt + (int64_t)i * nb + k; };
     if (blockIdx.x == 0) {
-        load_n(t0, p.A, rp, 0, 0);
+        load_n(t2, p.A, rp, 0, 0);
         __syncthreads();
-        factor_diag(t0, t1, &t2[0][0], p.err);
-        store_n(p.A, rp, 0, 0, t0);
-        store_n(p.Li, rp, 0, 0, t1);
-    }
-    grid_barrier(p.bar, p.err);
-
-    for (int j = 0; j < nb; ++j) {
-        // panel: L_ij = A_ij L_jj^-T
-        for (int i = j + 1 + blockIdx.x; i < nb; i += gridDim.x) {
+        chol_tile(t2, p.err);
+        store_n(p.A, rp, 0, 0, t2);
+        signal_count(CNT(0, 0), 1);
+        for (int j = 0; j + 1 < nb; ++j) {
+            // t2 holds L_jj: build lt, dinv from it
             __syncthreads();
-            load_t(t0, p.A, rp, i, j);
-            load_t(t1, p.Li, rp, j, j);
+            for (int e = threadIdx.x; e < TB * LTW; e += blockDim.x) {
+                const int c = e / LTW, k = e % LTW;
+                lt[c][k] = (k < TB) ? t2[k][c] : 0.f;
+            }
             __syncthreads();
-            float acc[4][4];
-            zero(acc);
-            mac(acc, t0, t1);
-            put(p.A, rp, i, j, acc, 1.f);
-        }
-        grid_barrier(p.bar, p.err);
-        if (j == nb - 1) break;
-        const int T = nb - 1 - j;
-        if (blockIdx.x == 0) {
-            // look-ahead: next diagonal tile, updated then factored
-            __syncthreads();
+            if (threadIdx.x < TB) dinv[threadIdx.x] = 1.f / t2[threadIdx.x][threadIdx.x];
+            wait_count(CNT(j + 1, j), j, p.err);  // its j updates
+            if (threadIdx.x < TB)
+                panel_row(p.A + (int64_t)(j + 1) * TB * rp + (int64_t)j * TB, rp, threadIdx.x, lt,
+                          dinv);
+            signal_count(CNT(j + 1, j), 1);
+            // look-ahead: (j+1, j+1) -= L_{j+1,j} L_{j+1,j}^T, then its Cholesky
+            wait_count(CNT(j + 1, j + 1), j, p.err);
             load_t(t0, p.A, rp, j + 1, j);
             load_n(t2, p.A, rp, j + 1, j + 1);
             __syncthreads();
             float acc[4][4];
             zero(acc);
-            mac(acc, t0, t0);  // L_{j+1,j} L_{j+1,j}^T with t0 holding L^T: XT = Y = t0
+            mac(acc, t0, t0);
             __syncthreads();
             {
                 const int a0 = blk_a0(), b0 = blk_b0();
@@ -254,111 +420,172 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     for (int q = 0; q < 4; ++q) t2[a0 + i][b0 + q] -= acc[i][q];
             }
             __syncthreads();
-            factor_diag(t2, t1, &t0[0][0], p.err);
+            chol_tile(t2, p.err);
             store_n(p.A, rp, j + 1, j + 1, t2);
-            store_n(p.Li, rp, j + 1, j + 1, t1);
-        } else {
-            const int64_t ntl = (int64_t)T * (T + 1) / 2;
-            for (int64_t idx = 1 + (blockIdx.x - 1); idx < ntl; idx += gridDim.x - 1) {
-                int ii, kk;
-                tri_index(idx, ii, kk);
-                const int i = j + 1 + ii, k = j + 1 + kk;
-                __syncthreads();
-                load_t(t0, p.A, rp, i, j);
-                load_t(t1, p.A, rp, k, j);
-                __syncthreads();
-                float acc[4][4];
-                zero(acc);
-                mac(acc, t0, t1);
-                // A_ik -= acc (read-modify-write of the thread's own block)
-                const int a0 = blk_a0(), b0 = blk_b0();
-                float *base = p.A + ((int64_t)i * TB + a0) * rp + (int64_t)k * TB + b0;
+            signal_count(CNT(j + 1, j + 1), 2);
+        }
+    } else {
+        const int64_t W = gridDim.x - 1, w = blockIdx.x - 1;
+        int64_t base = 0;
+        for (int j = 0; j + 1 < nb; ++j) {
+            const int T = nb - 1 - j;               // tiles below (j, j)
+            const int P = T - 1;                    // panels (i, j), i >= j + 2
+            const int64_t U = (int64_t)T * (T + 1) / 2 - 1;  // updates except (j+1, j+1)
+            const int64_t n = P + U;
+            for (int64_t idx = base + ((w - base % W) % W + W) % W; idx < base + n; idx += W) {
+                const int64_t loc = idx - base;
+                if (loc < P) {  // panel tile (i, j)
+                    const int i = j + 2 + (int)loc;
+                    wait_count(CNT(j, j), j + 1, p.err);
+                    load_lt(lt, dinv, p.A, rp, j);
+                    wait_count(CNT(i, j), j, p.err);
+                    if (threadIdx.x < TB)
+                        panel_row(p.A + (int64_t)i * TB * rp + (int64_t)j * TB, rp, threadIdx.x,
+                                  lt, dinv);
+                    signal_count(CNT(i, j), 1);
+                } else {  // update of tile (i, k) with step j: A_ik -= L_ij L_kj^T
+                    int ii, kk;
+                    tri_index(loc - P + 1, ii, kk);
+                    const int i = j + 1 + ii, k = j + 1 + kk;
+                    wait_count(CNT(i, j), j + 1, p.err);
+                    wait_count(CNT(k, j), j + 1, p.err);
+                    wait_count(CNT(i, k), j, p.err);
+                    load_t(t0, p.A, rp, i, j);
+                    load_t(t1, p.A, rp, k, j);
+                    __syncthreads();
+                    float acc[4][4];
+                    zero(acc);
+                    mac(acc, t0, t1);
+                    const int a0 = blk_a0(), b0 = blk_b0();
+                    float *bp = p.A + ((int64_t)i * TB + a0) * rp + (int64_t)k * TB + b0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float4 v = __ldcg(reinterpret_cast<const float4 *>(base + (int64_t)q * rp));
-                    v.x -= acc[q][0];
-                    v.y -= acc[q][1];
-                    v.z -= acc[q][2];
-                    v.w -= acc[q][3];
-                    __stcg(reinterpret_cast<float4 *>(base + (int64_t)q * rp), v);
+                    for (int q = 0; q < 4; ++q) {
+                        float4 v = __ldcg(reinterpret_cast<const float4 *>(bp + (int64_t)q * rp));
+                        v.x -= acc[q][0];
+                        v.y -= acc[q][1];
+                        v.z -= acc[q][2];
+                        v.w -= acc[q][3];
+                        __stcg(reinterpret_cast<float4 *>(bp + (int64_t)q * rp), v);
+                    }
+                    signal_count(CNT(i, k), 1);
                 }
             }
+            base += n;
         }
-        grid_barrier(p.bar, p.err);
     }
+    grid_barrier(p.bar, p.err);
 
-    // L^-1 by recursive doubling; T(a, b) = L21 Li11 kept in the unused upper tile (b, a)
+    // inverses of all diagonal tiles in parallel: column substitutions L x = e_c
+    for (int d = blockIdx.x; d < nb; d += gridDim.x) {
+        load_lt(lt, dinv, p.A, rp, d);
+        if (threadIdx.x < TB)
+            inverse_col(p.Li + (int64_t)d * TB * rp + (int64_t)d * TB, rp, threadIdx.x, lt, dinv);
+    }
+    grid_barrier(p.bar, p.err);
+
+    // L^-1 by recursive doubling over pairs of s x s tile blocks [L11 0; L21 L22]:
+    // T = L21 Li11 (kept in the unused upper tile (b, a)), then Li21 = -Li22 T.
+    // Jobs are ordered by decreasing number of tile products and dealt alternately;
+    // each job streams its operand tiles through two cp.async stages.
     for (int s = 1; s < nb; s *= 2) {
         const int npairs = (int)ceil_div(nb, 2 * s);
-        const int64_t jobs = (int64_t)npairs * s * s;
-        for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
-            const int pr = (int)(q / ((int64_t)s * s));
-            const int a = 2 * pr * s + s + (int)((q % ((int64_t)s * s)) / s);
-            const int b = 2 * pr * s + (int)(q % s);
-            if (a >= nb) continue;
-            const int top_end = 2 * pr * s + s;
-            float acc[4][4];
-            zero(acc);
-            for (int c = b; c < top_end; ++c) {
+        const int64_t per = (int64_t)npairs * s;  // jobs of equal cost
+        const int64_t jobs = per * s;
+        for (int half = 0; half < 2; ++half) {
+            for (int64_t k = 0;; ++k) {
+                const int64_t q = dealt_job(k);
+                if (q >= jobs) break;
+                const int cls = (int)(q / per);
+                const int64_t rem = q % per;
+                const int pr = (int)(rem / s), o = (int)(rem % s);
+                const int top0 = 2 * pr * s, bot0 = top0 + s;
+                int a, b, c0, c1;
+                if (half == 0) {  // T(a, b) = sum_{c=b}^{bot0-1} L(a, c) Li(c, b): s - b products
+                    a = bot0 + o;
+                    b = top0 + cls;
+                    c0 = b;
+                    c1 = bot0;
+                } else {  // Li(a, b) = -sum_{c=bot0}^{a} Li(a, c) T(c, b): a - bot0 + 1 products
+                    a = bot0 + (s - 1 - cls);
+                    b = top0 + o;
+                    c0 = bot0;
+                    c1 = a + 1;
+                }
+                if (a >= nb) continue;
+                float acc[4][4];
+                zero(acc);
                 __syncthreads();
-                load_t(t0, p.A, rp, a, c);   // L21(a, c)
-                load_n(t1, p.Li, rp, c, b);  // Li11(c, b)
-                __syncthreads();
-                mac(acc, t0, t1);
+                // stage 0: X in t0, Y in t1; stage 1: X in t2, Y in cb
+                auto issue = [&](int c, int st) {
+                    Tile &X = st ? t2 : t0;
+                    Tile &Y = st ? cb : t1;
+                    if (half == 0) {
+                        load_n_async(X, p.A, rp, a, c);   // L(a, c)
+                        load_n_async(Y, p.Li, rp, c, b);  // Li(c, b)
+                    } else {
+                        load_n_async(X, p.Li, rp, a, c);  // Li(a, c)
+                        load_n_async(Y, p.Li, rp, b, c);  // T(c, b) at tile (b, c)
+                    }
+                };
+                issue(c0, 0);
+                for (int c = c0; c < c1; ++c) {
+                    const int st = (c - c0) & 1;
+                    if (c + 1 < c1) {
+                        issue(c + 1, st ^ 1);
+                        cp_async_wait<2>();
+                    } else {
+                        cp_async_wait<0>();
+                    }
+                    __syncthreads();
+                    mac_n(acc, st ? t2 : t0, st ? cb : t1);
+                    __syncthreads();
+                }
+                if (half == 0)
+                    put(p.Li, rp, b, a, acc, 1.f);
+                else
+                    put(p.Li, rp, a, b, acc, -1.f);
             }
-            put(p.Li, rp, b, a, acc, 1.f);
+            grid_barrier(p.bar, p.err);
         }
-        grid_barrier(p.bar, p.err);
-        for (int64_t q = blockIdx.x; q < jobs; q += gridDim.x) {
-            const int pr = (int)(q / ((int64_t)s * s));
-            const int bot0 = 2 * pr * s + s;
-            const int a = bot0 + (int)((q % ((int64_t)s * s)) / s);
-            const int b = 2 * pr * s + (int)(q % s);
-            if (a >= nb) continue;
-            float acc[4][4];
-            zero(acc);
-            for (int c = bot0; c <= a; ++c) {
-                __syncthreads();
-                load_t(t0, p.Li, rp, a, c);  // Li22(a, c)
-                load_n(t1, p.Li, rp, b, c);  // T(c, b) lives at tile (b, c)
-                __syncthreads();
-                mac(acc, t0, t1);
-            }
-            put(p.Li, rp, a, b, acc, -1.f);
-        }
-        grid_barrier(p.bar, p.err);
     }
 
-    // G^-1 = Li^T Li, tiles a >= b, largest sums first; split into bf16 hi + lo
-    const int64_t ngi = (int64_t)nb * (nb + 1) / 2;
-    for (int64_t idx = blockIdx.x; idx < ngi; idx += gridDim.x) {
-        int a, b;
-        tri_index(idx, a, b);
-        // idx enumerates a ascending: small a = long sums come first
-        float acc[4][4];
-        zero(acc);
-        for (int c = a; c < nb; ++c) {
-            __syncthreads();
-            load_n(t0, p.Li, rp, c, a);
-            load_n(t1, p.Li, rp, c, b);
-            __syncthreads();
-            mac(acc, t0, t1);
-        }
-        const int a0 = blk_a0(), b0 = blk_b0();
+    // (L^-1)^T as bf16 hi + lo: LiT[x][y] = Li[y][x] (zero for y < x), all r x r entries,
+    // the operand of the tensor-core product G^-1 = Li^T Li.  Thread: 8 consecutive y.
+    const int64_t nt2 = (int64_t)nb * nb;
+    const bool vec_ok = (p.ldr % 8) == 0;
+    for (int64_t idx = blockIdx.x; idx < nt2; idx += gridDim.x) {
+        const int ta = (int)(idx / nb), tc = (int)(idx % nb);  // LiT tile (ta, tc)
+        __syncthreads();
+        if (tc >= ta) load_n(t0, p.Li, rp, tc, ta);              // t0[y][x] = Li_tile(tc,ta)
+        __syncthreads();
+        for (int e = threadIdx.x; e < TB * TB / 8; e += blockDim.x) {
+            const int x = e & 63, y8 = (e >> 6) * 8;
+            const int64_t gi = (int64_t)ta * TB + x, gj = (int64_t)tc * TB + y8;
+            if (gi >= p.r || gj >= p.r) continue;
+            uint32_t h[4], l[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t gi = (int64_t)a * TB + a0 + i;
+            for (int k = 0; k < 4; ++k) {
+                const float v0 = (tc >= ta) ? t0[y8 + 2 * k][x] : 0.f;
+                const float v1 = (tc >= ta) ? t0[y8 + 2 * k + 1][x] : 0.f;
+                const __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
+                const __nv_bfloat162 ll = __floats2bfloat162_rn(v0 - __low2float(hh),
+                                                                v1 - __high2float(hh));
+                h[k] = *reinterpret_cast<const uint32_t *>(&hh);
+                l[k] = *reinterpret_cast<const uint32_t *>(&ll);
+            }
+            __nv_bfloat16 *ph = p.hi + gi * p.ldr + gj, *pl = p.lo + gi * p.ldr + gj;
+            if (vec_ok && gj + 8 <= p.r) {
+                *reinterpret_cast<uint4 *>(ph) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(pl) = make_uint4(l[0], l[1], l[2], l[3]);
+            } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int64_t gj = (int64_t)b * TB + b0 + q;
-                if (gi < p.r && gj < p.r) {
-                    const float v = acc[i][q];
-                    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                    const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-                    p.hi[gi * p.ldr + gj] = h;
-                    p.lo[gi * p.ldr + gj] = l;
-                    p.hi[gj * p.ldr + gi] = h;
-                    p.lo[gj * p.ldr + gi] = l;
+                for (int k = 0; k < 8; ++k) {
+                    if (gj + k >= p.r) break;
+                    const uint32_t hw = h[k >> 1], lw = l[k >> 1];
+                    const unsigned short hs = (k & 1) ? (unsigned short)(hw >> 16) : (unsigned short)hw;
+                    const unsigned short ls = (k & 1) ? (unsigned short)(lw >> 16) : (unsigned short)lw;
+                    ph[k] = __ushort_as_bfloat16(hs);
+                    pl[k] = __ushort_as_bfloat16(ls);
                 }
             }
         }
@@ -370,10 +597,10 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
 int64_t chol_padded(int32_t r) { return (int64_t)(r + TB - 1) / TB * TB; }
 
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
-                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr, int *err,
-                         unsigned int *bar, cudaStream_t s) {
+                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
+                         unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
-    constexpr int smem = 3 * TB * LDS * sizeof(float);
+    constexpr int smem = (4 * TB * LDS + 128 + TB * LTW) * sizeof(float);
     static int grid = 0;
     if (!grid) {
         cudaError_t e = cudaFuncSetAttribute(chol2_kernel,
@@ -390,7 +617,10 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
     }
     cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    Chol2Args args{G, r, (int)(rp / TB), rp, A, Li, Gi_hi, Gi_lo, ldr, err, bar};
+    const int nb = (int)(rp / TB);
+    e = cudaMemsetAsync(flags, 0, (size_t)nb * nb * sizeof(unsigned int), s);
+    if (e != cudaSuccess) return e;
+    Chol2Args args{G, r, nb, rp, A, Li, Gi_hi, Gi_lo, ldr, flags, err, bar};
     void *params[] = {&args};
     count_launch();
     return cudaLaunchCooperativeKernel((const void *)chol2_kernel, dim3(grid), dim3(256), params,

@@ -161,6 +161,27 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
             for (int j = 0; j < 16; ++j)
                 if (full || col0 + j < p.N) o[j] = w[j];
         }
+    } else if constexpr (EPI == EPI_SPLIT) {
+        __nv_bfloat16 *hi = p.Rhi + (int64_t)row * p.ldr + col0;
+        __nv_bfloat16 *lo = p.Rlo + (int64_t)row * p.ldr + col0;
+        if (full) {
+            __align__(16) __nv_bfloat16 h[16], l[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                h[j] = __float2bfloat16_rn(v[j]);
+                l[j] = __float2bfloat16_rn(v[j] - __bfloat162float(h[j]));
+            }
+            reinterpret_cast<uint4 *>(hi)[0] = reinterpret_cast<uint4 *>(h)[0];
+            reinterpret_cast<uint4 *>(hi)[1] = reinterpret_cast<uint4 *>(h)[1];
+            reinterpret_cast<uint4 *>(lo)[0] = reinterpret_cast<uint4 *>(l)[0];
+            reinterpret_cast<uint4 *>(lo)[1] = reinterpret_cast<uint4 *>(l)[1];
+        } else {
+            for (int j = 0; j < 16 && col0 + j < p.N; ++j) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+                hi[j] = h;
+                lo[j] = __float2bfloat16_rn(v[j] - __bfloat162float(h));
+            }
+        }
     } else if constexpr (EPI == EPI_RHS) {
         const float ai = p.a[row];
         const float *Srow = p.S + (int64_t)row * p.ldf + col0;
@@ -326,19 +347,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
-                for (int kb = 0; kb < total_kb; ++kb, ++it) {
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    int seg = 0, k = kb;
+                    while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                    if (p.tri_k && k < (m0 > n0 ? m0 : n0) / BK) continue;
                     const int s = it % STAGES;
                     if (it >= STAGES &&
                         !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, p.err)) {
                         ok = false;
                         break;
                     }
-                    int seg = 0, k = kb;
-                    while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
                     uint8_t *a_dst = smem + s * STAGE_BYTES;
                     mbar_expect_tx(&full_bar[s], STAGE_BYTES);
                     tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
                     tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0, &full_bar[s]);
+                    ++it;
                 }
             }
         }
@@ -351,10 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             int lt = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
                 const int as = lt & 1;
+                const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
                 if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, p.err)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(as * BN);
-                for (int kb = 0; kb < total_kb; ++kb, ++it) {
+                bool first = true;
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    if (p.tri_k) {
+                        int seg = 0, k = kb;
+                        while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                        if (k < (m0 > n0 ? m0 : n0) / BK) continue;
+                    }
                     const int s = it % STAGES;
                     if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, p.err)) {
                         ok = false;
@@ -366,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0);
+                        mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
                     mma_commit(&empty_bar[s]);
+                    first = false;
+                    ++it;
                 }
                 if (ok) mma_commit(&tfull[as]);
             }
@@ -501,6 +533,7 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_RHS: return launch_bn<EPI_RHS>(maps, p, BN, s);
         case EPI_SOLVE: return launch_bn<EPI_SOLVE>(maps, p, BN, s);
         case EPI_RECON: return launch_bn<EPI_RECON>(maps, p, BN, s);
+        case EPI_SPLIT: return launch_bn<EPI_SPLIT>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -24,7 +24,7 @@ constexpr int A_TILE_BYTES = BM * BK * 2;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
-enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3 };
+enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4 };
 
 struct Maps {
     CUtensorMap a[3];
@@ -35,6 +35,7 @@ struct EpiParams {
     int M, N;
     int nseg;
     int kblocks[3];
+    int tri_k;          // operands zero for k < row index: start each tile's K at max(m0, n0)
     int *err;
     // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
     float *out;
@@ -46,6 +47,7 @@ struct EpiParams {
     const float *b;      // [N]
     int64_t ldf;
     float rho;
+    // EPI_SPLIT: Rhi/Rlo[row * ldr + col] = hi + lo bf16 split of acc
     // EPI_RHS: R = acc + rho (2 sign(S) a b^T - S) split into hi + lo bf16
     __nv_bfloat16 *Rhi, *Rlo;  // [M][ldr]
     int64_t ldr;

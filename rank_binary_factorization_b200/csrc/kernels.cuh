@@ -42,10 +42,11 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
                            __nv_bfloat16 *B, int64_t ldb, cudaStream_t s);
 
 // ---- Cholesky + inverse (cooperative, FP32) -------------------------------------
-// Gi = G^-1 for the SPD r x r matrix G (row stride r), written as hi + lo bf16 [r][ldr].
+// G = L L^T for the SPD r x r matrix G (row stride r); writes (L^-1)^T as hi + lo bf16
+// [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: (rp/64)^2 counters.
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
-                         __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr, int *err,
-                         unsigned int *bar, cudaStream_t s);
+                         __nv_bfloat16 *LiT_hi, __nv_bfloat16 *LiT_lo, int64_t ldr,
+                         unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s);
 
 // ---- SVID -------------------------------------------------------------------------
 // K power steps on |S| (S rows x r, row stride ldf): a = t/||t||, b = A^T t / ||t||.

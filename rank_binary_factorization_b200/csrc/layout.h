@@ -37,7 +37,7 @@ struct LbLayout {
     int nsv = 0;       // CTAs of an SVID pass (rows of its partial array)
     size_t scal = 0, what = 0, whatT = 0, x[2] = {0, 0}, s[2] = {0, 0}, a[2] = {0, 0},
            b[2] = {0, 0}, xt[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
-           gih = 0, gil = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
+           gih = 0, gil = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
            partb = 0, obj = 0, total = 0;
     size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
 
@@ -79,6 +79,9 @@ struct LbLayout {
         chLi = take((size_t)rp * rp * 4);
         gih = take((size_t)r * ldr * 2);
         gil = take((size_t)r * ldr * 2);
+        lth = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 hi
+        ltl = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 lo
+        chF = take((size_t)(rp / 64) * (rp / 64) * 4);  // Cholesky tile counters
         tvec = take((size_t)maxrows * 4);
         bcur = take((size_t)2 * r * 4);
         gk = take((size_t)r * 4);
