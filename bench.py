@@ -145,6 +145,19 @@ def kernel_units(cls, m, n, r, K, T):
     return None
 
 
+# DRAM bytes (read + write) per launch scope from the committed ncu captures
+# (profiles/*.md: `ncu --set full` of `bench.py --workload profile`, q_proj 4096 x 4096,
+# r = 2032, 65536-token streams).  The calibration figure scales with T x C (one read of
+# the stream); the others hold for the captured layer and rank only.
+def ncu_traffic(cls, m, n, r, T):
+    if cls == "calib":
+        return 540.4e6 * (T * max(m, n)) / (65536 * 4096)
+    if (m, n, r) != (4096, 4096, 2032):
+        return None
+    return {"chol": 20.66e6 + 9.41e6,      # chol2_kernel + EPI_SPLIT GEMM (G^-1)
+            "gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
+
+
 def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
     u = kernel_units(cls, m, n, r, K, T)
     if u is None or launches == 0 or ms <= 0:
@@ -158,7 +171,7 @@ def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
     else:
         achieved, peak, punit = amount / per_launch_s / 1e12, peaks["fp32_tflops"], "TFLOP/s"
     return dict(kernel=cls, bound=bound, achieved=round(achieved, 2), peak=round(peak, 1),
-                unit=punit, frac=round(achieved / peak, 4), traffic=None,
+                unit=punit, frac=round(achieved / peak, 4), traffic=ncu_traffic(cls, m, n, r, T),
                 launches=launches, ms_per_launch=round(ms / launches, 4),
                 share_of_step=None)
 

@@ -104,7 +104,8 @@ nq_status read_err(int *dev_err, cudaStream_t s, bool reset) {
 }
 
 size_t calib_ws_bytes(int64_t C) {
-    // token slabs * channels is bounded by 6 * 148 * 256 + C + 256 (see calib_num_slabs)
+    // token slabs * channels is at most 4 * 148 * 256 + C + 256 (see calib_num_slabs);
+    // the partial arrays are sized with headroom above that
     const size_t pd = (size_t)(6 * kNumSMsB200 * 256 + C + 256);
     return align_up(sizeof(Scalars)) + 2 * align_up(pd * 8) + 2 * align_up((size_t)C * 8);
 }

@@ -29,26 +29,37 @@ __device__ __forceinline__ void unpack16(const uint4 &raw, float (&x)[BF16 ? 8 :
     }
 }
 
+// Streaming 16-byte load that is not kept in L1 (each byte is read once).
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // CTA = 8 warps over one slab of 32*VEC channels; warp w takes tokens w, w+8, ...
 // of the CTA's token slab; each lane owns VEC consecutive channels (one 16-byte load
-// per token).  FP32 sums over 16 tokens are flushed into FP64 accumulators.
+// per token) and keeps 8 loads in flight.  FP32 sums over 16 tokens are added into the
+// warp's FP64 accumulators in shared memory (laid out [v][lane]: no bank conflicts),
+// which keeps the register count low enough for 4 CTAs (32 warps) per SM.
 template <bool BF16>
-__global__ void __launch_bounds__(256) calib_partial_vec(const void *__restrict__ Xv, int64_t T,
-                                                         int64_t C, int64_t tok_per_slab,
-                                                         double *__restrict__ ps,
-                                                         double *__restrict__ pq) {
+__global__ void __launch_bounds__(256, 4) calib_partial_vec(const void *__restrict__ Xv, int64_t T,
+                                                            int64_t C, int64_t tok_per_slab,
+                                                            double *__restrict__ ps,
+                                                            double *__restrict__ pq) {
     constexpr int VEC = BF16 ? 8 : 4;
     constexpr int ESZ = BF16 ? 2 : 4;
-    __shared__ double sh_s[8][32 * VEC];
-    __shared__ double sh_q[8][32 * VEC];
+    constexpr int U = 8;  // loads in flight per thread
+    __shared__ double sh_s[8][VEC][32];
+    __shared__ double sh_q[8][VEC][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t cbase = (int64_t)blockIdx.x * 32 * VEC;
     const int64_t c0 = cbase + lane * VEC;
     const int64_t t_begin = (int64_t)blockIdx.y * tok_per_slab;
     const int64_t t_end = min(T, t_begin + tok_per_slab);
-    double ds[VEC], dq[VEC];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) ds[v] = dq[v] = 0.0;
+    for (int v = 0; v < VEC; ++v) sh_s[warp][v][lane] = sh_q[warp][v][lane] = 0.0;
     if (c0 < C) {
         const char *base = reinterpret_cast<const char *>(Xv) + c0 * ESZ;
         const int64_t row_bytes = C * ESZ;
@@ -58,13 +69,12 @@ __global__ void __launch_bounds__(256) calib_partial_vec(const void *__restrict_
 #pragma unroll
             for (int v = 0; v < VEC; ++v) fs[v] = fq[v] = 0.f;
             int cnt = 0;
-            for (; t + 24 < t_end && cnt < 16; t += 32, cnt += 4) {
-                uint4 raw[4];
+            for (; cnt < 16 && t + 8 * (U - 1) < t_end; cnt += U, t += 8 * U) {
+                uint4 raw[U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    raw[u] = __ldcs(reinterpret_cast<const uint4 *>(base + (t + 8 * u) * row_bytes));
+                for (int u = 0; u < U; ++u) raw[u] = ld_stream16(base + (t + 8 * u) * row_bytes);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < U; ++u) {
                     float x[VEC];
                     unpack16<BF16>(raw[u], x);
 #pragma unroll
@@ -75,9 +85,9 @@ __global__ void __launch_bounds__(256) calib_partial_vec(const void *__restrict_
                     }
                 }
             }
-            for (; t < t_end && cnt < 16; t += 8, ++cnt) {
+            for (; cnt < 16 && t < t_end; ++cnt, t += 8) {
                 float x[VEC];
-                unpack16<BF16>(__ldcs(reinterpret_cast<const uint4 *>(base + t * row_bytes)), x);
+                unpack16<BF16>(ld_stream16(base + t * row_bytes), x);
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) {
                     const float x2 = x[v] * x[v];
@@ -87,24 +97,20 @@ __global__ void __launch_bounds__(256) calib_partial_vec(const void *__restrict_
             }
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
-                ds[v] += fs[v];
-                dq[v] += fq[v];
+                sh_s[warp][v][lane] += fs[v];
+                sh_q[warp][v][lane] += fq[v];
             }
         }
-    }
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-        sh_s[warp][lane * VEC + v] = ds[v];
-        sh_q[warp][lane * VEC + v] = dq[v];
     }
     __syncthreads();
     for (int c = threadIdx.x; c < 32 * VEC; c += blockDim.x) {
         if (cbase + c >= C) continue;
+        const int v = c % VEC, l = c / VEC;
         double a = 0.0, b = 0.0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-            a += sh_s[w][c];
-            b += sh_q[w][c];
+            a += sh_s[w][v][l];
+            b += sh_q[w][v][l];
         }
         ps[(int64_t)blockIdx.y * C + cbase + c] = a;
         pq[(int64_t)blockIdx.y * C + cbase + c] = b;
@@ -142,9 +148,11 @@ __global__ void __launch_bounds__(256) calib_partial_scalar(const void *__restri
     pq[(int64_t)blockIdx.y * C + c] = dq;
 }
 
+// Token slabs: as many CTAs as fit in one wave (4 CTAs of 256 channels per SM) without
+// spilling a partial second wave.
 int calib_num_slabs(int64_t T, int64_t C) {
     const int64_t cx = ceil_div(C, 256);
-    int64_t ns = ceil_div(6 * kNumSMsB200, cx);
+    int64_t ns = (4 * kNumSMsB200) / cx;
     const int64_t max_by_T = ceil_div(T, 256);
     if (ns > max_by_T) ns = max_by_T;
     if (ns < 1) ns = 1;
