@@ -12,8 +12,9 @@
 //     of a diagonal tile is not on the chain of block steps; the diagonal inverses are
 //     formed afterwards, one CTA per tile, all at once;
 //   * the 64 x 64 tile Cholesky works in 16-column blocks factored by one warp with
-//     shuffles (no CTA barrier per column); panel rows are independent substitutions,
-//     one thread per row with no barrier at all;
+//     shuffles (no CTA barrier per column); the diagonal tile is inverted right away
+//     (warp-parallel 16 x 16 blocks, two doubling levels), so every panel tile is one
+//     tile product A_ij L_jj^-T;
 //   * (L^-1)_21 = -L22^-1 L21 L11^-1 level by level (log2(r/64) levels, two barriers each);
 //   * (L^-1)^T is written as bf16 hi + lo; G^-1 = L^-T L^-1 is then one split-BF16
 //     tensor-core GEMM (see gemm_tc.cu, EPI_SPLIT).
@@ -157,9 +158,11 @@ __device__ __forceinline__ void put(float *M, int64_t ld, int ti, int tj, const 
 
 // ---- 64 x 64 tile Cholesky: four 16-column blocks -----------------------------------
 // Block b: all threads subtract the finished columns from block column b (rows 16b ..
-// 63), then warp 0 factors it column by column with shuffles (lane l holds rows
-// 16b + l and 16b + l + 32), so the 64 sequential column steps need no CTA barrier.
-__device__ void chol_tile(Tile &s, int *err) {
+// 63), then warp 0 factors it column by column (lane l holds rows 16b + l and
+// 16b + l + 32).  Column k's multipliers of the block's diagonal rows are broadcast by
+// shuffles; every lane also keeps the 16 diagonal entries of the block and updates them
+// from those broadcasts, so the next pivot needs no shuffle.  rdiag[c] = 1 / L_cc.
+__device__ void chol_tile(Tile &s, float *rdiag, int *err) {
     const int t = threadIdx.x, lane = t & 31;
     bool bad = false;
 #pragma unroll 1
@@ -183,28 +186,31 @@ __device__ void chol_tile(Tile &s, int *err) {
         }
         if (t < 32) {
             const int r0 = c0 + lane, r1 = r0 + 32;
-            float a0[16], a1[16];
+            float a0[16], a1[16], d[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 a0[c] = (r0 < TB) ? s[r0][c0 + c] : 0.f;
                 a1[c] = (r1 < TB) ? s[r1][c0 + c] : 0.f;
+                d[c] = s[c0 + c][c0 + c];
             }
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                float piv = __shfl_sync(0xffffffffu, a0[k], k);
+                float piv = d[k];
                 if (!(piv > 0.f)) {
                     bad = true;
                     piv = 1e-30f;
                 }
                 const float il = rsqrtf(piv);
+                if (lane == 0) rdiag[c0 + k] = il;
                 const float l0 = a0[k] * il, l1 = a1[k] * il;
                 a0[k] = l0;
                 a1[k] = l1;
 #pragma unroll
                 for (int c = k + 1; c < 16; ++c) {
-                    const float lc = __shfl_sync(0xffffffffu, l0, c);
+                    const float lc = __shfl_sync(0xffffffffu, l0, c);  // L_{c0+c, c0+k}
                     a0[c] = fmaf(-l0, lc, a0[c]);
                     a1[c] = fmaf(-l1, lc, a1[c]);
+                    d[c] = fmaf(-lc, lc, d[c]);
                 }
             }
 #pragma unroll
@@ -223,95 +229,96 @@ __device__ void chol_tile(Tile &s, int *err) {
     __syncthreads();
 }
 
-// ---- panel: X L_jj^T = A for a 64 x 64 tile, one thread per row ----------------------
-// Rows are independent forward substitutions, so they need no synchronisation.  The
-// thread keeps its row in registers as a window x[0..W) over columns c0 .. c0 + W - 1;
-// after each quad of 4 columns the finished values are stored and the window shifts by
-// 4.  W is the remaining width rounded up to 16 (64, 48, 32, 16): lt rows are padded with
-// zeros to LTW columns so the last window reads zeros past column 63.
-constexpr int LTW = 80;  // >= 60 + 16, multiple of 4
-using LtTile = float[TB][LTW];
+// ---- inverse of a lower-triangular 64 x 64 tile ------------------------------------
+// li = L^-1 (plain, zero above the diagonal), lit = (L^-1)^T.  The four 16 x 16 diagonal
+// blocks are inverted by four warps at once (lane = column, forward substitution with the
+// reciprocal diagonal rdiag); two doubling levels then form the off-diagonal blocks,
+// Li21 = -Li22 (L21 Li11), with tmp as scratch.
+template <int H>
+__device__ __forceinline__ void inv_level(const Tile &s, Tile &li, Tile &tmp) {
+    // thread job: one pair pr, one row a, four columns b .. b+3; entries above the
+    // diagonal of li are zero, so the K loops run over the full block (no predicates)
+    constexpr int NP = TB / (2 * H), G = H / 4;
+    for (int e = threadIdx.x; e < NP * H * G; e += blockDim.x) {  // tmp = L21 Li11
+        const int pr = e / (H * G), a = (e / G) % H, b = 4 * (e % G), o = 2 * H * pr;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < H; ++c) {
+            const float l = s[o + H + a][o + c];
+            const float4 y = *reinterpret_cast<const float4 *>(&li[o + c][o + b]);
+            acc.x = fmaf(l, y.x, acc.x);
+            acc.y = fmaf(l, y.y, acc.y);
+            acc.z = fmaf(l, y.z, acc.z);
+            acc.w = fmaf(l, y.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(&tmp[o + a][b]) = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < NP * H * G; e += blockDim.x) {  // Li21 = -Li22 tmp
+        const int pr = e / (H * G), a = (e / G) % H, b = 4 * (e % G), o = 2 * H * pr;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < H; ++c) {
+            const float l = li[o + H + a][o + H + c];
+            const float4 y = *reinterpret_cast<const float4 *>(&tmp[o + c][b]);
+            acc.x = fmaf(l, y.x, acc.x);
+            acc.y = fmaf(l, y.y, acc.y);
+            acc.z = fmaf(l, y.z, acc.z);
+            acc.w = fmaf(l, y.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(&li[o + H + a][o + b]) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+}
 
-template <int W, bool COL>
-__device__ __forceinline__ void subst_quad(float (&x)[64], const LtTile &lt, const float *dinv,
-                                           int c0, float *dst, int64_t ld) {
+__device__ void inverse_tile(const Tile &s, const float *rdiag, Tile &li, Tile &lit, Tile &tmp) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    for (int e = t; e < TB * TB; e += blockDim.x) li[e >> 6][e & 63] = 0.f;
+    __syncthreads();
+    if (warp < 4 && lane < 16) {  // diagonal 16 x 16 blocks: column `lane` of each inverse
+        const int o = 16 * warp;
+        float x[16];
 #pragma unroll
-    for (int g2 = 0; g2 < 4; ++g2) {
-        const int c = c0 + g2;
-        const float xc = x[g2] * dinv[c];
-        x[g2] = xc;
+        for (int c = 0; c < 16; ++c) x[c] = (c == lane) ? 1.f : 0.f;
 #pragma unroll
-        for (int m = 0; m < W / 4; ++m) {
-            const float4 l = *reinterpret_cast<const float4 *>(&lt[c][c0 + 4 * m]);
-            const float lv[4] = {l.x, l.y, l.z, l.w};
+        for (int c = 0; c < 16; ++c) {
+            x[c] *= rdiag[o + c];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if (4 * m + e > g2) x[4 * m + e] = fmaf(-xc, lv[e], x[4 * m + e]);
+            for (int k = c + 1; k < 16; ++k) x[k] = fmaf(-s[o + k][o + c], x[c], x[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) li[o + k][o + lane] = x[k];
+    }
+    __syncthreads();
+    inv_level<16>(s, li, tmp);
+    inv_level<32>(s, li, tmp);
+    for (int e = t; e < TB * TB; e += blockDim.x) {
+        const int c = e >> 6, b = e & 63;
+        lit[b][c] = li[c][b];
+    }
+    __syncthreads();
+}
+
+// Several counters at once: warp w < 3 polls counter w (null: none), then a CTA barrier.
+__device__ __forceinline__ void wait_counts(const unsigned int *c0, unsigned int v0,
+                                            const unsigned int *c1, unsigned int v1,
+                                            const unsigned int *c2, unsigned int v2, int *err) {
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0 && w < 3 && !(*(volatile int *)err == NQ_ERR_TIMEOUT)) {
+        const unsigned int *c = (w == 0) ? c0 : ((w == 1) ? c1 : c2);
+        const unsigned int v = (w == 0) ? v0 : ((w == 1) ? v1 : v2);
+        if (c) {
+            uint32_t spins = 0;
+            while (ld_acquire_gpu(c) < v) {
+                if (++spins > kGridSpinLimit) {
+                    raise_error(err, NQ_ERR_TIMEOUT);
+                    break;
+                }
+                if (spins > 64) __nanosleep(32);
+            }
         }
     }
-    if (COL) {  // entries c0 .. c0 + 3 of a column: rows of the output
-#pragma unroll
-        for (int e = 0; e < 4; ++e) __stcg(dst + (int64_t)(c0 + e) * ld, x[e]);
-    } else {
-        __stcg(reinterpret_cast<float4 *>(dst + c0), make_float4(x[0], x[1], x[2], x[3]));
-    }
-#pragma unroll
-    for (int p = 0; p < W - 4; ++p) x[p] = x[p + 4];
-}
-
-template <bool COL>
-__device__ __forceinline__ void subst_run(float (&x)[64], const LtTile &lt, const float *dinv,
-                                          float *dst, int64_t ld) {
-#pragma unroll 1
-    for (int qb = 0; qb < 16; ++qb) {
-        const int c0 = 4 * qb;
-        if (qb < 4)
-            subst_quad<64, COL>(x, lt, dinv, c0, dst, ld);
-        else if (qb < 8)
-            subst_quad<48, COL>(x, lt, dinv, c0, dst, ld);
-        else if (qb < 12)
-            subst_quad<32, COL>(x, lt, dinv, c0, dst, ld);
-        else
-            subst_quad<16, COL>(x, lt, dinv, c0, dst, ld);
-    }
-}
-
-// Row `row` of the tile at Ag (row stride ld) is replaced by its solution x, x L^T = a.
-// lt[c][k] = L_kc (zero for k >= 64), dinv[c] = 1 / L_cc.
-__device__ void panel_row(float *Ag, int64_t ld, int row, const LtTile &lt, const float *dinv) {
-    float *rp = Ag + (int64_t)row * ld;
-    float x[64];
-#pragma unroll
-    for (int p = 0; p < 64; p += 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(rp + p));
-        x[p] = v.x;
-        x[p + 1] = v.y;
-        x[p + 2] = v.z;
-        x[p + 3] = v.w;
-    }
-    subst_run<false>(x, lt, dinv, rp, ld);
-}
-
-// Column `col` of L^-1 (L x = e_col) into the tile at Og (row stride ld).
-__device__ void inverse_col(float *Og, int64_t ld, int col, const LtTile &lt, const float *dinv) {
-    float x[64];
-#pragma unroll
-    for (int p = 0; p < 64; ++p) x[p] = (p == col) ? 1.f : 0.f;
-    subst_run<true>(x, lt, dinv, Og + col, ld);
-}
-
-// lt[c][k] = L_kc for the lower tile (ti, ti) of A (zero-padded to LTW), dinv[c] = 1/L_cc.
-__device__ void load_lt(LtTile &lt, float *dinv, const float *A, int64_t ld, int ti) {
-    const float *L = A + (int64_t)ti * TB * ld + (int64_t)ti * TB;
-    __syncthreads();
-    for (int e = threadIdx.x; e < TB * TB; e += blockDim.x) {
-        const int k = e >> 6, c = e & 63;  // coalesced read of row k
-        lt[c][k] = __ldcg(L + (int64_t)k * ld + c);
-    }
-    for (int e = threadIdx.x; e < TB * (LTW - TB); e += blockDim.x)
-        lt[e / (LTW - TB)][TB + e % (LTW - TB)] = 0.f;
-    __syncthreads();
-    if (threadIdx.x < TB) dinv[threadIdx.x] = 1.f / lt[threadIdx.x][threadIdx.x];
     __syncthreads();
 }
 
@@ -327,19 +334,6 @@ __device__ __forceinline__ int64_t dealt_job(int64_t k) {
 // 0 .. k-1, then its Cholesky (i == k) or panel solve (i > k).  A task waits until the
 // counters of its operands reach the required values; waits are bounded and, once one
 // has timed out, skipped.
-__device__ __forceinline__ void wait_count(const unsigned int *c, unsigned int target, int *err) {
-    if (threadIdx.x == 0 && !(*(volatile int *)err == NQ_ERR_TIMEOUT)) {
-        uint32_t spins = 0;
-        while (ld_acquire_gpu(c) < target) {
-            if (++spins > kGridSpinLimit) {
-                raise_error(err, NQ_ERR_TIMEOUT);
-                break;
-            }
-            if (spins > 64) __nanosleep(32);
-        }
-    }
-    __syncthreads();
-}
 __device__ __forceinline__ void signal_count(unsigned int *c, unsigned int inc) {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -374,44 +368,46 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             dst[j] = (i < p.r && j < p.r) ? __ldg(src + j) : (i == j ? 1.f : 0.f);
     }
     grid_barrier(p.bar, p.err);
-    Tile &cb = *reinterpret_cast<Tile *>(smem_f + 3 * TB * LDS);  // published columns
-    float *rpv = smem_f + 4 * TB * LDS;     // 64 reciprocal pivots
-    float *dinv = rpv + 64;                 // 64 reciprocals of the current L_jj diagonal
-    LtTile &lt = *reinterpret_cast<LtTile *>(smem_f + 4 * TB * LDS + 128);  // L_jj^T, padded
-    // Dataflow factorisation.  CTA 0 runs the critical chain: Cholesky of (j, j), panel
-    // tile (j+1, j) from the L_jj it holds in shared memory, update of (j+1, j+1) and its
-    // Cholesky.  CTAs 1.. take the other panel tiles and trailing updates round-robin in
-    // a topological order (step by step), so every wait ends.
+    Tile &t3 = *reinterpret_cast<Tile *>(smem_f + 3 * TB * LDS);
+    Tile &t4 = *reinterpret_cast<Tile *>(smem_f + 4 * TB * LDS);
+    float *rdiag = smem_f + 5 * TB * LDS;  // 1 / L_cc of the tile just factored
+    // Dataflow factorisation.  CTA 0 runs the critical chain: Cholesky of the diagonal
+    // tile and its inverse (kept in shared memory), the panel tile below it as one tile
+    // product, the look-ahead update of the next diagonal tile.  CTAs 1.. take the other
+    // panel tiles (A_ij L_jj^-T, with L_jj^-1 from the Li diagonal tile) and the trailing
+    // updates round-robin in a topological order (step by step), so every wait ends.
     auto CNT = [&](int i, int k) { return p.cnt + (int64_t)i * nb + k; };
     if (blockIdx.x == 0) {
+        // t2: L_jj, t3: L_jj^-1, t4: (L_jj^-1)^T, t0: panel operand, t1: panel^T
         load_n(t2, p.A, rp, 0, 0);
         __syncthreads();
-        chol_tile(t2, p.err);
+        chol_tile(t2, rdiag, p.err);
+        inverse_tile(t2, rdiag, t3, t4, t1);
         store_n(p.A, rp, 0, 0, t2);
+        store_n(p.Li, rp, 0, 0, t3);
         signal_count(CNT(0, 0), 1);
         for (int j = 0; j + 1 < nb; ++j) {
-            // t2 holds L_jj: build lt, dinv from it
-            __syncthreads();
-            for (int e = threadIdx.x; e < TB * LTW; e += blockDim.x) {
-                const int c = e / LTW, k = e % LTW;
-                lt[c][k] = (k < TB) ? t2[k][c] : 0.f;
-            }
-            __syncthreads();
-            if (threadIdx.x < TB) dinv[threadIdx.x] = 1.f / t2[threadIdx.x][threadIdx.x];
-            wait_count(CNT(j + 1, j), j, p.err);  // its j updates
-            if (threadIdx.x < TB)
-                panel_row(p.A + (int64_t)(j + 1) * TB * rp + (int64_t)j * TB, rp, threadIdx.x, lt,
-                          dinv);
-            signal_count(CNT(j + 1, j), 1);
-            // look-ahead: (j+1, j+1) -= L_{j+1,j} L_{j+1,j}^T, then its Cholesky
-            wait_count(CNT(j + 1, j + 1), j, p.err);
-            load_t(t0, p.A, rp, j + 1, j);
-            load_n(t2, p.A, rp, j + 1, j + 1);
+            wait_counts(CNT(j + 1, j), j, CNT(j + 1, j + 1), j, nullptr, 0, p.err);
+            load_n_async(t0, p.A, rp, j + 1, j);       // panel tile, all j updates applied
+            load_n_async(t2, p.A, rp, j + 1, j + 1);   // next diagonal tile
+            cp_async_wait<1>();
             __syncthreads();
             float acc[4][4];
             zero(acc);
-            mac(acc, t0, t0);
+            mac_n(acc, t0, t4);                        // L_{j+1,j} = A_{j+1,j} L_jj^-T
+            put(p.A, rp, j + 1, j, acc, 1.f);
+            {
+                const int a0 = blk_a0(), b0 = blk_b0();
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) t1[b0 + q][a0 + i] = acc[i][q];
+            }
+            signal_count(CNT(j + 1, j), 1);
+            cp_async_wait<0>();
             __syncthreads();
+            zero(acc);
+            mac(acc, t1, t1);                          // L_{j+1,j} L_{j+1,j}^T
             {
                 const int a0 = blk_a0(), b0 = blk_b0();
 #pragma unroll
@@ -420,8 +416,10 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     for (int q = 0; q < 4; ++q) t2[a0 + i][b0 + q] -= acc[i][q];
             }
             __syncthreads();
-            chol_tile(t2, p.err);
+            chol_tile(t2, rdiag, p.err);
+            inverse_tile(t2, rdiag, t3, t4, t1);
             store_n(p.A, rp, j + 1, j + 1, t2);
+            store_n(p.Li, rp, j + 1, j + 1, t3);
             signal_count(CNT(j + 1, j + 1), 2);
         }
     } else {
@@ -434,27 +432,26 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             const int64_t n = P + U;
             for (int64_t idx = base + ((w - base % W) % W + W) % W; idx < base + n; idx += W) {
                 const int64_t loc = idx - base;
-                if (loc < P) {  // panel tile (i, j)
+                float acc[4][4];
+                zero(acc);
+                if (loc < P) {  // panel tile (i, j) = A_ij L_jj^-T
                     const int i = j + 2 + (int)loc;
-                    wait_count(CNT(j, j), j + 1, p.err);
-                    load_lt(lt, dinv, p.A, rp, j);
-                    wait_count(CNT(i, j), j, p.err);
-                    if (threadIdx.x < TB)
-                        panel_row(p.A + (int64_t)i * TB * rp + (int64_t)j * TB, rp, threadIdx.x,
-                                  lt, dinv);
+                    wait_counts(CNT(j, j), j + 1, CNT(i, j), j, nullptr, 0, p.err);
+                    load_n_async(t0, p.A, rp, i, j);
+                    load_t(t4, p.Li, rp, j, j);       // t4[c][x] = Li_jj[x][c]
+                    cp_async_wait<0>();
+                    __syncthreads();
+                    mac_n(acc, t0, t4);
+                    put(p.A, rp, i, j, acc, 1.f);
                     signal_count(CNT(i, j), 1);
                 } else {  // update of tile (i, k) with step j: A_ik -= L_ij L_kj^T
                     int ii, kk;
                     tri_index(loc - P + 1, ii, kk);
                     const int i = j + 1 + ii, k = j + 1 + kk;
-                    wait_count(CNT(i, j), j + 1, p.err);
-                    wait_count(CNT(k, j), j + 1, p.err);
-                    wait_count(CNT(i, k), j, p.err);
+                    wait_counts(CNT(i, j), j + 1, CNT(k, j), j + 1, CNT(i, k), j, p.err);
                     load_t(t0, p.A, rp, i, j);
                     load_t(t1, p.A, rp, k, j);
                     __syncthreads();
-                    float acc[4][4];
-                    zero(acc);
                     mac(acc, t0, t1);
                     const int a0 = blk_a0(), b0 = blk_b0();
                     float *bp = p.A + ((int64_t)i * TB + a0) * rp + (int64_t)k * TB + b0;
@@ -469,17 +466,10 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     }
                     signal_count(CNT(i, k), 1);
                 }
+                __syncthreads();  // shared tiles free for the next task
             }
             base += n;
         }
-    }
-    grid_barrier(p.bar, p.err);
-
-    // inverses of all diagonal tiles in parallel: column substitutions L x = e_c
-    for (int d = blockIdx.x; d < nb; d += gridDim.x) {
-        load_lt(lt, dinv, p.A, rp, d);
-        if (threadIdx.x < TB)
-            inverse_col(p.Li + (int64_t)d * TB * rp + (int64_t)d * TB, rp, threadIdx.x, lt, dinv);
     }
     grid_barrier(p.bar, p.err);
 
@@ -515,10 +505,10 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                 float acc[4][4];
                 zero(acc);
                 __syncthreads();
-                // stage 0: X in t0, Y in t1; stage 1: X in t2, Y in cb
+                // stage 0: X in t0, Y in t1; stage 1: X in t2, Y in t3
                 auto issue = [&](int c, int st) {
                     Tile &X = st ? t2 : t0;
-                    Tile &Y = st ? cb : t1;
+                    Tile &Y = st ? t3 : t1;
                     if (half == 0) {
                         load_n_async(X, p.A, rp, a, c);   // L(a, c)
                         load_n_async(Y, p.Li, rp, c, b);  // Li(c, b)
@@ -537,7 +527,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                         cp_async_wait<0>();
                     }
                     __syncthreads();
-                    mac_n(acc, st ? t2 : t0, st ? cb : t1);
+                    mac_n(acc, st ? t2 : t0, st ? t3 : t1);
                     __syncthreads();
                 }
                 if (half == 0)
@@ -600,7 +590,7 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
                          __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
-    constexpr int smem = (4 * TB * LDS + 128 + TB * LTW) * sizeof(float);
+    constexpr int smem = (5 * TB * LDS + TB) * sizeof(float);
     static int grid = 0;
     if (!grid) {
         cudaError_t e = cudaFuncSetAttribute(chol2_kernel,
