@@ -1,21 +1,22 @@
-// Cholesky G = L L^T of the r x r SPD system matrix of the U (V) step and L^-1 by
-// recursive doubling; (L^-1)^T is emitted as BF16 hi + lo for the tensor-core product
-// G^-1 = L^-T L^-1.  NanoQuant summary page, "Core method" (核心方法), step (a): the
-// regularised linear system is solved through a Cholesky factorisation.
+// Cholesky G = L L^T of the r x r SPD system matrix of the U (V) step and L^-1;
+// (L^-1)^T is emitted as BF16 hi + lo for the tensor-core product G^-1 = L^-T L^-1.
+// NanoQuant summary page, "Core method" (核心方法), step (a): the regularised linear
+// system is solved through a Cholesky factorisation.
 //
-// One cooperative launch of FP32 SIMT work on 64 x 64 tiles (4 x 4 register blocks per
-// thread, float4 traffic) with bounded grid barriers:
-//   * right-looking blocked Cholesky with look-ahead: while CTAs 1.. apply the trailing
-//     update of step j, CTA 0 updates the next diagonal tile and factors it, so a step
-//     costs two barriers and the diagonal factorisation overlaps the update;
-//   * panel tiles are solved by forward substitution (all in parallel), so the inverse
-//     of a diagonal tile is not on the chain of block steps; the diagonal inverses are
-//     formed afterwards, one CTA per tile, all at once;
+// One cooperative launch (one CTA of 256 threads per SM) of FP32 SIMT work on 64 x 64
+// tiles, scheduled as a dataflow with per-tile completion counters (bounded waits):
+//   * CTA 0 runs the critical chain of the blocked right-looking factorisation: tile
+//     Cholesky of the diagonal tile, its inverse, the panel tile below it (one tile
+//     product A L_jj^-T) and the look-ahead update of the next diagonal tile;
+//   * CTA 1 takes the tasks CTA 0 needs next (panel (j+2, j), updates of (j+2, j+1) and
+//     (j+2, j+2)); CTAs 2.. take the other panel tiles and the trailing updates
+//     round-robin in a topological order, so every wait ends;
 //   * the 64 x 64 tile Cholesky works in 16-column blocks factored by one warp with
-//     shuffles (no CTA barrier per column); the diagonal tile is inverted right away
-//     (warp-parallel 16 x 16 blocks, two doubling levels), so every panel tile is one
-//     tile product A_ij L_jj^-T;
-//   * (L^-1)_21 = -L22^-1 L21 L11^-1 level by level (log2(r/64) levels, two barriers each);
+//     shuffles (no CTA barrier per column); the tile inverse takes 16 x 16 diagonal blocks
+//     in four warps at once and two doubling levels;
+//   * L^-1 in the same dataflow: block column m is a forward substitution advanced one
+//     block row per factorisation step (X_jm = -L_jj^-1 sum_k L_jk X_km), so the inverse
+//     trails the factorisation instead of following it;
 //   * (L^-1)^T is written as bf16 hi + lo; G^-1 = L^-T L^-1 is then one split-BF16
 //     tensor-core GEMM (see gemm_tc.cu, EPI_SPLIT).
 #include "kernels.cuh"
@@ -37,7 +38,7 @@ struct Chol2Args {
     float *Li;    // rp x rp: L^-1 (lower tiles), scratch T in upper tiles
     __nv_bfloat16 *hi, *lo;
     int64_t ldr;
-    unsigned int *cnt;  // nb x nb: operations completed on tile (i, k)
+    unsigned int *cnt;  // 2 x nb x nb: operations completed on tile (i, k) of L, of L^-1
     int *err;
     unsigned int *bar;
 };
@@ -300,33 +301,37 @@ __device__ void inverse_tile(const Tile &s, const float *rdiag, Tile &li, Tile &
     __syncthreads();
 }
 
+// lower-triangular enumeration idx -> (ii >= kk)
+__device__ __forceinline__ void tri_index(int64_t idx, int &ii, int &kk) {
+    int a = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
+    while ((int64_t)(a + 1) * (a + 2) / 2 <= idx) ++a;
+    while ((int64_t)a * (a + 1) / 2 > idx) --a;
+    ii = a;
+    kk = (int)(idx - (int64_t)a * (a + 1) / 2);
+}
+
+// Bounded poll of one counter by the calling thread (null: nothing to wait for).
+__device__ __forceinline__ void poll_count(const unsigned int *c, unsigned int v, int *err) {
+    if (!c || *(volatile int *)err == NQ_ERR_TIMEOUT) return;
+    uint32_t spins = 0;
+    while (ld_acquire_gpu(c) < v) {
+        if (++spins > kGridSpinLimit) {
+            raise_error(err, NQ_ERR_TIMEOUT);
+            return;
+        }
+        if (spins > 64) __nanosleep(32);
+    }
+}
+
 // Several counters at once: warp w < 3 polls counter w (null: none), then a CTA barrier.
 __device__ __forceinline__ void wait_counts(const unsigned int *c0, unsigned int v0,
                                             const unsigned int *c1, unsigned int v1,
                                             const unsigned int *c2, unsigned int v2, int *err) {
     const int w = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0 && w < 3 && !(*(volatile int *)err == NQ_ERR_TIMEOUT)) {
-        const unsigned int *c = (w == 0) ? c0 : ((w == 1) ? c1 : c2);
-        const unsigned int v = (w == 0) ? v0 : ((w == 1) ? v1 : v2);
-        if (c) {
-            uint32_t spins = 0;
-            while (ld_acquire_gpu(c) < v) {
-                if (++spins > kGridSpinLimit) {
-                    raise_error(err, NQ_ERR_TIMEOUT);
-                    break;
-                }
-                if (spins > 64) __nanosleep(32);
-            }
-        }
-    }
+    if ((threadIdx.x & 31) == 0 && w < 3)
+        poll_count((w == 0) ? c0 : ((w == 1) ? c1 : c2), (w == 0) ? v0 : ((w == 1) ? v1 : v2),
+                   err);
     __syncthreads();
-}
-
-// Job order for a CTA: rounds of gridDim.x jobs dealt in alternating direction, so
-// that with jobs sorted by decreasing cost the per-CTA totals stay balanced.
-__device__ __forceinline__ int64_t dealt_job(int64_t k) {
-    const int64_t G = gridDim.x;
-    return k * G + ((k & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
 }
 
 // ---- tile counters of the factorisation ------------------------------------------
@@ -340,15 +345,6 @@ __device__ __forceinline__ void signal_count(unsigned int *c, unsigned int inc) 
         __threadfence();
         atomicAdd(c, inc);
     }
-}
-
-// lower-triangular enumeration idx -> (ii >= kk)
-__device__ __forceinline__ void tri_index(int64_t idx, int &ii, int &kk) {
-    int a = (int)((sqrt(8.0 * (double)idx + 1.0) - 1.0) * 0.5);
-    while ((int64_t)(a + 1) * (a + 2) / 2 <= idx) ++a;
-    while ((int64_t)a * (a + 1) / 2 > idx) --a;
-    ii = a;
-    kk = (int)(idx - (int64_t)a * (a + 1) / 2);
 }
 
 __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
@@ -377,6 +373,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
     // panel tiles (A_ij L_jj^-T, with L_jj^-1 from the Li diagonal tile) and the trailing
     // updates round-robin in a topological order (step by step), so every wait ends.
     auto CNT = [&](int i, int k) { return p.cnt + (int64_t)i * nb + k; };
+    auto ICNT = [&](int i, int k) { return p.cnt + (int64_t)(nb + i) * nb + k; };  // L^-1 tiles
     if (blockIdx.x == 0) {
         // t2: L_jj, t3: L_jj^-1, t4: (L_jj^-1)^T, t0: panel operand, t1: panel^T
         load_n(t2, p.A, rp, 0, 0);
@@ -422,20 +419,83 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             store_n(p.Li, rp, j + 1, j + 1, t3);
             signal_count(CNT(j + 1, j + 1), 2);
         }
+    } else if (blockIdx.x == 1) {
+        // CTA 1 takes the tasks CTA 0 needs next: panel (j+2, j) and the step-j updates of
+        // (j+2, j+1) and (j+2, j+2), keeping the panel in shared memory.
+        for (int j = 0; j + 2 < nb; ++j) {
+            float acc[4][4];
+            zero(acc);
+            wait_counts(CNT(j, j), j + 1, CNT(j + 2, j), j, nullptr, 0, p.err);
+            load_n_async(t0, p.A, rp, j + 2, j);
+            load_t(t4, p.Li, rp, j, j);
+            cp_async_wait<0>();
+            __syncthreads();
+            mac_n(acc, t0, t4);                        // L_{j+2,j} = A_{j+2,j} L_jj^-T
+            put(p.A, rp, j + 2, j, acc, 1.f);
+            {
+                const int a0 = blk_a0(), b0 = blk_b0();
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) t1[b0 + q][a0 + i] = acc[i][q];
+            }
+            signal_count(CNT(j + 2, j), 1);
+            wait_counts(CNT(j + 1, j), j + 1, CNT(j + 2, j + 1), j, CNT(j + 2, j + 2), j, p.err);
+            load_t(t0, p.A, rp, j + 1, j);           // t0 = L_{j+1,j}^T
+            __syncthreads();
+            for (int h = 0; h < 2; ++h) {              // h = 0: tile (j+2, j+1); 1: (j+2, j+2)
+                zero(acc);
+                mac(acc, t1, h ? t1 : t0);
+                const int a0 = blk_a0(), b0 = blk_b0();
+                float *bp = p.A + ((int64_t)(j + 2) * TB + a0) * rp + (int64_t)(j + 1 + h) * TB + b0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float4 v = __ldcg(reinterpret_cast<const float4 *>(bp + (int64_t)q * rp));
+                    v.x -= acc[q][0];
+                    v.y -= acc[q][1];
+                    v.z -= acc[q][2];
+                    v.w -= acc[q][3];
+                    __stcg(reinterpret_cast<float4 *>(bp + (int64_t)q * rp), v);
+                }
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                __threadfence();
+                atomicAdd(CNT(j + 2, j + 1), 1u);
+                atomicAdd(CNT(j + 2, j + 2), 1u);
+            }
+            __syncthreads();
+        }
     } else {
-        const int64_t W = gridDim.x - 1, w = blockIdx.x - 1;
+        // Worker tasks of step j, in this order: panel tiles (i, j), i >= j+3; trailing
+        // updates of step j; L^-1 tasks: finalise X_jm = -L_jj^-1 acc_jm (m < j), then
+        // acc_im += L_ij X_jm for m <= j < i (block column m of L^-1 is a forward
+        // substitution, advanced one block row per step of the factorisation).  The L^-1
+        // tasks of step j are placed after the factorisation tasks of step j + 1 (still a
+        // topological order), so the tasks CTA 0 waits for come first.  One tile per task:
+        // grouping tiles that share an operand serialises them on one CTA and was slower.
+        const int64_t W = gridDim.x - 2, w = blockIdx.x - 2;
         int64_t base = 0;
-        for (int j = 0; j + 1 < nb; ++j) {
-            const int T = nb - 1 - j;               // tiles below (j, j)
-            const int P = T - 1;                    // panels (i, j), i >= j + 2
-            const int64_t U = (int64_t)T * (T + 1) / 2 - 1;  // updates except (j+1, j+1)
-            const int64_t n = P + U;
+        for (int sj = 0; sj <= nb; ++sj) {
+            const int jf = sj < nb ? sj : -1;       // factorisation tasks of step jf
+            const int ji = sj - 1;                  // L^-1 tasks of step ji
+            const int Tf = jf >= 0 ? nb - 1 - jf : 0;
+            // panels i >= jf + 3; updates except (jf+1, jf+1) [CTA 0], (jf+2, jf+1) and
+            // (jf+2, jf+2) [CTA 1]
+            const int P = Tf > 1 ? Tf - 2 : 0;
+            const int64_t U = Tf > 1 ? (int64_t)Tf * (Tf + 1) / 2 - 3 : 0;
+            const int Ti = ji >= 0 ? nb - 1 - ji : 0;
+            const int F = ji >= 0 ? ji : 0;                              // finalise (ji, m)
+            const int64_t V = ji >= 0 ? (int64_t)(ji + 1) * Ti : 0;      // L^-1 updates
+            const int64_t n = P + U + F + V;
             for (int64_t idx = base + ((w - base % W) % W + W) % W; idx < base + n; idx += W) {
                 const int64_t loc = idx - base;
+                const int a0 = blk_a0(), b0 = blk_b0();
                 float acc[4][4];
                 zero(acc);
+                const int j = (loc < P + U) ? jf : ji;
                 if (loc < P) {  // panel tile (i, j) = A_ij L_jj^-T
-                    const int i = j + 2 + (int)loc;
+                    const int i = j + 3 + (int)loc;
                     wait_counts(CNT(j, j), j + 1, CNT(i, j), j, nullptr, 0, p.err);
                     load_n_async(t0, p.A, rp, i, j);
                     load_t(t4, p.Li, rp, j, j);       // t4[c][x] = Li_jj[x][c]
@@ -444,16 +504,15 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     mac_n(acc, t0, t4);
                     put(p.A, rp, i, j, acc, 1.f);
                     signal_count(CNT(i, j), 1);
-                } else {  // update of tile (i, k) with step j: A_ik -= L_ij L_kj^T
+                } else if (loc < P + U) {  // update of tile (i, k): A_ik -= L_ij L_kj^T
                     int ii, kk;
-                    tri_index(loc - P + 1, ii, kk);
+                    tri_index(loc - P + 3, ii, kk);
                     const int i = j + 1 + ii, k = j + 1 + kk;
                     wait_counts(CNT(i, j), j + 1, CNT(k, j), j + 1, CNT(i, k), j, p.err);
                     load_t(t0, p.A, rp, i, j);
                     load_t(t1, p.A, rp, k, j);
                     __syncthreads();
                     mac(acc, t0, t1);
-                    const int a0 = blk_a0(), b0 = blk_b0();
                     float *bp = p.A + ((int64_t)i * TB + a0) * rp + (int64_t)k * TB + b0;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -465,6 +524,44 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                         __stcg(reinterpret_cast<float4 *>(bp + (int64_t)q * rp), v);
                     }
                     signal_count(CNT(i, k), 1);
+                } else if (loc < P + U + F) {  // finalise X_jm = -L_jj^-1 acc_jm
+                    const int m = (int)(loc - P - U);
+                    wait_counts(ICNT(j, m), j - m, CNT(j, j), j + 1, nullptr, 0, p.err);
+                    load_n_async(t0, p.Li, rp, j, j);
+                    load_n_async(t1, p.Li, rp, j, m);
+                    cp_async_wait<0>();
+                    __syncthreads();
+                    mac_n(acc, t0, t1);
+                    put(p.Li, rp, j, m, acc, -1.f);
+                    signal_count(ICNT(j, m), 1);
+                } else {  // acc_im += L_ij X_jm
+                    const int64_t v = loc - P - U - F;
+                    const int m = (int)(v / Ti), i = j + 1 + (int)(v % Ti);
+                    if (m < j)
+                        wait_counts(CNT(i, j), j + 1, ICNT(j, m), j - m + 1, ICNT(i, m), j - m,
+                                    p.err);
+                    else
+                        wait_counts(CNT(i, j), j + 1, CNT(j, j), j + 1, nullptr, 0, p.err);
+                    load_n_async(t0, p.A, rp, i, j);   // L_ij
+                    load_n_async(t1, p.Li, rp, j, m);  // X_jm (L_jj^-1 when m == j)
+                    cp_async_wait<0>();
+                    __syncthreads();
+                    mac_n(acc, t0, t1);
+                    if (m == j) {
+                        put(p.Li, rp, i, m, acc, 1.f);
+                    } else {
+                        float *bp = p.Li + ((int64_t)i * TB + a0) * rp + (int64_t)m * TB + b0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float4 x = __ldcg(reinterpret_cast<const float4 *>(bp + (int64_t)q * rp));
+                            x.x += acc[q][0];
+                            x.y += acc[q][1];
+                            x.z += acc[q][2];
+                            x.w += acc[q][3];
+                            __stcg(reinterpret_cast<float4 *>(bp + (int64_t)q * rp), x);
+                        }
+                    }
+                    signal_count(ICNT(i, m), 1);
                 }
                 __syncthreads();  // shared tiles free for the next task
             }
@@ -472,72 +569,6 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
         }
     }
     grid_barrier(p.bar, p.err);
-
-    // L^-1 by recursive doubling over pairs of s x s tile blocks [L11 0; L21 L22]:
-    // T = L21 Li11 (kept in the unused upper tile (b, a)), then Li21 = -Li22 T.
-    // Jobs are ordered by decreasing number of tile products and dealt alternately;
-    // each job streams its operand tiles through two cp.async stages.
-    for (int s = 1; s < nb; s *= 2) {
-        const int npairs = (int)ceil_div(nb, 2 * s);
-        const int64_t per = (int64_t)npairs * s;  // jobs of equal cost
-        const int64_t jobs = per * s;
-        for (int half = 0; half < 2; ++half) {
-            for (int64_t k = 0;; ++k) {
-                const int64_t q = dealt_job(k);
-                if (q >= jobs) break;
-                const int cls = (int)(q / per);
-                const int64_t rem = q % per;
-                const int pr = (int)(rem / s), o = (int)(rem % s);
-                const int top0 = 2 * pr * s, bot0 = top0 + s;
-                int a, b, c0, c1;
-                if (half == 0) {  // T(a, b) = sum_{c=b}^{bot0-1} L(a, c) Li(c, b): s - b products
-                    a = bot0 + o;
-                    b = top0 + cls;
-                    c0 = b;
-                    c1 = bot0;
-                } else {  // Li(a, b) = -sum_{c=bot0}^{a} Li(a, c) T(c, b): a - bot0 + 1 products
-                    a = bot0 + (s - 1 - cls);
-                    b = top0 + o;
-                    c0 = bot0;
-                    c1 = a + 1;
-                }
-                if (a >= nb) continue;
-                float acc[4][4];
-                zero(acc);
-                __syncthreads();
-                // stage 0: X in t0, Y in t1; stage 1: X in t2, Y in t3
-                auto issue = [&](int c, int st) {
-                    Tile &X = st ? t2 : t0;
-                    Tile &Y = st ? t3 : t1;
-                    if (half == 0) {
-                        load_n_async(X, p.A, rp, a, c);   // L(a, c)
-                        load_n_async(Y, p.Li, rp, c, b);  // Li(c, b)
-                    } else {
-                        load_n_async(X, p.Li, rp, a, c);  // Li(a, c)
-                        load_n_async(Y, p.Li, rp, b, c);  // T(c, b) at tile (b, c)
-                    }
-                };
-                issue(c0, 0);
-                for (int c = c0; c < c1; ++c) {
-                    const int st = (c - c0) & 1;
-                    if (c + 1 < c1) {
-                        issue(c + 1, st ^ 1);
-                        cp_async_wait<2>();
-                    } else {
-                        cp_async_wait<0>();
-                    }
-                    __syncthreads();
-                    mac_n(acc, st ? t2 : t0, st ? t3 : t1);
-                    __syncthreads();
-                }
-                if (half == 0)
-                    put(p.Li, rp, b, a, acc, 1.f);
-                else
-                    put(p.Li, rp, a, b, acc, -1.f);
-            }
-            grid_barrier(p.bar, p.err);
-        }
-    }
 
     // (L^-1)^T as bf16 hi + lo: LiT[x][y] = Li[y][x] (zero for y < x), all r x r entries,
     // the operand of the tensor-core product G^-1 = Li^T Li.  Thread: 8 consecutive y.
@@ -603,12 +634,12 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         grid = sms * (per_sm < 1 ? per_sm : 1);
-        if (grid < 2) return cudaErrorLaunchOutOfResources;
+        if (grid < 3) return cudaErrorLaunchOutOfResources;
     }
     cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
     const int nb = (int)(rp / TB);
-    e = cudaMemsetAsync(flags, 0, (size_t)nb * nb * sizeof(unsigned int), s);
+    e = cudaMemsetAsync(flags, 0, (size_t)2 * nb * nb * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
     Chol2Args args{G, r, nb, rp, A, Li, Gi_hi, Gi_lo, ldr, flags, err, bar};
     void *params[] = {&args};

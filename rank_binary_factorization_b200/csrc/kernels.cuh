@@ -43,7 +43,7 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 
 // ---- Cholesky + inverse (cooperative, FP32) -------------------------------------
 // G = L L^T for the SPD r x r matrix G (row stride r); writes (L^-1)^T as hi + lo bf16
-// [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: (rp/64)^2 counters.
+// [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: 2 (rp/64)^2 counters.
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *LiT_hi, __nv_bfloat16 *LiT_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s);

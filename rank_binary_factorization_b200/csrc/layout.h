@@ -81,7 +81,7 @@ struct LbLayout {
         gil = take((size_t)r * ldr * 2);
         lth = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 hi
         ltl = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 lo
-        chF = take((size_t)(rp / 64) * (rp / 64) * 4);  // Cholesky tile counters
+        chF = take((size_t)2 * (rp / 64) * (rp / 64) * 4);  // Cholesky / inverse tile counters
         tvec = take((size_t)maxrows * 4);
         bcur = take((size_t)2 * r * 4);
         gk = take((size_t)r * 4);
