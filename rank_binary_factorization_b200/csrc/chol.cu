@@ -8,6 +8,9 @@
 //   * CTA 0 runs the critical chain of the blocked right-looking factorisation: tile
 //     Cholesky of the diagonal tile, its inverse, the panel tile below it (one tile
 //     product A L_jj^-T) and the look-ahead update of the next diagonal tile;
+//   * every panel tile L_ij is also stored transposed in the unused upper tile (j, i) of
+//     A, and L_jj^-T in the unused upper tile (j, j+1) of L^-1, so all operand tiles are
+//     plain cp.async copies;
 //   * CTA 1 takes the tasks CTA 0 needs next (panel (j+2, j), updates of (j+2, j+1) and
 //     (j+2, j+2)); CTAs 2.. take the other panel tiles and the trailing updates
 //     round-robin in a topological order, so every wait ends;
@@ -50,18 +53,6 @@ __device__ __forceinline__ void load_n(Tile &d, const float *M, int64_t ld, int 
         const int row = f >> 4, c4 = (f & 15) * 4;
         const float4 v = __ldcg(reinterpret_cast<const float4 *>(base + (int64_t)row * ld + c4));
         *reinterpret_cast<float4 *>(&d[row][c4]) = v;
-    }
-}
-// d[c][r] = M_tile[r][c]
-__device__ __forceinline__ void load_t(Tile &d, const float *M, int64_t ld, int ti, int tj) {
-    const float *base = M + (int64_t)ti * TB * ld + (int64_t)tj * TB;
-    for (int f = threadIdx.x; f < TB * TB / 4; f += blockDim.x) {
-        const int row = f >> 4, c4 = (f & 15) * 4;
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(base + (int64_t)row * ld + c4));
-        d[c4][row] = v.x;
-        d[c4 + 1][row] = v.y;
-        d[c4 + 2][row] = v.z;
-        d[c4 + 3][row] = v.w;
     }
 }
 __device__ __forceinline__ void store_n(float *M, int64_t ld, int ti, int tj, const Tile &s) {
@@ -155,6 +146,18 @@ __device__ __forceinline__ void put(float *M, int64_t ld, int ti, int tj, const 
     for (int i = 0; i < 4; ++i)
         __stcg(reinterpret_cast<float4 *>(base + (int64_t)i * ld),
                make_float4(sgn * acc[i][0], sgn * acc[i][1], sgn * acc[i][2], sgn * acc[i][3]));
+}
+
+// Write the transpose of the thread's 4 x 4 block (of a tile product) into tile (ti, tj):
+// entry (a0 + i, b0 + q) of the product goes to row b0 + q, column a0 + i.
+__device__ __forceinline__ void put_t(float *M, int64_t ld, int ti, int tj,
+                                      const float (&acc)[4][4]) {
+    const int a0 = blk_a0(), b0 = blk_b0();
+    float *base = M + ((int64_t)ti * TB + b0) * ld + (int64_t)tj * TB + a0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        __stcg(reinterpret_cast<float4 *>(base + (int64_t)q * ld),
+               make_float4(acc[0][q], acc[1][q], acc[2][q], acc[3][q]));
 }
 
 // ---- 64 x 64 tile Cholesky: four 16-column blocks -----------------------------------
@@ -382,6 +385,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
         inverse_tile(t2, rdiag, t3, t4, t1);
         store_n(p.A, rp, 0, 0, t2);
         store_n(p.Li, rp, 0, 0, t3);
+        if (nb > 1) store_n(p.Li, rp, 0, 1, t4);      // L_00^-T in an unused upper tile
         signal_count(CNT(0, 0), 1);
         for (int j = 0; j + 1 < nb; ++j) {
             wait_counts(CNT(j + 1, j), j, CNT(j + 1, j + 1), j, nullptr, 0, p.err);
@@ -393,6 +397,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             zero(acc);
             mac_n(acc, t0, t4);                        // L_{j+1,j} = A_{j+1,j} L_jj^-T
             put(p.A, rp, j + 1, j, acc, 1.f);
+            put_t(p.A, rp, j, j + 1, acc);             // L_{j+1,j}^T in the upper tile
             {
                 const int a0 = blk_a0(), b0 = blk_b0();
 #pragma unroll
@@ -417,6 +422,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             inverse_tile(t2, rdiag, t3, t4, t1);
             store_n(p.A, rp, j + 1, j + 1, t2);
             store_n(p.Li, rp, j + 1, j + 1, t3);
+            if (j + 2 < nb) store_n(p.Li, rp, j + 1, j + 2, t4);  // L^-T, unused upper tile
             signal_count(CNT(j + 1, j + 1), 2);
         }
     } else if (blockIdx.x == 1) {
@@ -427,25 +433,30 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             zero(acc);
             wait_counts(CNT(j, j), j + 1, CNT(j + 2, j), j, nullptr, 0, p.err);
             load_n_async(t0, p.A, rp, j + 2, j);
-            load_t(t4, p.Li, rp, j, j);
+            load_n_async(t4, p.Li, rp, j, j + 1);    // L_jj^-T
             cp_async_wait<0>();
             __syncthreads();
             mac_n(acc, t0, t4);                        // L_{j+2,j} = A_{j+2,j} L_jj^-T
             put(p.A, rp, j + 2, j, acc, 1.f);
+            put_t(p.A, rp, j, j + 2, acc);
             {
                 const int a0 = blk_a0(), b0 = blk_b0();
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) t1[b0 + q][a0 + i] = acc[i][q];
+                    for (int q = 0; q < 4; ++q) {
+                        t1[a0 + i][b0 + q] = acc[i][q];   // L_{j+2,j}
+                        t3[b0 + q][a0 + i] = acc[i][q];   // L_{j+2,j}^T
+                    }
             }
             signal_count(CNT(j + 2, j), 1);
             wait_counts(CNT(j + 1, j), j + 1, CNT(j + 2, j + 1), j, CNT(j + 2, j + 2), j, p.err);
-            load_t(t0, p.A, rp, j + 1, j);           // t0 = L_{j+1,j}^T
+            load_n_async(t0, p.A, rp, j, j + 1);      // L_{j+1,j}^T
+            cp_async_wait<0>();
             __syncthreads();
             for (int h = 0; h < 2; ++h) {              // h = 0: tile (j+2, j+1); 1: (j+2, j+2)
                 zero(acc);
-                mac(acc, t1, h ? t1 : t0);
+                mac_n(acc, t1, h ? t3 : t0);
                 const int a0 = blk_a0(), b0 = blk_b0();
                 float *bp = p.A + ((int64_t)(j + 2) * TB + a0) * rp + (int64_t)(j + 1 + h) * TB + b0;
 #pragma unroll
@@ -498,21 +509,23 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     const int i = j + 3 + (int)loc;
                     wait_counts(CNT(j, j), j + 1, CNT(i, j), j, nullptr, 0, p.err);
                     load_n_async(t0, p.A, rp, i, j);
-                    load_t(t4, p.Li, rp, j, j);       // t4[c][x] = Li_jj[x][c]
+                    load_n_async(t4, p.Li, rp, j, j + 1);  // L_jj^-T
                     cp_async_wait<0>();
                     __syncthreads();
                     mac_n(acc, t0, t4);
                     put(p.A, rp, i, j, acc, 1.f);
+                    put_t(p.A, rp, j, i, acc);
                     signal_count(CNT(i, j), 1);
                 } else if (loc < P + U) {  // update of tile (i, k): A_ik -= L_ij L_kj^T
                     int ii, kk;
                     tri_index(loc - P + 3, ii, kk);
                     const int i = j + 1 + ii, k = j + 1 + kk;
                     wait_counts(CNT(i, j), j + 1, CNT(k, j), j + 1, CNT(i, k), j, p.err);
-                    load_t(t0, p.A, rp, i, j);
-                    load_t(t1, p.A, rp, k, j);
+                    load_n_async(t0, p.A, rp, i, j);   // L_ij
+                    load_n_async(t1, p.A, rp, j, k);   // L_kj^T (upper-tile copy)
+                    cp_async_wait<0>();
                     __syncthreads();
-                    mac(acc, t0, t1);
+                    mac_n(acc, t0, t1);
                     float *bp = p.A + ((int64_t)i * TB + a0) * rp + (int64_t)k * TB + b0;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
