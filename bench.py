@@ -154,7 +154,7 @@ def ncu_traffic(cls, m, n, r, T):
         return 540.4e6 * (T * max(m, n)) / (65536 * 4096)
     if (m, n, r) != (4096, 4096, 2032):
         return None
-    return {"chol": 20.66e6 + 9.41e6,      # chol2_kernel + EPI_SPLIT GEMM (G^-1)
+    return {"chol": 19.31e6 + 9.41e6,      # chol2_kernel + EPI_SPLIT GEMM (G^-1)
             "gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
 
 
