@@ -281,6 +281,27 @@ nq_status nq_profile_enable(int32_t enable);
  * Synchronises with the recorded events. */
 nq_status nq_profile_get(int32_t kernel_class, int64_t *launches, double *total_ms);
 
+/* ------------------------------------------------------------------------- */
+/* Diagnostics (no counterpart in the pages): run a device-side error path on  */
+/* purpose so that a test can check it ends with a status and leaves the       */
+/* context usable.                                                             */
+/* ------------------------------------------------------------------------- */
+typedef enum {
+    NQ_SELFTEST_WAIT_TIMEOUT = 0, /* the bounded counter wait of the Cholesky dataflow, on a
+                                     word nothing sets, with a poll budget of a few ms:
+                                     returns NQ_ERR_TIMEOUT */
+    NQ_SELFTEST_NOT_SPD = 1       /* the cooperative Cholesky + inverse kernel on G = -I
+                                     (64 x 64): returns NQ_ERR_NOT_SPD */
+} nq_selftest_kind;
+
+/* Bytes of device workspace nq_selftest needs (256-byte aligned). */
+size_t nq_selftest_workspace_size(void);
+
+/* Run one diagnostic; the workspace (device, caller-owned, 256-byte aligned) is cleared
+ * first.  Returns the device status the run raised (NQ_OK if none), NQ_ERR_INVALID_ARG /
+ * NQ_ERR_WORKSPACE for bad arguments, NQ_ERR_UNSUPPORTED off sm_100.  Synchronises. */
+nq_status nq_selftest(int32_t kind, void *ws, size_t ws_bytes, nq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

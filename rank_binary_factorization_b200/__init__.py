@@ -21,7 +21,7 @@ from ._lib import FIELDS, NQ_BF16, NQ_F32, NQError, check, lib, status_string
 __all__ = [
     "nq_bpw", "nq_rank_for_bpw", "nq_calib_stats", "nq_calib_precond", "nq_lbadmm",
     "nq_recon_error", "nq_pack_signs", "LBState", "NQError", "status_string", "lib",
-    "nq_launch_count", "nq_profile_enable", "nq_profile_get",
+    "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
 ]
 
 
@@ -155,6 +155,15 @@ def nq_profile_get():
         check("nq_profile_get", lib.nq_profile_get(i, ctypes.byref(n), ctypes.byref(ms)))
         out[name] = (n.value, ms.value)
     return out
+
+
+def nq_selftest(kind):
+    """Run a device-side error path on purpose ("wait_timeout" or "not_spd"); returns the
+    status code the library reports (NQ_ERR_TIMEOUT / NQ_ERR_NOT_SPD expected)."""
+    code = {"wait_timeout": _lib.NQ_SELFTEST_WAIT_TIMEOUT,
+            "not_spd": _lib.NQ_SELFTEST_NOT_SPD}[kind]
+    ws = workspace(lib.nq_selftest_workspace_size())
+    return lib.nq_selftest(code, _ptr(ws), ws.numel(), _stream())
 
 
 class LBState:

@@ -60,7 +60,10 @@ SIGNATURES = {
     "nq_launch_count": (c_i64, []),
     "nq_profile_enable": (c_i32, [c_i32]),
     "nq_profile_get": (c_i32, [c_i32, ctypes.POINTER(c_i64), ctypes.POINTER(c_f64)]),
+    "nq_selftest_workspace_size": (c_sz, []),
+    "nq_selftest": (c_i32, [c_i32, c_vp, c_sz, c_vp]),
 }
+NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
                   "objective", "finish", "recon"]
 

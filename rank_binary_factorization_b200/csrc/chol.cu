@@ -316,14 +316,7 @@ __device__ __forceinline__ void tri_index(int64_t idx, int &ii, int &kk) {
 // Bounded poll of one counter by the calling thread (null: nothing to wait for).
 __device__ __forceinline__ void poll_count(const unsigned int *c, unsigned int v, int *err) {
     if (!c || *(volatile int *)err == NQ_ERR_TIMEOUT) return;
-    uint32_t spins = 0;
-    while (ld_acquire_gpu(c) < v) {
-        if (++spins > kGridSpinLimit) {
-            raise_error(err, NQ_ERR_TIMEOUT);
-            return;
-        }
-        if (spins > 64) __nanosleep(32);
-    }
+    if (!wait_geq(c, v, kGridSpinLimit)) raise_error(err, NQ_ERR_TIMEOUT);
 }
 
 // Several counters at once: warp w < 3 polls counter w (null: none), then a CTA barrier.

@@ -50,6 +50,17 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
     return v;
 }
 
+// Bounded wait until *c >= v (acquire loads, short sleeps after the first polls).
+// Returns false when ``limit`` polls ran out; the caller raises NQ_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_geq(const unsigned int *c, unsigned int v, uint32_t limit) {
+    uint32_t spins = 0;
+    while (ld_acquire_gpu(c) < v) {
+        if (++spins > limit) return false;
+        if (spins > 64) __nanosleep(32);
+    }
+    return true;
+}
+
 // Grid-wide barrier for kernels launched cooperatively (all CTAs co-resident).
 // ``bar`` points at two words: [0] arrival count, [1] generation.  Bounded: a
 // barrier that does not complete within the spin budget raises NQ_ERR_TIMEOUT and

@@ -92,6 +92,12 @@ def test_argument_errors_are_reported_before_any_device_work():
                        null, null, fake, 1 << 30, null) == INV
     assert L.nq_lbadmm(fake, 0, 8, 8, null, null, 2, 1.0, 1e-4, 1, 0, 0, fake, fake, fake, fake,
                        null, null, fake, 1 << 30, null) == INV
+    # diagnostics: unknown kind, null / misaligned / short workspace
+    assert L.nq_selftest(7, fake, 1 << 30, null) == INV
+    assert L.nq_selftest(0, null, 1 << 30, null) == INV
+    assert L.nq_selftest(1, ctypes.c_void_p((1 << 40) + 8), 1 << 30, null) == INV
+    assert L.nq_selftest(0, fake, 16, null) == WS
+    assert L.nq_selftest_workspace_size() > 64 * 64 * 4
     # rank above min(m, n)
     assert L.nq_lbadmm(fake, 0, 8, 4, null, null, 5, 1.0, 1e-4, 1, 1, 0, fake, fake, fake, fake,
                        null, null, fake, 1 << 30, null) == INV
