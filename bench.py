@@ -131,7 +131,7 @@ class ClockSampler:
 def kernel_units(cls, m, n, r, K, T):
     """Algorithmic work of one launch scope of a kernel class: (amount, unit, bound)."""
     if cls == "calib":
-        return T * max(m, n) * 2, "B", "hbm"                 # one BF16 stream read once
+        return T * (m + n), "B", "hbm"   # per launch: mean of the two BF16 streams (T x n, T x m)
     if cls == "rhs":
         return 2.0 * m * n * r, "FLOP", "tensor"             # W^ X (either side)
     if cls == "solve":
@@ -151,7 +151,7 @@ def kernel_units(cls, m, n, r, K, T):
 # the stream); the others hold for the captured layer and rank only.
 def ncu_traffic(cls, m, n, r, T):
     if cls == "calib":
-        return 540.4e6 * (T * max(m, n)) / (65536 * 4096)
+        return 540.4e6 * (T * (m + n) / 2) / (65536 * 4096)
     if (m, n, r) != (4096, 4096, 2032):
         return None
     return {"chol": 19.31e6 + 9.41e6,      # chol2_kernel + EPI_SPLIT GEMM (G^-1)
@@ -206,14 +206,24 @@ def oracle_sample(W_h, acts_h, grads_h, r, iters, T):
         est_step_s=round(step_s, 2))
 
 
-def make_host_inputs(seed, m, n, T):
-    """Seeded synthetic inputs generated on the device, kept in pinned host memory too."""
+def make_host_inputs(seed, m, n, T, w_kind="outlier_cols"):
+    """Seeded synthetic inputs generated on the device, kept in pinned host memory too.
+
+    w_kind "outlier_cols": W ~ N(0, 0.02^2) with 1 % of input columns x10;
+    "student_t": W ~ N(0, 0.02^2) with input column j scaled by max(1, |t_j|),
+    t_j ~ Student-t(3) (a normal over the root of a chi-square(3) / 3)."""
     import torch
     g = torch.Generator(device="cuda")
     g.manual_seed(1000 + seed)
     W = torch.randn(m, n, device="cuda", generator=g) * 0.02
-    cols = torch.randperm(n, device="cuda", generator=g)[: max(1, n // 100)]
-    W[:, cols] *= 10.0
+    if w_kind == "student_t":
+        z = torch.randn(n, device="cuda", generator=g, dtype=torch.float64)
+        chi2 = (torch.randn(3, n, device="cuda", generator=g, dtype=torch.float64) ** 2).sum(0)
+        t = z / torch.sqrt(chi2 / 3.0)
+        W *= torch.clamp(t.abs(), min=1.0).float()[None, :]
+    else:
+        cols = torch.randperm(n, device="cuda", generator=g)[: max(1, n // 100)]
+        W[:, cols] *= 10.0
     W = W.to(torch.bfloat16)
 
     def stream(C):
@@ -282,8 +292,9 @@ def run_ours(args):
 
     m, n, T, iters = WORKLOAD["m"], WORKLOAD["n"], WORKLOAD["T"], args.iters
     rho, lam, K = WORKLOAD["rho"], WORKLOAD["lam"], WORKLOAD["K"]
-    r = nq.nq_rank_for_bpw(m, n, WORKLOAD["bpw"])
-    (W, acts, grads), (W_h, acts_h, grads_h) = make_host_inputs(rank, m, n, T)
+    r = WORKLOAD.get("r") or nq.nq_rank_for_bpw(m, n, WORKLOAD["bpw"])
+    (W, acts, grads), (W_h, acts_h, grads_h) = make_host_inputs(
+        rank, m, n, T, WORKLOAD.get("w_kind", "outlier_cols"))
     calib_ws = nq.workspace(nq.lib.nq_calib_workspace_size(T, max(m, n)))
     lb_ws = nq.workspace(nq.lib.nq_lbadmm_workspace_size(m, n, r))
 
@@ -354,6 +365,12 @@ def run_ours(args):
     dominant = max(entries.values(), key=lambda e: e["launches"] * e["ms_per_launch"])
     value = world * iters * args.steps / t
     tflops = 4.0 * m * n * r * iters * world * args.steps / t / 1e12
+    ms_iter = (step_ms - (prof["calib"][1] + prof["calib_finalize"][1]) / args.steps) / iters
+    # executed work of an iteration by the convention 4mnr (both contractions)
+    # + 3 (m+n) r^2 (Grams and solves) + 2 r^3 / 3 (factorisations)
+    tflops_exec = (4.0 * m * n * r + 3.0 * (m + n) * r * r + 2.0 * r ** 3 / 3.0) / (ms_iter / 1e3) / 1e12
+    t_roof = max(4.0 * m * n * r / (peaks["bf16_tflops_sustained"] * 1e12),
+                 (4.0 * m * n + 16.0 * (m + n) * r) / (peaks["hbm_gbs"] * 1e9))
     calib = entries.get("calib")
     line = dict(
         metric=METRIC, value=round(value, 3), unit=UNIT, n_gpus=world, steps=args.steps,
@@ -361,10 +378,14 @@ def run_ours(args):
         scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
         config=dict(workload=WORKLOAD["name"], m=m, n=n, r=r, iters=iters, T=T, rho=rho,
                     lam=lam, K=K, parallelism=f"replicas x{world}",
-                    l2="inputs larger than L2 (2 x 2.1 GB calibration streams read every step)"),
+                    l2="inputs larger than L2 (calibration streams of "
+                       f"{T * (m + n) * 2 / 1e9:.1f} GB read every step)"),
         tflops_4mnr=round(tflops, 2),
-        lbadmm_ms_per_iter=round((step_ms - (prof["calib"][1] + prof["calib_finalize"][1])
-                                  / args.steps) / iters, 4),
+        tflops_executed=round(tflops_exec, 2),
+        lbadmm_ms_per_iter=round(ms_iter, 4),
+        lbadmm_roofline=dict(t_roof_us=round(t_roof * 1e6, 2),
+                             basis="max(4mnr / sustained bf16, (4mn + 16(m+n)r) / HBM)",
+                             frac=round(t_roof / (ms_iter / 1e3), 4)),
         calib_gbs=calib["achieved"] if calib else None,
         roofline=dominant,
         kernels=entries,
@@ -395,10 +416,16 @@ def main():
     ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["q_proj", "profile"], default="q_proj",
+    ap.add_argument("--workload", choices=["q_proj", "profile", "gate_proj"], default="q_proj",
                     help="profile: the same layer with 65536-token streams and 2 iterations, "
-                         "the small case used for ncu section captures")
+                         "the small case used for ncu section captures; gate_proj: the "
+                         "11008x4096 Llama-2-7B gate/up shape at r = 1000 with Student-t(3) "
+                         "column factors (the LB-ADMM throughput target)")
     args = ap.parse_args()
+    if args.workload == "gate_proj":
+        WORKLOAD.update(m=11008, n=4096, r=1000, w_kind="student_t",
+                        name="llama2-7b gate_proj 11008x4096 bf16, r=1000, 100 LB-ADMM "
+                             "iterations, calibration 262144x4096 + 262144x11008 bf16 streams")
     if args.workload == "profile":
         WORKLOAD.update(T=65536, name="profiling case: q_proj 4096x4096 bf16, r=2032, "
                                       "2 x 65536x4096 bf16 streams")
