@@ -250,9 +250,12 @@ def run_reference(args):
     import torch
     m, n, T, iters = WORKLOAD["m"], WORKLOAD["n"], WORKLOAD["T"], args.iters
     from oracle.bpw import rank_for_bpw
-    r = rank_for_bpw(m, n, WORKLOAD["bpw"])
-    from synth import gaussian_weight, stream_tensor
-    W_h = gaussian_weight(0, "W", m, n, 0.02, 0.01, 10.0)
+    r = WORKLOAD.get("r") or rank_for_bpw(m, n, WORKLOAD["bpw"])
+    from synth import gaussian_weight, stream_tensor, student_t_weight
+    if WORKLOAD.get("w_kind") == "student_t":
+        W_h = student_t_weight(0, "W", m, n, 0.02, 3)
+    else:
+        W_h = gaussian_weight(0, "W", m, n, 0.02, 0.01, 10.0)
     Ts = 16384
     acts_h = stream_tensor(0, "acts", Ts, n)
     grads_h = stream_tensor(0, "grads", Ts, m)
