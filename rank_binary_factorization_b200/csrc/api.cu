@@ -203,11 +203,12 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
                            &lb.sc->err, lb.sc->bar, s));
-        // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo
+        // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo; G^-1 is
+        // symmetric, so only its lower-triangular tiles are computed and mirrored
         tc::Maps maps;
         memset(&maps, 0, sizeof(maps));
         const void *th = lb.p<void>(L.lth), *tl = lb.p<void>(L.ltl);
-        const int BNg = L.r > 1024 ? 128 : BN;
+        const int BNg = tc::BM;  // square tiles: only the lower triangle is computed
         if (!tc::make_map_bf16(&maps.a[0], th, L.r, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.a[1], th, L.r, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.a[2], tl, L.r, L.r, L.ldr, tc::BM) ||
@@ -222,6 +223,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
         ep.nseg = 3;
         ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
         ep.tri_k = 1;
+        ep.sym = 1;
         ep.err = &lb.sc->err;
         ep.Rhi = lb.p<__nv_bfloat16>(L.gih);
         ep.Rlo = lb.p<__nv_bfloat16>(L.gil);

@@ -145,6 +145,20 @@ __device__ __forceinline__ void ld16_bf16(float (&d)[16], const __nv_bfloat16 *s
     for (int j = 0; j < 16; ++j) d[j] = __bfloat162float(h[j]);
 }
 
+// Mirrored store of a symmetric result (EPI_SPLIT): entry (row, col0 + j) also goes to
+// (col0 + j, row); consecutive lanes hold consecutive rows, so each store is coalesced.
+__device__ __forceinline__ void split_mirror(const EpiParams &p, int row, int col0,
+                                             const float (&v)[16]) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        if (col0 + j >= p.N) break;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+        const int64_t o = (int64_t)(col0 + j) * p.ldr + row;
+        p.Rhi[o] = h;
+        p.Rlo[o] = __float2bfloat16_rn(v[j] - __bfloat162float(h));
+    }
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int col0,
                                                const float (&v)[16], float &acc_sum) {
@@ -288,6 +302,23 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
     }
 }
 
+// Output tile -> (m0, n0).  Plain: m fastest.  Symmetric (BN == BM): the lower-triangular
+// tiles (tm >= tn) row by row, so tiles come in order of decreasing K range under tri_k.
+template <int BN>
+__device__ __forceinline__ void tile_origin(const EpiParams &p, int tile, int num_m, int &m0,
+                                            int &n0) {
+    if (p.sym) {
+        int a = (int)((sqrtf(8.f * (float)tile + 1.f) - 1.f) * 0.5f);
+        while ((a + 1) * (a + 2) / 2 <= tile) ++a;
+        while (a * (a + 1) / 2 > tile) --a;
+        m0 = a * BM;
+        n0 = (tile - a * (a + 1) / 2) * BN;
+    } else {
+        m0 = (tile % num_m) * BM;
+        n0 = (tile / num_m) * BN;
+    }
+}
+
 // ---------------------------------------------------------------------------------
 // The kernel: persistent, one CTA per SM, tiles assigned round-robin (m fastest, so
 // consecutive CTAs share the B tile).  Two TMEM accumulator stages let the epilogue
@@ -313,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int num_m = (int)ceil_div(p.M, BM);
-    const int num_tiles = num_m * (int)ceil_div(p.N, BN);
+    const int num_tiles = p.sym ? num_m * (num_m + 1) / 2 : num_m * (int)ceil_div(p.N, BN);
     const int total_kb = p.kblocks[0] + (p.nseg > 1 ? p.kblocks[1] : 0) +
                          (p.nseg > 2 ? p.kblocks[2] : 0);
 
@@ -346,7 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+                int m0, n0;
+                tile_origin<BN>(p, tile, num_m, m0, n0);
                 for (int kb = 0; kb < total_kb; ++kb) {
                     int seg = 0, k = kb;
                     while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
@@ -374,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int lt = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
                 const int as = lt & 1;
-                const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+                int m0, n0;
+                tile_origin<BN>(p, tile, num_m, m0, n0);
                 if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, p.err)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(as * BN);
@@ -412,7 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool dead = false;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
             const int as = lt & 1;
-            const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+            int m0, n0;
+            tile_origin<BN>(p, tile, num_m, m0, n0);
             const int row = m0 + 32 * q + lane;
             float acc_sum = 0.f;
             if (!dead) {
@@ -430,7 +464,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BN; c += 16) {
                     float v[16];
                     tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
-                    if (row < p.M && n0 + c < p.N) epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
+                    if (row < p.M && n0 + c < p.N) {
+                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
+                        if constexpr (EPI == EPI_SPLIT)
+                            if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();

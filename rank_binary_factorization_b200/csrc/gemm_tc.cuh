@@ -36,6 +36,8 @@ struct EpiParams {
     int nseg;
     int kblocks[3];
     int tri_k;          // operands zero for k < row index: start each tile's K at max(m0, n0)
+    int sym;            // symmetric result (EPI_SPLIT, BN == BM): lower-triangular tiles only,
+                        // each off-diagonal tile also written mirrored
     int *err;
     // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
     float *out;
