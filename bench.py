@@ -154,9 +154,8 @@ def ncu_traffic(cls, m, n, r, T):
         return 540.4e6 * (T * (m + n) / 2) / (65536 * 4096)
     if (m, n, r) != (4096, 4096, 2032):
         return None
-    # "chol" (chol2_kernel + the G^-1 GEMM) is left out: the G^-1 GEMM changed after the
-    # last capture (chol2_kernel alone: 19.31 MB)
-    return {"gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
+    return {"chol": 19.31e6 + 9.42e6,      # chol2_kernel + the symmetric G^-1 GEMM
+            "gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
 
 
 def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
