@@ -46,7 +46,7 @@ struct Chol2Args {
     unsigned int *bar;
 };
 
-// ---- tile movement (L2-coherent loads: tiles change between grid barriers) ----------
+// ---- tile movement (L2-coherent loads: other CTAs write the tiles between tasks) -----
 __device__ __forceinline__ void load_n(Tile &d, const float *M, int64_t ld, int ti, int tj) {
     const float *base = M + (int64_t)ti * TB * ld + (int64_t)tj * TB;
     for (int f = threadIdx.x; f < TB * TB / 4; f += blockDim.x) {
@@ -365,9 +365,10 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
     float *rdiag = smem_f + 5 * TB * LDS;  // 1 / L_cc of the tile just factored
     // Dataflow factorisation.  CTA 0 runs the critical chain: Cholesky of the diagonal
     // tile and its inverse (kept in shared memory), the panel tile below it as one tile
-    // product, the look-ahead update of the next diagonal tile.  CTAs 1.. take the other
-    // panel tiles (A_ij L_jj^-T, with L_jj^-1 from the Li diagonal tile) and the trailing
-    // updates round-robin in a topological order (step by step), so every wait ends.
+    // product, the look-ahead update of the next diagonal tile.  CTA 1 takes the tasks CTA 0
+    // needs next; CTAs 2.. take the other panel tiles (A_ij L_jj^-T, with L_jj^-T from the
+    // upper tile (j, j+1) of Li), the trailing updates and the L^-1 tasks round-robin in a
+    // topological order (step by step), so every wait ends.
     auto CNT = [&](int i, int k) { return p.cnt + (int64_t)i * nb + k; };
     auto ICNT = [&](int i, int k) { return p.cnt + (int64_t)(nb + i) * nb + k; };  // L^-1 tiles
     if (blockIdx.x == 0) {
@@ -620,8 +621,6 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
 }
 
 }  // namespace
-
-int64_t chol_padded(int32_t r) { return (int64_t)(r + TB - 1) / TB * TB; }
 
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
