@@ -337,10 +337,7 @@ __device__ __forceinline__ void wait_counts(const unsigned int *c0, unsigned int
 // has timed out, skipped.
 __device__ __forceinline__ void signal_count(unsigned int *c, unsigned int inc) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(c, inc);
-    }
+    if (threadIdx.x == 0) release_add(c, inc);
 }
 
 __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
@@ -465,9 +462,8 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
             }
             __syncthreads();
             if (threadIdx.x == 0) {
-                __threadfence();
-                atomicAdd(CNT(j + 2, j + 1), 1u);
-                atomicAdd(CNT(j + 2, j + 2), 1u);
+                release_add(CNT(j + 2, j + 1), 1u);
+                release_add(CNT(j + 2, j + 2), 1u);
             }
             __syncthreads();
         }

@@ -50,6 +50,13 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
     return v;
 }
 
+// Publish: *c += inc with release semantics at GPU scope.  Called by one thread after a
+// CTA barrier, it makes the CTA's earlier writes visible to any thread that then reads
+// the counter with an acquire load (wait_geq).
+__device__ __forceinline__ void release_add(unsigned int *c, unsigned int inc) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(c), "r"(inc) : "memory");
+}
+
 // Bounded wait until *c >= v (acquire loads, short sleeps after the first polls).
 // Returns false when ``limit`` polls ran out; the caller raises NQ_ERR_TIMEOUT.
 __device__ __forceinline__ bool wait_geq(const unsigned int *c, unsigned int v, uint32_t limit) {
