@@ -154,7 +154,7 @@ def ncu_traffic(cls, m, n, r, T):
         return 540.4e6 * (T * (m + n) / 2) / (65536 * 4096)
     if (m, n, r) != (4096, 4096, 2032):
         return None
-    return {"chol": 19.31e6 + 9.42e6,      # chol2_kernel + the symmetric G^-1 GEMM
+    return {"chol": 17.21e6 + 9.42e6,      # chol2_kernel + the symmetric G^-1 GEMM
             "gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
 
 
