@@ -2,10 +2,12 @@
 """Benchmark of the NanoQuant hot path on B200.
 
 One step = the whole hot path over one layer's synthetic inputs, resident in HBM:
-  calibration preconditioners from two 262144 x 4096 BF16 token streams
-  (nq_calib_precond), then LB-ADMM on the 4096 x 4096 BF16 q_proj-shaped layer at
-  1 BPW (r = 2032): target preparation, 100 iterations, balancing, scales, packing and
-  the reconstruction error (nq_lbadmm).
+  calibration preconditioners from the layer's two 262144-token BF16 streams
+  (nq_calib_precond), then LB-ADMM on the layer: target preparation, 100 iterations,
+  balancing, scales, packing and the reconstruction error (nq_lbadmm).
+Default layer: the Llama-2-7B gate/up shape 11008 x 4096 (BF16, Student-t(3) column
+factors) at r = 1000, with 262144 x 4096 activation and 262144 x 11008 gradient
+streams.  --workload q_proj: the 4096 x 4096 q_proj at 1 BPW (r = 2032).
 Metric: LB-ADMM layer-iterations per second of the whole step (iterations x layers /
 step time), with 4mnr TFLOP/s, calibration GB/s and the roofline fraction of the
 dominant kernel alongside.
@@ -29,9 +31,13 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LB-ADMM layer-iters/s & TFLOP/s vs roofline; calib-stats GB/s vs HBM peak"
 UNIT = "layer-iters/s"
-WORKLOAD = dict(name="llama2-7b q_proj 4096x4096 bf16, r=2032 (1.0 BPW), 100 LB-ADMM iterations, "
-                     "calibration 2 x 262144x4096 bf16 streams",
-                m=4096, n=4096, bpw=1.0, iters=100, T=128 * 2048, rho=1.0, lam=1e-4, K=4)
+WORKLOAD = dict(name="llama2-7b gate_proj 11008x4096 bf16, r=1000, 100 LB-ADMM iterations, "
+                     "calibration 262144x4096 + 262144x11008 bf16 streams",
+                m=11008, n=4096, r=1000, w_kind="student_t", iters=100, T=128 * 2048, rho=1.0,
+                lam=1e-4, K=4)
+Q_PROJ = dict(name="llama2-7b q_proj 4096x4096 bf16, r=2032 (1.0 BPW), 100 LB-ADMM iterations, "
+                   "calibration 2 x 262144x4096 bf16 streams",
+              m=4096, n=4096, r=None, bpw=1.0, w_kind="outlier_cols")
 FP32_LANES_PER_SM = 128
 NUM_SMS = 148
 
@@ -129,7 +135,12 @@ class ClockSampler:
 
 
 def kernel_units(cls, m, n, r, K, T):
-    """Algorithmic work of one launch scope of a kernel class: (amount, unit, bound)."""
+    """Algorithmic work of one launch scope of a kernel class: (amount, unit, bound).
+
+    Per launch scope, averaged over the two sides where they differ.  "chol" counts the
+    method's own work, one Cholesky factorisation (r^3 / 3); the triangular inverse the
+    library also forms there is executed work beyond it.  "ginv" is the product
+    L^-T L^-1 of two triangular factors (r^3 / 3)."""
     if cls == "calib":
         return T * (m + n), "B", "hbm"   # per launch: mean of the two BF16 streams (T x n, T x m)
     if cls == "rhs":
@@ -137,25 +148,24 @@ def kernel_units(cls, m, n, r, K, T):
     if cls == "solve":
         return 2.0 * (m + n) / 2 * r * r, "FLOP", "tensor"   # R G^-1 (mean of both sides)
     if cls == "gram":
-        return 2.0 * (m + n) / 2 * r * r, "FLOP", "tensor"   # X^T X (full square)
+        return 1.0 * (m + n) / 2 * r * r, "FLOP", "tensor"   # X^T X (symmetric half)
     if cls == "chol":
-        return float(r) ** 3, "FLOP", "alu"                  # Cholesky + inverse + L^-T L^-1
+        return float(r) ** 3 / 3.0, "FLOP", "alu"            # Cholesky of the r x r system
+    if cls == "ginv":
+        return float(r) ** 3 / 3.0, "FLOP", "tensor"         # L^-T L^-1
     if cls == "svid":
         return 4.0 * K * (m + n) / 2 * r, "B", "hbm"         # K reads of S (FP32)
     return None
 
 
-# DRAM bytes (read + write) per launch scope from the committed ncu captures
-# (profiles/*.md: `ncu --set full` of `bench.py --workload profile`, q_proj 4096 x 4096,
-# r = 2032, 65536-token streams).  The calibration figure scales with T x C (one read of
-# the stream); the others hold for the captured layer and rank only.
+# DRAM bytes (read + write) per launch scope from an ncu capture of the current kernels
+# (calibration: `ncu --set full` of `bench.py --workload profile`, 65536 x 4096 BF16
+# streams; one read of the stream, so it scales with T x C).  Classes whose kernels
+# changed since their last capture report null.
 def ncu_traffic(cls, m, n, r, T):
     if cls == "calib":
         return 540.4e6 * (T * (m + n) / 2) / (65536 * 4096)
-    if (m, n, r) != (4096, 4096, 2032):
-        return None
-    return {"chol": 17.21e6 + 9.42e6,      # chol2_kernel + the symmetric G^-1 GEMM
-            "gram": 16.69e6, "rhs": 96.36e6, "solve": 134.63e6}.get(cls)
+    return None
 
 
 def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
@@ -166,14 +176,17 @@ def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
     per_launch_s = ms / 1e3 / launches
     if unit == "B":
         achieved, peak, punit = amount / per_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        peak_kind = f"measured HBM copy ({peaks['source']})"
     elif bound == "tensor":
         achieved, peak, punit = amount / per_launch_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        peak_kind = f"measured sustained cuBLAS bf16 ({peaks['source']})"
     else:
         achieved, peak, punit = amount / per_launch_s / 1e12, peaks["fp32_tflops"], "TFLOP/s"
+        peak_kind = "derived FP32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz"
     return dict(kernel=cls, bound=bound, achieved=round(achieved, 2), peak=round(peak, 1),
                 unit=punit, frac=round(achieved / peak, 4), traffic=ncu_traffic(cls, m, n, r, T),
                 launches=launches, ms_per_launch=round(ms / launches, 4),
-                share_of_step=None)
+                share_of_step=None, peak_kind=peak_kind)
 
 
 # ---------------------------------------------------------------------------------------
@@ -198,7 +211,7 @@ def oracle_sample(W_h, acts_h, grads_h, r, iters, T):
     step_s = t_calib + iters * t_one
     cores = max([ti.get("num_threads", 1) for ti in threadpool_info()] + [1])
     return iters / step_s, dict(
-        kind="oracle", cores=cores,
+        kind="oracle", cores=cores, extrapolated=True,
         sample=f"calibration on {Ts} of {T} tokens per stream (time scaled by {T // Ts}); "
                f"one full LB-ADMM iteration (with preparation, balancing, packing and the "
                f"reconstruction error) on the whole {Wd.shape[0]}x{Wd.shape[1]} layer, time "
@@ -419,19 +432,19 @@ def main():
     ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["q_proj", "profile", "gate_proj"], default="q_proj",
-                    help="profile: the same layer with 65536-token streams and 2 iterations, "
-                         "the small case used for ncu section captures; gate_proj: the "
-                         "11008x4096 Llama-2-7B gate/up shape at r = 1000 with Student-t(3) "
-                         "column factors (the LB-ADMM throughput target)")
+    ap.add_argument("--workload", choices=["gate_proj", "q_proj", "profile", "q_proj_profile"],
+                    default="gate_proj",
+                    help="gate_proj (default): the 11008x4096 Llama-2-7B gate/up shape at "
+                         "r = 1000 with Student-t(3) column factors; q_proj: 4096x4096 at "
+                         "1 BPW (r = 2032); profile / q_proj_profile: the same layers with "
+                         "65536-token streams and 2 iterations, the small cases of the ncu "
+                         "section captures")
     args = ap.parse_args()
-    if args.workload == "gate_proj":
-        WORKLOAD.update(m=11008, n=4096, r=1000, w_kind="student_t",
-                        name="llama2-7b gate_proj 11008x4096 bf16, r=1000, 100 LB-ADMM "
-                             "iterations, calibration 262144x4096 + 262144x11008 bf16 streams")
-    if args.workload == "profile":
-        WORKLOAD.update(T=65536, name="profiling case: q_proj 4096x4096 bf16, r=2032, "
-                                      "2 x 65536x4096 bf16 streams")
+    if args.workload in ("q_proj", "q_proj_profile"):
+        WORKLOAD.update(Q_PROJ)
+    if args.workload in ("profile", "q_proj_profile"):
+        WORKLOAD.update(T=65536, name="profiling case: " + WORKLOAD["name"].split(",")[0] +
+                                      f", r={WORKLOAD['r'] or 'at 1 BPW'}, 65536-token streams")
         if args.iters == WORKLOAD["iters"]:
             args.iters = 2
     if args.impl == "reference":

@@ -24,7 +24,9 @@
  *     current device; "host" pointers are ordinary host memory.
  *   - The caller owns every buffer.  The library allocates no device memory:
  *     all scratch lives in the caller's workspace ``ws`` (size from the matching
- *     *_workspace_size function; 256-byte alignment required).
+ *     *_workspace_size function; 256-byte alignment required).  One exception:
+ *     nq_calib_stats_noalloc takes no workspace and keeps its scratch in a fixed
+ *     4 MiB array inside the library image (see its declaration).
  *   - All device work is enqueued on ``stream``.  Entry points that fill host
  *     outputs synchronise ``stream`` before returning; the others return as soon
  *     as the work is enqueued.
@@ -59,6 +61,15 @@ typedef enum {
 } nq_status;
 
 typedef enum { NQ_F32 = 0, NQ_BF16 = 1 } nq_dtype;
+
+/* Arithmetic of the LB-ADMM tensor-core contractions (W^ X, the Grams X^T X):
+ *   NQ_PREC_BF16  W^ and the latent factor are rounded to BF16 (RNE) as MMA operands;
+ *   NQ_PREC_FP32  both are split into BF16 hi + lo parts and each contraction runs as
+ *                 three MMA passes (hi.hi + lo.hi + hi.lo): FP32-level accuracy at three
+ *                 times the tensor work.
+ * Accumulation is FP32 in both; the solve with G^-1 is always split (FP32-level).
+ * nq_lbadmm uses NQ_PREC_BF16 for BF16 weights and NQ_PREC_FP32 for FP32 weights. */
+typedef enum { NQ_PREC_BF16 = 0, NQ_PREC_FP32 = 1 } nq_precision;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *nq_status_string(nq_status s);
@@ -159,7 +170,8 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  *   g_k = sqrt(||V_:k|| / ||U_:k||);  U_:k *= g_k;  V_:k /= g_k
  *   s1_i = gamma mean_k |U_ik|,  s2_j = mean_k |V_jk|
  *   sign bit = (latent < 0), LSB-first along k, row-major uint32[rows][(r+31)/32]
- * Tensor-core operands (W^ and the latent factor of the contraction) are BF16;
+ * Tensor-core operands (W^ and the latent factor of the contraction) are BF16 for BF16
+ * weights and split BF16 (FP32-accurate, see nq_precision) for FP32 weights;
  * accumulation and every other quantity is FP32 (reductions FP64 where noted).
  *
  * W: device, m x n, dtype dt.  d_in (n), d_out (m): device float, or NULL for 1.
@@ -203,20 +215,24 @@ nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,
 /* ------------------------------------------------------------------------- */
 
 /* Form W^ (and its transpose) from W, d_in, d_out; set V = V_0(seed) and zero the
- * dual state.  gamma_out: host double or NULL (synchronises when non-NULL). */
+ * dual state.  ``prec`` selects the operand precision of the following iterations (the
+ * split low parts are formed for NQ_PREC_FP32 and zeroed otherwise).
+ * gamma_out: host double or NULL (synchronises when non-NULL). */
 nq_status nq_lbadmm_prepare(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
-                            const float *d_out, int32_t r, uint64_t seed, double *gamma_out,
-                            void *ws, size_t ws_bytes, nq_stream_t stream);
+                            const float *d_out, int32_t r, uint64_t seed, nq_precision prec,
+                            double *gamma_out, void *ws, size_t ws_bytes, nq_stream_t stream);
 
-/* Run ``iters`` full iterations (U side then V side).  objective: host float[iters]
- * or NULL (synchronises when non-NULL). */
+/* Run ``iters`` full iterations (U side then V side) at precision ``prec`` (use the one
+ * given to nq_lbadmm_prepare).  objective: host float[iters] or NULL (synchronises when
+ * non-NULL). */
 nq_status nq_lbadmm_iterate(int64_t m, int64_t n, int32_t r, float rho, float lambda,
-                            int32_t iters, int32_t K, float *objective, void *ws, size_t ws_bytes,
-                            nq_stream_t stream);
+                            int32_t iters, int32_t K, nq_precision prec, float *objective,
+                            void *ws, size_t ws_bytes, nq_stream_t stream);
 
 /* One half iteration: side 0 updates U from V, side 1 updates V from U. */
 nq_status nq_lbadmm_half_step(int64_t m, int64_t n, int32_t r, float rho, float lambda, int32_t K,
-                              int32_t side, void *ws, size_t ws_bytes, nq_stream_t stream);
+                              int32_t side, nq_precision prec, void *ws, size_t ws_bytes,
+                              nq_stream_t stream);
 
 /* Balance, extract s1/s2, pack, and (when final_rel_err != NULL) the reconstruction
  * error against W~ formed from W, d_in, d_out (synchronises then). */
@@ -228,10 +244,12 @@ nq_status nq_lbadmm_finish(const void *W, nq_dtype dt, int64_t m, int64_t n, con
 /* State fields.  X = latent after its last step (rows x r, float); S = X + L, the
  * SVID input, from which the dual state is Z = sign(S) a b^T, L = S - Z (rows x r,
  * float); A = a (rows, float); B = b (r, float); WHAT = W^ (m x n, bf16, row
- * stride ld elements); GAMMA = gamma (1 double). */
+ * stride ld elements); WHAT_LO = its low part in NQ_PREC_FP32 (zero otherwise);
+ * GAMMA = gamma (1 double). */
 typedef enum {
     NQ_FIELD_U = 0, NQ_FIELD_V = 1, NQ_FIELD_SU = 2, NQ_FIELD_SV = 3, NQ_FIELD_AU = 4,
-    NQ_FIELD_AV = 5, NQ_FIELD_BU = 6, NQ_FIELD_BV = 7, NQ_FIELD_WHAT = 8, NQ_FIELD_GAMMA = 9
+    NQ_FIELD_AV = 5, NQ_FIELD_BU = 6, NQ_FIELD_BV = 7, NQ_FIELD_WHAT = 8, NQ_FIELD_GAMMA = 9,
+    NQ_FIELD_WHAT_LO = 10
 } nq_field;
 
 /* Device address, element count, element size and row stride (elements) of a
@@ -240,10 +258,11 @@ nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, voi
                                 size_t ws_bytes, void **dev_ptr, int64_t *count,
                                 int32_t *elem_bytes, int64_t *ld);
 
-/* Re-derive the BF16 operand copies (transposes of U and V and W^^T) after a
- * caller has written NQ_FIELD_U / NQ_FIELD_V / NQ_FIELD_WHAT directly. */
-nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
-                                  nq_stream_t stream);
+/* Re-derive the BF16 operand copies (transposes of U and V, with their low parts at
+ * NQ_PREC_FP32, and W^^T) after a caller has written NQ_FIELD_U / NQ_FIELD_V /
+ * NQ_FIELD_WHAT (/ NQ_FIELD_WHAT_LO) directly. */
+nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, nq_precision prec, void *ws,
+                                  size_t ws_bytes, nq_stream_t stream);
 
 /* Device error word of a workspace: 0 if clean, else the first nq_status raised
  * on the device since the last reset; resets it.  Synchronises the stream. */
@@ -253,7 +272,8 @@ nq_status nq_lbadmm_check(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_b
 /* ------------------------------------------------------------------------- */
 /* Measurement helpers (not steps of the method).  When enabled, the library   */
 /* records a pair of CUDA events on the launching stream around every kernel   */
-/* launch and attributes the elapsed device time to the kernel's class.        */
+/* launch and attributes the elapsed device time to the kernel's class.  Each  */
+/* class's launches are also wrapped in an NVTX range named "nq.<class>".      */
 /* Off by default; recording costs one event pair per launch.  Not for use     */
 /* while the stream is being captured into a CUDA graph.                       */
 /* ------------------------------------------------------------------------- */
@@ -262,14 +282,15 @@ typedef enum {
     NQ_K_CALIB_FIN = 1, /* moments finalize + Ledoit-Wolf                            */
     NQ_K_PREP = 2,      /* target preparation, V_0                                   */
     NQ_K_GRAM = 3,      /* tcgen05 Gram X^T X + (lambda + rho) I                     */
-    NQ_K_CHOL = 4,      /* Cholesky + inverse                                        */
+    NQ_K_CHOL = 4,      /* Cholesky factorisation + triangular inverse (FP32 SIMT)   */
     NQ_K_RHS = 5,       /* tcgen05 W^ X + rho (Z - L)                                */
     NQ_K_SOLVE = 6,     /* tcgen05 R G^-1 with the dual-state epilogue               */
     NQ_K_SVID = 7,      /* SVID power passes                                         */
     NQ_K_OBJ = 8,       /* per-iteration objective                                   */
     NQ_K_FINISH = 9,    /* balancing, scales, packing                                */
     NQ_K_RECON = 10,    /* tcgen05 +-1 reconstruction error                          */
-    NQ_K_COUNT = 11
+    NQ_K_GINV = 11,     /* tcgen05 G^-1 = L^-T L^-1 (symmetric, split BF16)          */
+    NQ_K_COUNT = 12
 } nq_kernel_class;
 
 /* Number of kernel launches the library has issued in this process. */

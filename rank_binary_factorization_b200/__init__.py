@@ -16,7 +16,8 @@ if os.environ.get("NQ_NO_AUTOBUILD") != "1":
     _build.build()          # no-op unless libnq.so is missing or older than its sources
 
 from . import _lib
-from ._lib import FIELDS, NQ_BF16, NQ_F32, NQError, check, lib, status_string
+from ._lib import (FIELDS, NQ_BF16, NQ_F32, NQ_PREC_BF16, NQ_PREC_FP32, NQError, check, lib,
+                   status_string)
 
 __all__ = [
     "nq_bpw", "nq_rank_for_bpw", "nq_calib_stats", "nq_calib_precond", "nq_lbadmm",
@@ -167,12 +168,17 @@ def nq_selftest(kind):
 
 
 class LBState:
-    """Step-level access to an LB-ADMM workspace (prepare / half steps / state fields)."""
+    """Step-level access to an LB-ADMM workspace (prepare / half steps / state fields).
+
+    ``prec`` is the operand precision of the contractions ("bf16" or "fp32", see
+    nq_precision); nq_lbadmm picks "fp32" for FP32 weights and "bf16" for BF16 weights.
+    """
 
     _DT = {2: torch.bfloat16, 4: torch.float32, 8: torch.float64}
 
-    def __init__(self, m, n, r, device="cuda"):
+    def __init__(self, m, n, r, device="cuda", prec="bf16"):
         self.m, self.n, self.r = m, n, r
+        self.prec = {"bf16": NQ_PREC_BF16, "fp32": NQ_PREC_FP32}[prec]
         self.nbytes = lib.nq_lbadmm_workspace_size(m, n, r)
         if self.nbytes == 0:
             raise NQError("nq_lbadmm_workspace_size", _lib.NQ_ERR_INVALID_ARG)
@@ -185,18 +191,19 @@ class LBState:
         g = ctypes.c_double(0.0)
         check("nq_lbadmm_prepare", lib.nq_lbadmm_prepare(
             _ptr(W), _dtype(W), self.m, self.n, _ptr(d_in), _ptr(d_out), self.r, seed,
-            ctypes.byref(g), _ptr(self.ws), self.nbytes, _stream()))
+            self.prec, ctypes.byref(g), _ptr(self.ws), self.nbytes, _stream()))
         return g.value
 
     def iterate(self, iters, rho=1.0, lam=1e-4, K=4, want_objective=True):
         obj = (ctypes.c_float * iters)() if want_objective else None
         check("nq_lbadmm_iterate", lib.nq_lbadmm_iterate(
-            *self._args(), rho, lam, iters, K, obj, _ptr(self.ws), self.nbytes, _stream()))
+            *self._args(), rho, lam, iters, K, self.prec, obj, _ptr(self.ws), self.nbytes,
+            _stream()))
         return list(obj) if want_objective else None
 
     def half_step(self, side, rho=1.0, lam=1e-4, K=4):
         check("nq_lbadmm_half_step", lib.nq_lbadmm_half_step(
-            *self._args(), rho, lam, K, side, _ptr(self.ws), self.nbytes, _stream()))
+            *self._args(), rho, lam, K, side, self.prec, _ptr(self.ws), self.nbytes, _stream()))
 
     def finish(self, W=None, d_in=None, d_out=None, want_error=True):
         m, n, r = self._args()
@@ -228,7 +235,7 @@ class LBState:
 
     def sync_operands(self):
         check("nq_lbadmm_sync_operands", lib.nq_lbadmm_sync_operands(
-            *self._args(), _ptr(self.ws), self.nbytes, _stream()))
+            *self._args(), self.prec, _ptr(self.ws), self.nbytes, _stream()))
 
     def check_device_error(self):
         return lib.nq_lbadmm_check(*self._args(), _ptr(self.ws), self.nbytes, _stream())

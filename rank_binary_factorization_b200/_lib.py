@@ -24,7 +24,8 @@ c_vp, c_sz = ctypes.c_void_p, ctypes.c_size_t
 NQ_OK, NQ_ERR_INVALID_ARG, NQ_ERR_WORKSPACE, NQ_ERR_CUDA, NQ_ERR_NONFINITE, NQ_ERR_NOT_SPD, \
     NQ_ERR_TIMEOUT, NQ_ERR_UNSUPPORTED = range(8)
 NQ_F32, NQ_BF16 = 0, 1
-FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9)
+NQ_PREC_BF16, NQ_PREC_FP32 = 0, 1
+FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9, WHAT_LO=10)
 
 # name -> (restype, argtypes); the list is the full set of exported entry points
 SIGNATURES = {
@@ -44,18 +45,18 @@ SIGNATURES = {
     "nq_recon_error": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp,
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_pack_signs": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_vp]),
-    "nq_lbadmm_prepare": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_u64, c_vp,
+    "nq_lbadmm_prepare": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_u64, c_i32,
+                                  c_vp, c_vp, c_sz, c_vp]),
+    "nq_lbadmm_iterate": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_i32, c_vp,
                                   c_vp, c_sz, c_vp]),
-    "nq_lbadmm_iterate": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp,
-                                  c_sz, c_vp]),
-    "nq_lbadmm_half_step": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_sz,
-                                    c_vp]),
+    "nq_lbadmm_half_step": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_i32, c_vp,
+                                    c_sz, c_vp]),
     "nq_lbadmm_finish": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_state_field": (c_i32, [c_i64, c_i64, c_i32, c_i32, c_vp, c_sz,
                                       ctypes.POINTER(c_vp), ctypes.POINTER(c_i64),
                                       ctypes.POINTER(c_i32), ctypes.POINTER(c_i64)]),
-    "nq_lbadmm_sync_operands": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
+    "nq_lbadmm_sync_operands": (c_i32, [c_i64, c_i64, c_i32, c_i32, c_vp, c_sz, c_vp]),
     "nq_lbadmm_check": (c_i32, [c_i64, c_i64, c_i32, c_vp, c_sz, c_vp]),
     "nq_launch_count": (c_i64, []),
     "nq_profile_enable": (c_i32, [c_i32]),
@@ -65,7 +66,7 @@ SIGNATURES = {
 }
 NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
-                  "objective", "finish", "recon"]
+                  "objective", "finish", "recon", "ginv"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -16,6 +18,34 @@ using namespace nq;
 namespace nq {
 static std::atomic<long long> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
+int device_sm_count() {
+    static std::atomic<int> cache[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return kNumSMsB200;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+        v = kNumSMsB200;
+    cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+cudaError_t ensure_smem_limit(const void *func, int bytes, std::atomic<uint64_t> &done) {
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 }  // namespace nq
 
 namespace {
@@ -38,10 +68,18 @@ std::vector<ProfRec> g_prof;
 size_t g_prof_used = 0;
 bool g_prof_on = false;
 
+// NVTX range names of the kernel classes (nq_kernel_class order)
+const char *const kClassNames[NQ_K_COUNT] = {
+    "nq.calib", "nq.calib_finalize", "nq.prep", "nq.gram", "nq.chol", "nq.rhs",
+    "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv"};
+
+// Scope of one kernel class's launches: an NVTX range on the host timeline (seen by
+// profilers; inert otherwise) and, when recording is on, a CUDA event pair on the stream.
 struct ProfScope {
     ProfRec *rec = nullptr;
     cudaStream_t s;
     ProfScope(int cls, cudaStream_t st) : s(st) {
+        nvtxRangePushA(kClassNames[cls]);
         if (!g_prof_on) return;
         std::lock_guard<std::mutex> lk(g_prof_mu);
         if (g_prof_used == g_prof.size()) {
@@ -56,6 +94,7 @@ struct ProfScope {
     }
     ~ProfScope() {
         if (rec) cudaEventRecord(rec->b, s);
+        nvtxRangePop();
     }
 };
 
@@ -68,13 +107,16 @@ inline T *at(void *ws, size_t off) {
 nq_status check_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NQ_ERR_CUDA;
-    static int cached[64];
-    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? NQ_OK : NQ_ERR_UNSUPPORTED;
+    static std::atomic<int> cached[kMaxDevices];
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c) return c == 1 ? NQ_OK : NQ_ERR_UNSUPPORTED;
+    }
     int major = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
         return NQ_ERR_CUDA;
     const bool ok = major == 10;
-    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
     return ok ? NQ_OK : NQ_ERR_UNSUPPORTED;
 }
 
@@ -94,6 +136,8 @@ nq_status check_ws(void *ws, size_t ws_bytes, size_t need) {
 }
 
 int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
+
+inline bool valid_prec(int prec) { return prec == NQ_PREC_BF16 || prec == NQ_PREC_FP32; }
 
 nq_status read_err(int *dev_err, cudaStream_t s, bool reset) {
     int h = 0;
@@ -164,23 +208,30 @@ nq_status lb_open(Lb &lb, int64_t m, int64_t n, int32_t r, void *ws, size_t ws_b
     return check_device();
 }
 
-// Gram of the operand of side ``other`` (its BF16 transpose) into g[other].
-nq_status lb_gram(const Lb &lb, int other, float diag, cudaStream_t s) {
+// Gram of the operand of side ``other`` (its BF16 transpose) into g[other]; the result is
+// symmetric, so only its lower-triangular 128 x 128 tiles are computed and mirrored.  In
+// the FP32-accurate mode the operand is split (hi + lo) and the Gram takes three passes.
+nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s) {
     const LbLayout &L = lb.L;
     const int64_t K = L.rows(other), ld = L.ld_rows(other);
     const __nv_bfloat16 *xt = lb.p<__nv_bfloat16>(L.xt[other]);
-    const int BN = pick_bn(L.r);
+    const __nv_bfloat16 *xl = lb.p<__nv_bfloat16>(L.xtl[other]);
+    constexpr int BN = tc::BM;
     tc::Maps maps;
     memset(&maps, 0, sizeof(maps));
-    if (!tc::make_map_bf16(&maps.a[0], xt, L.r, K, ld, tc::BM) ||
-        !tc::make_map_bf16(&maps.b[0], xt, L.r, K, ld, BN))
-        return NQ_ERR_CUDA;
+    const int nseg = prec == NQ_PREC_FP32 ? 3 : 1;
+    const void *as[3] = {xt, xl, xt}, *bs[3] = {xt, xt, xl};
+    for (int g = 0; g < nseg; ++g)
+        if (!tc::make_map_bf16(&maps.a[g], as[g], L.r, K, ld, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[g], bs[g], L.r, K, ld, BN))
+            return NQ_ERR_CUDA;
     tc::EpiParams ep;
     memset(&ep, 0, sizeof(ep));
     ep.M = L.r;
     ep.N = L.r;
-    ep.nseg = 1;
-    ep.kblocks[0] = (int)ceil_div(K, tc::BK);
+    ep.nseg = nseg;
+    for (int g = 0; g < nseg; ++g) ep.kblocks[g] = (int)ceil_div(K, tc::BK);
+    ep.sym = 1;
     ep.err = &lb.sc->err;
     ep.out = lb.p<float>(L.g[other]);
     ep.ldo = L.r;
@@ -190,12 +241,13 @@ nq_status lb_gram(const Lb &lb, int other, float diag, cudaStream_t s) {
     return NQ_OK;
 }
 
-nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, cudaStream_t s) {
+nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, int prec,
+                       cudaStream_t s) {
     const LbLayout &L = lb.L;
     const int other = 1 - side;
     const int64_t rows = L.rows(side), Kd = L.rows(other);
     const int BN = pick_bn(L.r);
-    nq_status st = lb_gram(lb, other, lambda + rho, s);
+    nq_status st = lb_gram(lb, other, lambda + rho, prec, s);
     if (st) return st;
     {
         ProfScope ps(NQ_K_CHOL, s);
@@ -203,6 +255,9 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
                            &lb.sc->err, lb.sc->bar, s));
+    }
+    {
+        ProfScope ps(NQ_K_GINV, s);
         // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo; G^-1 is
         // symmetric, so only its lower-triangular tiles are computed and mirrored
         tc::Maps maps;
@@ -231,21 +286,27 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, s));
     }
 
-    // R = W^ X_other + rho (Z - L), split into hi + lo bf16
+    // R = W^ X_other + rho (Z - L), split into hi + lo bf16.  FP32-accurate mode: both
+    // operands split, three passes [W^_hi, W^_lo, W^_hi] . [X_hi, X_hi, X_lo].
     {
         tc::Maps maps;
         memset(&maps, 0, sizeof(maps));
         const void *A = side == 0 ? lb.p<void>(L.what) : lb.p<void>(L.whatT);
+        const void *Al = side == 0 ? lb.p<void>(L.whatL) : lb.p<void>(L.whatTL);
         const int64_t lda = side == 0 ? L.ldn : L.ldm;
-        if (!tc::make_map_bf16(&maps.a[0], A, rows, Kd, lda, tc::BM) ||
-            !tc::make_map_bf16(&maps.b[0], lb.p<void>(L.xt[other]), L.r, Kd, L.ld_rows(other), BN))
-            return NQ_ERR_CUDA;
+        const void *B = lb.p<void>(L.xt[other]), *Bl = lb.p<void>(L.xtl[other]);
+        const int nseg = prec == NQ_PREC_FP32 ? 3 : 1;
+        const void *as[3] = {A, Al, A}, *bs[3] = {B, B, Bl};
+        for (int g = 0; g < nseg; ++g)
+            if (!tc::make_map_bf16(&maps.a[g], as[g], rows, Kd, lda, tc::BM) ||
+                !tc::make_map_bf16(&maps.b[g], bs[g], L.r, Kd, L.ld_rows(other), BN))
+                return NQ_ERR_CUDA;
         tc::EpiParams ep;
         memset(&ep, 0, sizeof(ep));
         ep.M = (int)rows;
         ep.N = L.r;
-        ep.nseg = 1;
-        ep.kblocks[0] = (int)ceil_div(Kd, tc::BK);
+        ep.nseg = nseg;
+        for (int g = 0; g < nseg; ++g) ep.kblocks[g] = (int)ceil_div(Kd, tc::BK);
         ep.err = &lb.sc->err;
         ep.S = lb.p<float>(L.s[side]);
         ep.a = lb.p<float>(L.a[side]);
@@ -288,6 +349,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, c
         ep.ldr = L.ldr;
         ep.X = lb.p<float>(L.x[side]);
         ep.Xt = lb.p<__nv_bfloat16>(L.xt[side]);
+        ep.XtL = prec == NQ_PREC_FP32 ? lb.p<__nv_bfloat16>(L.xtl[side]) : nullptr;
         ep.ldxt = L.ld_rows(side);
         ep.objective = side == 1;
         ep.part = lb.p<double>(L.part);
@@ -311,7 +373,8 @@ nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
 }
 
 nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
-                     const float *d_out, uint64_t seed, cudaStream_t s) {
+                     const float *d_out, uint64_t seed, int prec, cudaStream_t s) {
+    const bool split = prec == NQ_PREC_FP32;
     const LbLayout &L = lb.L;
     ProfScope ps(NQ_K_PREP, s);
     NQ_CK(cudaMemsetAsync(lb.sc, 0, sizeof(Scalars), s));
@@ -319,7 +382,9 @@ nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
     NQ_CK(reduce_partials(lb.p<double>(L.part), kRedBlocks, &lb.sc->wt_norm2, &lb.sc->gamma, L.r,
                           s));
     NQ_CK(what_cast(W, bf16, L.m, L.n, d_in, d_out, &lb.sc->gamma, lb.p<__nv_bfloat16>(L.what),
-                    L.ldn, lb.p<__nv_bfloat16>(L.whatT), L.ldm, lb.p<double>(L.part), s));
+                    L.ldn, lb.p<__nv_bfloat16>(L.whatT), L.ldm,
+                    split ? lb.p<__nv_bfloat16>(L.whatL) : nullptr,
+                    split ? lb.p<__nv_bfloat16>(L.whatTL) : nullptr, lb.p<double>(L.part), s));
     NQ_CK(reduce_partials(lb.p<double>(L.part), kRedBlocks, &lb.sc->what_norm2, nullptr, L.r, s));
     for (int sd = 0; sd < 2; ++sd) {
         const int64_t rw = L.rows(sd);
@@ -327,21 +392,26 @@ nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
         NQ_CK(cudaMemsetAsync(lb.p<void>(L.a[sd]), 0, (size_t)rw * 4, s));
         NQ_CK(cudaMemsetAsync(lb.p<void>(L.b[sd]), 0, (size_t)L.r * 4, s));
         NQ_CK(cudaMemsetAsync(lb.p<void>(L.xt[sd]), 0, (size_t)L.r * L.ld_rows(sd) * 2, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.xtl[sd]), 0, (size_t)L.r * L.ld_rows(sd) * 2, s));
+    }
+    if (!split) {   // the low parts read as zero (state fields, precision switches)
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.whatL), 0, (size_t)L.m * L.ldn * 2, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.whatTL), 0, (size_t)L.n * L.ldm * 2, s));
     }
     NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[0]), 0, (size_t)L.m * L.ldr * 4, s));
     NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[1]), 0, (size_t)L.n * L.ldr * 4, s));
-    NQ_CK(init_v0(L.n, L.r, seed, lb.p<float>(L.x[1]), L.ldr, lb.p<__nv_bfloat16>(L.xt[1]), L.ldn,
-                  s));
+    NQ_CK(init_v0(L.n, L.r, seed, lb.p<float>(L.x[1]), L.ldr, lb.p<__nv_bfloat16>(L.xt[1]),
+                  split ? lb.p<__nv_bfloat16>(L.xtl[1]) : nullptr, L.ldn, s));
     return NQ_OK;
 }
 
-nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, float *objective_h,
-                     cudaStream_t s) {
+nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, int prec,
+                     float *objective_h, cudaStream_t s) {
     for (int t = 0; t < iters; ++t) {
-        nq_status st = lb_half_step(lb, 0, rho, lambda, K, s);
+        nq_status st = lb_half_step(lb, 0, rho, lambda, K, prec, s);
         if (st) return st;
         if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
-        if ((st = lb_half_step(lb, 1, rho, lambda, K, s))) return st;
+        if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s))) return st;
         if (objective_h && t > 0 && (t % kObjRing) == 0) {
             // the ring holds the objectives of iterations t - kObjRing .. t - 1; the copy is
             // stream-ordered before the next write to slot 0
@@ -350,7 +420,7 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, fl
         }
     }
     // objective of the last iteration needs the Gram of the last V
-    nq_status st = lb_gram(lb, 1, lambda + rho, s);
+    nq_status st = lb_gram(lb, 1, lambda + rho, prec, s);
     if (st) return st;
     if ((st = lb_objective(lb, lambda + rho, (iters - 1) % kObjRing, s))) return st;
     if (objective_h) {
@@ -509,14 +579,14 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r) {
 }
 
 nq_status nq_lbadmm_prepare(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
-                            const float *d_out, int32_t r, uint64_t seed, double *gamma_out,
-                            void *ws, size_t ws_bytes, nq_stream_t stream) {
-    if (!W || (dt != NQ_F32 && dt != NQ_BF16)) return NQ_ERR_INVALID_ARG;
+                            const float *d_out, int32_t r, uint64_t seed, nq_precision prec,
+                            double *gamma_out, void *ws, size_t ws_bytes, nq_stream_t stream) {
+    if (!W || (dt != NQ_F32 && dt != NQ_BF16) || !valid_prec(prec)) return NQ_ERR_INVALID_ARG;
     Lb lb;
     nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
     if (st) return st;
     cudaStream_t s = cs(stream);
-    if ((st = lb_prepare(lb, W, dt == NQ_BF16, d_in, d_out, seed, s))) return st;
+    if ((st = lb_prepare(lb, W, dt == NQ_BF16, d_in, d_out, seed, prec, s))) return st;
     if (gamma_out) {
         NQ_CK(cudaMemcpyAsync(gamma_out, &lb.sc->gamma, sizeof(double), cudaMemcpyDeviceToHost, s));
         return read_err(&lb.sc->err, s, false);
@@ -525,28 +595,30 @@ nq_status nq_lbadmm_prepare(const void *W, nq_dtype dt, int64_t m, int64_t n, co
 }
 
 nq_status nq_lbadmm_iterate(int64_t m, int64_t n, int32_t r, float rho, float lambda,
-                            int32_t iters, int32_t K, float *objective, void *ws, size_t ws_bytes,
-                            nq_stream_t stream) {
+                            int32_t iters, int32_t K, nq_precision prec, float *objective,
+                            void *ws, size_t ws_bytes, nq_stream_t stream) {
     if (!(rho > 0.f) || !(lambda >= 0.f) || iters < 1 || K < 1 || !isfinite(rho) ||
-        !isfinite(lambda))
+        !isfinite(lambda) || !valid_prec(prec))
         return NQ_ERR_INVALID_ARG;
     Lb lb;
     nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
     if (st) return st;
     cudaStream_t s = cs(stream);
-    if ((st = lb_iterate(lb, rho, lambda, iters, K, objective, s))) return st;
+    if ((st = lb_iterate(lb, rho, lambda, iters, K, prec, objective, s))) return st;
     if (objective) return read_err(&lb.sc->err, s, false);
     return NQ_OK;
 }
 
 nq_status nq_lbadmm_half_step(int64_t m, int64_t n, int32_t r, float rho, float lambda, int32_t K,
-                              int32_t side, void *ws, size_t ws_bytes, nq_stream_t stream) {
-    if (!(rho > 0.f) || !(lambda >= 0.f) || K < 1 || (side != 0 && side != 1))
+                              int32_t side, nq_precision prec, void *ws, size_t ws_bytes,
+                              nq_stream_t stream) {
+    if (!(rho > 0.f) || !(lambda >= 0.f) || K < 1 || (side != 0 && side != 1) ||
+        !valid_prec(prec))
         return NQ_ERR_INVALID_ARG;
     Lb lb;
     nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
     if (st) return st;
-    return lb_half_step(lb, side, rho, lambda, K, cs(stream));
+    return lb_half_step(lb, side, rho, lambda, K, prec, cs(stream));
 }
 
 nq_status nq_lbadmm_finish(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
@@ -587,8 +659,11 @@ nq_status nq_lbadmm(const void *W, nq_dtype dt, int64_t m, int64_t n, const floa
     if (st) return st;
     cudaStream_t s = cs(stream);
     const int bf16 = dt == NQ_BF16;
-    if ((st = lb_prepare(lb, W, bf16, d_in, d_out, seed, s))) return st;
-    if ((st = lb_iterate(lb, rho, lambda, iters, K, objective, s))) return st;
+    // precision follows the weights: BF16 operands for BF16 weights, split (FP32-accurate)
+    // operands for FP32 weights
+    const int prec = bf16 ? NQ_PREC_BF16 : NQ_PREC_FP32;
+    if ((st = lb_prepare(lb, W, bf16, d_in, d_out, seed, prec, s))) return st;
+    if ((st = lb_iterate(lb, rho, lambda, iters, K, prec, objective, s))) return st;
     if ((st = lb_finish(lb, W, bf16, d_in, d_out, U_packed, V_packed, s1, s2,
                         final_rel_err != nullptr, s)))
         return st;
@@ -690,6 +765,7 @@ nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, voi
         case NQ_FIELD_BU: off = L.b[0]; cnt = r; l = 1; break;
         case NQ_FIELD_BV: off = L.b[1]; cnt = r; l = 1; break;
         case NQ_FIELD_WHAT: off = L.what; cnt = m * L.ldn; l = L.ldn; eb = 2; break;
+        case NQ_FIELD_WHAT_LO: off = L.whatL; cnt = m * L.ldn; l = L.ldn; eb = 2; break;
         case NQ_FIELD_GAMMA: off = L.scal + offsetof(Scalars, gamma); cnt = 1; l = 1; eb = 8; break;
         default: return NQ_ERR_INVALID_ARG;
     }
@@ -700,19 +776,24 @@ nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, voi
     return NQ_OK;
 }
 
-nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, void *ws, size_t ws_bytes,
-                                  nq_stream_t stream) {
+nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, nq_precision prec, void *ws,
+                                  size_t ws_bytes, nq_stream_t stream) {
+    if (!valid_prec(prec)) return NQ_ERR_INVALID_ARG;
     Lb lb;
     nq_status st = lb_open(lb, m, n, r, ws, ws_bytes);
     if (st) return st;
     cudaStream_t s = cs(stream);
     const LbLayout &L = lb.L;
+    const bool split = prec == NQ_PREC_FP32;
     NQ_CK(transpose_to_bf16(lb.p<float>(L.x[0]), L.m, L.r, L.ldr, lb.p<__nv_bfloat16>(L.xt[0]),
-                            L.ldm, s));
+                            split ? lb.p<__nv_bfloat16>(L.xtl[0]) : nullptr, L.ldm, s));
     NQ_CK(transpose_to_bf16(lb.p<float>(L.x[1]), L.n, L.r, L.ldr, lb.p<__nv_bfloat16>(L.xt[1]),
-                            L.ldn, s));
+                            split ? lb.p<__nv_bfloat16>(L.xtl[1]) : nullptr, L.ldn, s));
     NQ_CK(transpose_bf16(lb.p<__nv_bfloat16>(L.what), L.m, L.n, L.ldn,
                          lb.p<__nv_bfloat16>(L.whatT), L.ldm, s));
+    if (split)
+        NQ_CK(transpose_bf16(lb.p<__nv_bfloat16>(L.whatL), L.m, L.n, L.ldn,
+                             lb.p<__nv_bfloat16>(L.whatTL), L.ldm, s));
     return NQ_OK;
 }
 

@@ -623,7 +623,11 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
                          unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
     constexpr int smem = (5 * TB * LDS + TB) * sizeof(float);
-    static int grid = 0;
+    // grid of the cooperative launch (one CTA per SM), per device
+    static std::atomic<int> grids[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    int grid = grids[dev].load();
     if (!grid) {
         cudaError_t e = cudaFuncSetAttribute(chol2_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -631,11 +635,10 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
         int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chol2_kernel, 256, smem);
         if (e != cudaSuccess) return e;
-        int dev = 0, sms = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        grid = sms * (per_sm < 1 ? per_sm : 1);
+        if (per_sm < 1) return cudaErrorLaunchOutOfResources;
+        grid = device_sm_count();
         if (grid < 3) return cudaErrorLaunchOutOfResources;
+        grids[dev].store(grid);
     }
     cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;

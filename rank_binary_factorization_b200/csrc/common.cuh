@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/nq.h"
 
 #define NQ_HD __host__ __device__ __forceinline__
@@ -14,6 +16,18 @@ constexpr int kNumSMsB200 = 148;
 
 // Host-side count of kernel launches issued by the library (nq_launch_count).
 void count_launch(int n = 1);
+
+// ---- per-device launch state (host) ------------------------------------------------
+// Launch settings depend on the device a call runs on, so every cache is kept per
+// device ordinal; one process may drive several GPUs, from several host threads.
+constexpr int kMaxDevices = 64;
+// Ordinal of the current device, or -1 if it cannot be read or is >= kMaxDevices.
+int current_device();
+// SM count of the current device (cached per device; kNumSMsB200 if unknown).
+int device_sm_count();
+// Set the dynamic shared-memory limit of ``func`` to ``bytes`` once per device; ``done``
+// is the caller's per-kernel bit set of configured devices.
+cudaError_t ensure_smem_limit(const void *func, int bytes, std::atomic<uint64_t> &done);
 
 NQ_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 NQ_HD int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }

@@ -159,6 +159,17 @@ __device__ __forceinline__ void split_mirror(const EpiParams &p, int row, int co
     }
 }
 
+// Mirrored store of a symmetric Gram tile (EPI_GRAM with sym): entry (row, col0 + j) also
+// goes to (col0 + j, row).  Off-diagonal tiles only, so no ridge term is added here.
+__device__ __forceinline__ void gram_mirror(const EpiParams &p, int row, int col0,
+                                            const float (&v)[16]) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        if (col0 + j >= p.N) break;
+        p.out[(int64_t)(col0 + j) * p.ldo + row] = v[j];
+    }
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int col0,
                                                const float (&v)[16], float &acc_sum) {
@@ -256,8 +267,13 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
             st16(Xrow, v);
             st16(Srow, sn);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = __float2bfloat16_rn(v[j]);
+            for (int j = 0; j < 16; ++j) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = h;
+                if (p.XtL)
+                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] =
+                        __float2bfloat16_rn(v[j] - __bfloat162float(h));
+            }
         } else {
             for (int j = 0; j < 16 && col0 + j < p.N; ++j) {
                 const float x = v[j];
@@ -266,7 +282,11 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
                 const float z = sgn(sold) * ai * p.b[col0 + j];
                 Xrow[j] = x;
                 Srow[j] = x + sold - z;
-                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = __float2bfloat16_rn(x);
+                const __nv_bfloat16 h = __float2bfloat16_rn(x);
+                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = h;
+                if (p.XtL)
+                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] =
+                        __float2bfloat16_rn(x - __bfloat162float(h));
                 if (p.objective) {
                     const int64_t o = (int64_t)row * p.ldr + col0 + j;
                     const float r = __bfloat162float(p.Rhi[o]) + __bfloat162float(p.Rlo[o]);
@@ -468,6 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
                         if constexpr (EPI == EPI_SPLIT)
                             if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
+                        if constexpr (EPI == EPI_GRAM)
+                            if (p.sym && m0 != n0) gram_mirror(p, row, n0 + c, v);
                     }
                 }
                 tc_fence_before();
@@ -534,20 +556,13 @@ template <int BN, int STAGES, int EPI>
 static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s) {
     constexpr int smem = STAGES * (A_TILE_BYTES + BN * BK * 2) + 1024 + 256;  // + barriers
     auto kern = gemm_kernel<BN, STAGES, EPI>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms < 1) sms = kNumSMsB200;
-    }
-    const int64_t tiles = num_tiles(p.M, p.N, BN);
+    static std::atomic<uint64_t> configured{0};   // devices whose smem limit is set
+    cudaError_t e = ensure_smem_limit((const void *)kern, smem, configured);
+    if (e != cudaSuccess) return e;
+    int sms = device_sm_count();
+    if (p.max_ctas > 0 && p.max_ctas < sms) sms = p.max_ctas;
+    const int64_t tiles = p.sym ? ceil_div(p.M, BM) * (ceil_div(p.M, BM) + 1) / 2
+                                : num_tiles(p.M, p.N, BN);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     kern<<<grid, kThreads, smem, s>>>(maps, p);
     count_launch();

@@ -36,8 +36,10 @@ struct EpiParams {
     int nseg;
     int kblocks[3];
     int tri_k;          // operands zero for k < row index: start each tile's K at max(m0, n0)
-    int sym;            // symmetric result (EPI_SPLIT, BN == BM): lower-triangular tiles only,
-                        // each off-diagonal tile also written mirrored
+    int sym;            // symmetric result (EPI_SPLIT / EPI_GRAM, BN == BM, M == N): lower-
+                        // triangular tiles only, each off-diagonal tile also written mirrored
+    int max_ctas;       // 0: one CTA per SM; else at most this many CTAs (SMs left free for
+                        // kernels running beside this one on another stream)
     int *err;
     // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
     float *out;
@@ -53,9 +55,10 @@ struct EpiParams {
     // EPI_RHS: R = acc + rho (2 sign(S) a b^T - S) split into hi + lo bf16
     __nv_bfloat16 *Rhi, *Rlo;  // [M][ldr]
     int64_t ldr;
-    // EPI_SOLVE: X = acc; S <- X + S - sign(S) a b^T; Xt[col][row] = bf16(X)
+    // EPI_SOLVE: X = acc; S <- X + S - sign(S) a b^T; Xt[col][row] = bf16(X) and, when XtL
+    // is set, XtL[col][row] = bf16(X - Xt) (the low part of a split-BF16 operand)
     float *X;                  // [M][ldf]
-    __nv_bfloat16 *Xt;         // [N][ldxt]
+    __nv_bfloat16 *Xt, *XtL;   // [N][ldxt]
     int64_t ldxt;
     int objective;             // also sum (R - rho (2Z - S_old)) . X into part[tile]
     double *part;              // per-tile partial sums (EPI_SOLVE objective, EPI_RECON)

@@ -332,9 +332,12 @@ __global__ void __launch_bounds__(256)
     what_cast_kernel(const void *__restrict__ W, int w_bf16, int64_t m, int64_t n,
                      const float *__restrict__ d_in, const float *__restrict__ d_out,
                      const double *__restrict__ gamma, __nv_bfloat16 *What, int64_t ldn,
-                     __nv_bfloat16 *WhatT, int64_t ldm, double *part) {
+                     __nv_bfloat16 *WhatT, int64_t ldm, __nv_bfloat16 *WhatL,
+                     __nv_bfloat16 *WhatTL, double *part) {
     __shared__ __nv_bfloat16 tile[32][34];
+    __shared__ __nv_bfloat16 tile_lo[32][34];
     __shared__ double sh[256];
+    const bool split = WhatL != nullptr;
     const double g = *gamma;
     const float inv = g > 0.0 ? (float)(1.0 / g) : 0.f;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
@@ -345,22 +348,34 @@ __global__ void __launch_bounds__(256)
         float f = 0.f;
         for (int k = ty; k < 32; k += 8) {
             const int64_t i = i0 + k, j = j0 + tx;
-            __nv_bfloat16 h = __float2bfloat16_rn(0.f);
+            __nv_bfloat16 h = __float2bfloat16_rn(0.f), l = h;
             if (i < m && j < n) {
                 const float w = (d_out ? d_out[i] : 1.f) * load_wf(W, w_bf16, i * n + j) *
                                 (d_in ? d_in[j] : 1.f);
-                h = __float2bfloat16_rn(w * inv);
-                const float hv = __bfloat162float(h);
+                const float x = w * inv;
+                h = __float2bfloat16_rn(x);
+                float hv = __bfloat162float(h);
+                if (split) {
+                    l = __float2bfloat16_rn(x - hv);
+                    hv += __bfloat162float(l);
+                }
                 f = fmaf(hv, hv, f);
             }
-            if (i < m && j < ldn) What[i * ldn + j] = h;
+            if (i < m && j < ldn) {
+                What[i * ldn + j] = h;
+                if (split) WhatL[i * ldn + j] = l;
+            }
             tile[k][tx] = h;
+            tile_lo[k][tx] = l;
         }
         acc += f;
         __syncthreads();
         for (int k = ty; k < 32; k += 8) {
             const int64_t j = j0 + k, i = i0 + tx;
-            if (j < n && i < ldm) WhatT[j * ldm + i] = tile[tx][k];
+            if (j < n && i < ldm) {
+                WhatT[j * ldm + i] = tile[tx][k];
+                if (split) WhatTL[j * ldm + i] = tile_lo[tx][k];
+            }
         }
         __syncthreads();
     }
@@ -370,9 +385,10 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t what_cast(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
                       const float *d_out, const double *gamma, __nv_bfloat16 *What, int64_t ldn,
-                      __nv_bfloat16 *WhatT, int64_t ldm, double *part, cudaStream_t s) {
+                      __nv_bfloat16 *WhatT, int64_t ldm, __nv_bfloat16 *WhatL,
+                      __nv_bfloat16 *WhatTL, double *part, cudaStream_t s) {
     what_cast_kernel<<<kRedBlocks, 256, 0, s>>>(W, w_bf16, m, n, d_in, d_out, gamma, What, ldn,
-                                                WhatT, ldm, part);
+                                                WhatT, ldm, WhatL, WhatTL, part);
     count_launch();
     return cudaGetLastError();
 }
@@ -386,7 +402,7 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t idx) {
 }
 
 __global__ void init_v0_kernel(int64_t n, int32_t r, uint64_t seed, float c, float *X,
-                               int64_t ldr, __nv_bfloat16 *Xt, int64_t ldn) {
+                               int64_t ldr, __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldn) {
     const int64_t total = n * (int64_t)r;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -397,21 +413,23 @@ __global__ void init_v0_kernel(int64_t n, int32_t r, uint64_t seed, float c, flo
         // column-major pass over Xt (j fastest): element (k2, j2)
         const int64_t k2 = e / n, j2 = e % n;
         const float v2 = (splitmix64(seed, (uint64_t)(j2 * r + k2)) >> 63) ? -c : c;
-        Xt[k2 * ldn + j2] = __float2bfloat16_rn(v2);
+        const __nv_bfloat16 h = __float2bfloat16_rn(v2);
+        Xt[k2 * ldn + j2] = h;
+        if (XtL) XtL[k2 * ldn + j2] = __float2bfloat16_rn(v2 - __bfloat162float(h));
     }
 }
 
 cudaError_t init_v0(int64_t n, int32_t r, uint64_t seed, float *X, int64_t ldr,
-                    __nv_bfloat16 *Xt, int64_t ldn, cudaStream_t s) {
+                    __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldn, cudaStream_t s) {
     const float c = sqrtf(2.0f / (float)n);
-    init_v0_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(n, r, seed, c, X, ldr, Xt, ldn);
+    init_v0_kernel<<<4 * kNumSMsB200, 256, 0, s>>>(n, r, seed, c, X, ldr, Xt, XtL, ldn);
     count_launch();
     return cudaGetLastError();
 }
 
 __global__ void __launch_bounds__(256)
     transpose_to_bf16_kernel(const float *__restrict__ X, int64_t rows, int32_t r, int64_t ldx,
-                             __nv_bfloat16 *Xt, int64_t ldt) {
+                             __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldt) {
     __shared__ float tile[32][33];
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
     const int64_t i0 = (int64_t)blockIdx.y * 32, k0 = (int64_t)blockIdx.x * 32;
@@ -422,14 +440,19 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     for (int a = ty; a < 32; a += 8) {
         const int64_t k = k0 + a, i = i0 + tx;
-        if (k < r && i < rows) Xt[k * ldt + i] = __float2bfloat16_rn(tile[tx][a]);
+        if (k < r && i < rows) {
+            const float x = tile[tx][a];
+            const __nv_bfloat16 h = __float2bfloat16_rn(x);
+            Xt[k * ldt + i] = h;
+            if (XtL) XtL[k * ldt + i] = __float2bfloat16_rn(x - __bfloat162float(h));
+        }
     }
 }
 
 cudaError_t transpose_to_bf16(const float *X, int64_t rows, int32_t r, int64_t ldx,
-                              __nv_bfloat16 *Xt, int64_t ldt, cudaStream_t s) {
+                              __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldt, cudaStream_t s) {
     dim3 grid((unsigned)ceil_div(r, 32), (unsigned)ceil_div(rows, 32));
-    transpose_to_bf16_kernel<<<grid, 256, 0, s>>>(X, rows, r, ldx, Xt, ldt);
+    transpose_to_bf16_kernel<<<grid, 256, 0, s>>>(X, rows, r, ldx, Xt, XtL, ldt);
     count_launch();
     return cudaGetLastError();
 }
@@ -585,13 +608,18 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
                  float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
                  cudaStream_t s) {
     const size_t smem = (size_t)(kSvidRows * ldf + r) * sizeof(float);
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
+    // largest dynamic shared-memory limit set so far, per device
+    static std::atomic<size_t> configured[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (smem > 48 * 1024 && smem > configured[dev].load()) {
         cudaError_t e = cudaFuncSetAttribute(svid_pass_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        configured = smem;
+        size_t prev = configured[dev].load();
+        while (prev < smem && !configured[dev].compare_exchange_weak(prev, smem)) {
+        }
     }
     for (int pass = 1; pass <= K; ++pass) {
         const float *b_in = pass == 1 ? nullptr : bcur + (size_t)((pass - 1) & 1) * r;

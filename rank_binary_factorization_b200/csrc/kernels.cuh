@@ -27,16 +27,19 @@ cudaError_t wt_norm_partials(const void *W, int w_bf16, int64_t m, int64_t n, co
 cudaError_t reduce_partials(const double *part, int count, double *sum, double *gamma, int r,
                             cudaStream_t s);
 // W^ = bf16(d_out W d_in / gamma) into What [m][ldn] and WhatT [n][ldm] (zero padded);
-// part[b] = partial sums of W^^2.
+// with WhatL / WhatTL non-null also the low parts bf16(x - bf16(x)) of a split operand.
+// part[b] = partial sums of W^^2 (of hi + lo when split).
 cudaError_t what_cast(const void *W, int w_bf16, int64_t m, int64_t n, const float *d_in,
                       const float *d_out, const double *gamma, __nv_bfloat16 *What, int64_t ldn,
-                      __nv_bfloat16 *WhatT, int64_t ldm, double *part, cudaStream_t s);
-// V_0 = sqrt(2/n) * splitmix64 signs into X [n][ldr] (float) and Xt [r][ldn] (bf16).
+                      __nv_bfloat16 *WhatT, int64_t ldm, __nv_bfloat16 *WhatL,
+                      __nv_bfloat16 *WhatTL, double *part, cudaStream_t s);
+// V_0 = sqrt(2/n) * splitmix64 signs into X [n][ldr] (float) and Xt [r][ldn] (bf16; XtL,
+// when non-null, the low part).
 cudaError_t init_v0(int64_t n, int32_t r, uint64_t seed, float *X, int64_t ldr,
-                    __nv_bfloat16 *Xt, int64_t ldn, cudaStream_t s);
-// Xt[k][i] = bf16(X[i][k]) for i < rows, k < r.
+                    __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldn, cudaStream_t s);
+// Xt[k][i] = bf16(X[i][k]) for i < rows, k < r (XtL, when non-null: the low part).
 cudaError_t transpose_to_bf16(const float *X, int64_t rows, int32_t r, int64_t ldx,
-                              __nv_bfloat16 *Xt, int64_t ldt, cudaStream_t s);
+                              __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldt, cudaStream_t s);
 // B[j][i] = A[i][j] (bf16), A rows x cols with row stride lda, B row stride ldb.
 cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, int64_t lda,
                            __nv_bfloat16 *B, int64_t ldb, cudaStream_t s);

@@ -35,8 +35,8 @@ struct LbLayout {
     int64_t ldm = 0;   // leading dim of W^^T rows (m padded) and of Ut
     int64_t rp = 0;    // r padded to 64 (Cholesky tiles)
     int nsv = 0;       // CTAs of an SVID pass (rows of its partial array)
-    size_t scal = 0, what = 0, whatT = 0, x[2] = {0, 0}, s[2] = {0, 0}, a[2] = {0, 0},
-           b[2] = {0, 0}, xt[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
+    size_t scal = 0, what = 0, whatT = 0, whatL = 0, whatTL = 0, x[2] = {0, 0}, s[2] = {0, 0},
+           a[2] = {0, 0}, b[2] = {0, 0}, xt[2] = {0, 0}, xtl[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
            gih = 0, gil = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
            partb = 0, obj = 0, total = 0;
     size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
@@ -64,6 +64,9 @@ struct LbLayout {
         scal = take(sizeof(Scalars));
         what = take((size_t)m * ldn * 2);
         whatT = take((size_t)n * ldm * 2);
+        // low BF16 parts (split operands of the FP32-accurate precision mode)
+        whatL = take((size_t)m * ldn * 2);
+        whatTL = take((size_t)n * ldm * 2);
         for (int sd = 0; sd < 2; ++sd) {
             const int64_t rw = sd == 0 ? m : n;
             x[sd] = take((size_t)rw * ldr * 4);
@@ -71,6 +74,7 @@ struct LbLayout {
             a[sd] = take((size_t)rw * 4);
             b[sd] = take((size_t)r * 4);
             xt[sd] = take((size_t)r * (sd == 0 ? ldm : ldn) * 2);
+            xtl[sd] = take((size_t)r * (sd == 0 ? ldm : ldn) * 2);
             g[sd] = take((size_t)r * r * 4);
         }
         rhi = take((size_t)maxrows * ldr * 2);

@@ -18,9 +18,12 @@ def test_kernel_units():
     m, n, r, K, T = 11008, 4096, 1000, 4, 262144
     assert bench.kernel_units("calib", m, n, r, K, T) == (T * (m + n), "B", "hbm")
     assert bench.kernel_units("rhs", m, n, r, K, T) == (2.0 * m * n * r, "FLOP", "tensor")
-    assert bench.kernel_units("gram", m, n, r, K, T)[0] == pytest.approx((m + n) * r * r)
+    # symmetric Gram: half of 2 rows r^2, averaged over the two sides
+    assert bench.kernel_units("gram", m, n, r, K, T)[0] == pytest.approx((m + n) * r * r / 2)
     assert bench.kernel_units("solve", m, n, r, K, T)[0] == pytest.approx((m + n) * r * r)
-    assert bench.kernel_units("chol", m, n, r, K, T) == (float(r) ** 3, "FLOP", "alu")
+    # the method's Cholesky: r^3 / 3 (the inverse the library also forms is not counted)
+    assert bench.kernel_units("chol", m, n, r, K, T) == (float(r) ** 3 / 3, "FLOP", "alu")
+    assert bench.kernel_units("ginv", m, n, r, K, T) == (float(r) ** 3 / 3, "FLOP", "tensor")
     assert bench.kernel_units("svid", m, n, r, K, T)[0] == pytest.approx(2.0 * K * (m + n) * r)
     assert bench.kernel_units("objective", m, n, r, K, T) is None
 
@@ -47,10 +50,18 @@ def test_roofline_entry_fractions():
     assert bench.roofline_entry("rhs", 0, 1.0, m, n, r, K, T, peaks) is None
 
 
-def test_traffic_only_for_the_captured_problem():
-    assert bench.ncu_traffic("chol", 4096, 4096, 2032, 262144) > 0
-    assert bench.ncu_traffic("chol", 8192, 8192, 4080, 262144) is None
+def test_traffic_only_for_captured_kernels():
+    # only the calibration kernel's capture is current; it scales with the stream size
+    assert bench.ncu_traffic("calib", 4096, 4096, 2032, 262144) > 0
+    assert bench.ncu_traffic("chol", 4096, 4096, 2032, 262144) is None
     assert bench.ncu_traffic("svid", 4096, 4096, 2032, 262144) is None
+
+
+def test_alu_peak_is_marked_derived():
+    peaks = dict(hbm_gbs=6000.0, bf16_tflops=1600.0, bf16_tflops_sustained=1400.0,
+                 fp32_tflops=70.0, source="test")
+    e = bench.roofline_entry("chol", 2, 1.0, 4096, 4096, 2032, 4, 1024, peaks)
+    assert e["bound"] == "alu" and e["peak"] == 70.0 and "derived" in e["peak_kind"]
 
 
 def test_peaks_measured_or_fallback(tmp_path, monkeypatch):

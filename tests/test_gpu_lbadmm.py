@@ -2,13 +2,13 @@
 
 Tolerances:
   * single U (V) step on identical inputs: max|dX| / max|X_ref| <= 2e-3, same for S, a, b;
-    a sign of S may differ only where |S_ref| < 1e-3 rms(S_ref);
+    a sign of S may differ only where |S_ref| < 1e-3 rms(S_ref).  In the FP32-accurate
+    precision mode (split BF16 operands) on FP32 inputs: 1e-4;
   * packing on identical signs: bit-exact;
-  * end-to-end reconstruction error within 1% of the oracle's, per instance where the
-    iteration is insensitive to BF16-size perturbations, else within the range the oracle
-    itself spans under such perturbations.
-Inputs of the single-step tests are generated here (BF16-exact target and latent
-operand), imported into the GPU state, and fed unchanged to the oracle.
+  * end-to-end reconstruction error within 1% of the oracle's, per instance.
+Inputs of the single-step tests are generated here (BF16-exact target and latent operand
+for the BF16 mode, FP32 values for the FP32-accurate mode), imported into the GPU state,
+and fed unchanged to the oracle.
 """
 import numpy as np
 import pytest
@@ -22,6 +22,7 @@ from synth import gaussian_weight, planted_problem, stream_tensor
 
 pytestmark = pytest.mark.gpu
 TOL_STEP = 2e-3
+TOL_STEP_FP32 = 1e-4
 TOL_E2E = 0.01
 
 
@@ -65,8 +66,18 @@ def test_pack_signs_bit_exact(nq, r):
     np.testing.assert_array_equal(bits.cpu().numpy().view(np.uint32), O.pack_signs(X))
 
 
+def _split_bf16(a):
+    """hi = bf16(a), lo = bf16(a - hi) of a float32 array (the split operand of the
+    FP32-accurate mode)."""
+    t = torch.from_numpy(np.asarray(a, dtype=np.float32))
+    hi = t.to(torch.bfloat16)
+    return hi, (t - hi.float()).to(torch.bfloat16)
+
+
 def _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV):
-    st.field("WHAT")[:, :n].copy_(torch.from_numpy(Wh).to(torch.bfloat16).cuda())
+    hi, lo = _split_bf16(Wh)
+    st.field("WHAT")[:, :n].copy_(hi.cuda())
+    st.field("WHAT_LO")[:, :n].copy_(lo.cuda())
     for name, val in (("U", U), ("V", V), ("SU", SU), ("SV", SV)):
         st.field(name)[:, :r].copy_(torch.from_numpy(val).float().cuda())
     for name, val in (("AU", aU), ("BU", bU), ("AV", aV), ("BV", bV)):
@@ -74,16 +85,20 @@ def _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV):
     st.sync_operands()
 
 
-def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4):
+def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4, prec="bf16"):
     rng = np.random.default_rng(seed)
-    Wh = bf16_exact(rng.standard_normal((m, n)) * 0.1)
-    U = bf16_exact(rng.standard_normal((m, r)) * 0.2).astype(np.float64)
-    V = bf16_exact(rng.standard_normal((n, r)) * 0.2).astype(np.float64)
+    # BF16 mode: BF16-exact target and latent operand (the values its MMAs see);
+    # FP32-accurate mode: plain FP32 values
+    cast = bf16_exact if prec == "bf16" else (lambda a: np.asarray(a, dtype=np.float32))
+    tol = TOL_STEP if prec == "bf16" else TOL_STEP_FP32
+    Wh = cast(rng.standard_normal((m, n)) * 0.1)
+    U = cast(rng.standard_normal((m, r)) * 0.2).astype(np.float64)
+    V = cast(rng.standard_normal((n, r)) * 0.2).astype(np.float64)
     SU = rng.standard_normal((m, r)).astype(np.float32)
     SV = rng.standard_normal((n, r)).astype(np.float32)
     aU, aV = [np.abs(rng.standard_normal(k)).astype(np.float32) / np.sqrt(k) for k in (m, n)]
     bU, bV = [np.abs(rng.standard_normal(r)).astype(np.float32) for _ in range(2)]
-    st = nq.LBState(m, n, r)
+    st = nq.LBState(m, n, r, prec=prec)
     st.prepare(torch.zeros(m, n, device="cuda"), seed=0)
     _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV)
     st.half_step(side, rho, lam, K)
@@ -102,10 +117,10 @@ def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4):
     S = st.field("S" + tag)[:, :r].cpu().double().numpy()
     a = st.field("A" + tag).cpu().double().numpy()
     b = st.field("B" + tag).cpu().double().numpy()
-    assert max_rel(X, Xr) <= TOL_STEP
-    assert max_rel(S, Sr) <= TOL_STEP
-    assert max_rel(a, ar) <= TOL_STEP
-    assert max_rel(b, br) <= TOL_STEP
+    assert max_rel(X, Xr) <= tol
+    assert max_rel(S, Sr) <= tol
+    assert max_rel(a, ar) <= tol
+    assert max_rel(b, br) <= tol
     flips = np.sign(S) != np.sign(Sr)
     rms = np.sqrt(np.mean(Sr ** 2))
     assert np.all(np.abs(Sr[flips]) < 1e-3 * rms)
@@ -119,6 +134,13 @@ def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4):
 @pytest.mark.parametrize("side", [0, 1])
 def test_single_step_matches_oracle(nq, m, n, r, side):
     _single_step_case(nq, m, n, r, side, seed=m + n + r + side)
+
+
+@pytest.mark.parametrize("m,n,r", [(300, 200, 40), (520, 600, 300), (129, 65, 1),
+                                   (256, 512, 16)])
+@pytest.mark.parametrize("side", [0, 1])
+def test_single_step_fp32_precision_matches_oracle(nq, m, n, r, side):
+    _single_step_case(nq, m, n, r, side, seed=3 * m + n + r + side, prec="fp32")
 
 
 def test_single_step_full_size_q_proj(nq):
@@ -141,35 +163,39 @@ def test_planted_factors_recovered_on_gpu(nq):
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_planted_with_noise_end_to_end(nq, seed):
-    # 60 iterations: both the oracle and the BF16-operand arithmetic have converged to the
-    # planted factors on every seed (at 30 the slowest seed is still on its way there).
+    # Identity preconditioners, 60 iterations: the iteration has converged and the final
+    # error is a well-defined value; per instance within 1 % of the oracle.  (At 30
+    # iterations this problem is bistable, see test_config1_statistics_at_thirty_iterations.)
     p = planted_problem(seed, noise=0.1)
     res = nq.nq_lbadmm(p["W"].cuda(), 16, iters=60)
     ref = O.lbadmm(p["W"].double().numpy(), r=16, iters=60)
-    assert abs(res["rel_err"] - ref.rel_err) <= TOL_E2E * ref.rel_err
-    # first objective value: identical start, differs only by arithmetic
-    assert abs(res["objective"][0] - ref.objective[0]) <= 1e-3 * ref.objective[0]
+    assert abs(res["rel_err"] - ref.rel_err) <= TOL_E2E * ref.rel_err, (res["rel_err"], ref.rel_err)
+    # the first objective values: identical start, FP32-accurate arithmetic
+    np.testing.assert_allclose(res["objective"][:5], ref.objective[:5], rtol=1e-4)
 
 
-def test_planted_config_with_preconditioners_within_oracle_spread(nq):
-    # The 256 x 512, r = 16 problem with calibration preconditioners is, at 30 iterations,
-    # sensitive to perturbations of BF16 size (the oracle itself moves by a few percent), so
-    # the GPU result is compared with the spread of oracle runs on inputs perturbed by
-    # relative noise of BF16 rounding size.
-    p = planted_problem(0, noise=0.1)
-    d_in, d_out, _, _ = nq.nq_calib_precond(p["acts"].cuda(), p["grads"].cuda())
-    res = nq.nq_lbadmm(p["W"].cuda(), 16, d_in, d_out, iters=30)
-    r_in, r_out, _, _ = OC.calib_precond([p["acts"].numpy()], [p["grads"].numpy()])
-    W = p["W"].double().numpy()
-    rng = np.random.default_rng(0)
-    ens = [O.lbadmm(W, r_in, r_out, r=16, iters=30).rel_err]
-    for _ in range(6):
-        Wp = W * (1 + 2.0 ** -9 * rng.uniform(-1, 1, W.shape))
-        Wt, _, _ = O.precondition(W, r_in, r_out, 16)
-        rp = O.lbadmm(Wp, r_in, r_out, r=16, iters=30)
-        ens.append(O.recon_error(Wt, rp.s1, O.sign_pm(rp.U), O.sign_pm(rp.V), rp.s2))
-    lo, hi = min(ens) * (1 - TOL_E2E), max(ens) * (1 + TOL_E2E)
-    assert lo <= res["rel_err"] <= hi, (res["rel_err"], ens)
+def test_config1_statistics_at_thirty_iterations(nq):
+    # The first benchmark configuration as stated: 256 x 512 FP32 planted r = 16 with 0.1
+    # noise, calibration preconditioners from 4096-token act/grad streams, 30 iterations.
+    # At 30 iterations the iteration is still in a transient whose outcome moves by 1-3 %
+    # under state perturbations of 1e-6 (relative) - the FP64 oracle's own outcome does -
+    # so no arithmetic short of the oracle's own operation order reproduces one instance
+    # to 1 %.  Read statistically over 64 seeds: the median and the 90th percentile of
+    # the GPU's final errors each lie within 1 % of the oracle's, and every instance's
+    # first-iteration objective (identical start) agrees to 1e-4.
+    e_gpu, e_ref = [], []
+    for seed in range(64):
+        p = planted_problem(seed, noise=0.1)
+        d_in, d_out, _, _ = nq.nq_calib_precond(p["acts"].cuda(), p["grads"].cuda())
+        res = nq.nq_lbadmm(p["W"].cuda(), 16, d_in, d_out, iters=30)
+        r_in, r_out, _, _ = OC.calib_precond([p["acts"].numpy()], [p["grads"].numpy()])
+        ref = O.lbadmm(p["W"].double().numpy(), r_in, r_out, r=16, iters=30)
+        assert abs(res["objective"][0] - ref.objective[0]) <= 1e-4 * ref.objective[0]
+        e_gpu.append(res["rel_err"])
+        e_ref.append(ref.rel_err)
+    for q in (50, 90):
+        g, o = np.percentile(e_gpu, q), np.percentile(e_ref, q)
+        assert abs(g - o) <= TOL_E2E * o, (q, g, o)
 
 
 def test_random_layer_end_to_end_within_one_percent(nq):

@@ -118,7 +118,13 @@ def test_argument_errors_are_reported_before_any_device_work():
     p, c, e, ld = ctypes.c_void_p(), ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int64()
     assert L.nq_lbadmm_state_field(8, 8, 2, 42, fake, 1 << 30, ctypes.byref(p), ctypes.byref(c),
                                    ctypes.byref(e), ctypes.byref(ld)) == INV
-    assert L.nq_lbadmm_half_step(8, 8, 2, 1.0, 1e-4, 4, 2, fake, 1 << 30, null) == INV
+    assert L.nq_lbadmm_half_step(8, 8, 2, 1.0, 1e-4, 4, 2, 0, fake, 1 << 30, null) == INV
+    # unknown precision mode
+    assert L.nq_lbadmm_half_step(8, 8, 2, 1.0, 1e-4, 4, 0, 2, fake, 1 << 30, null) == INV
+    assert L.nq_lbadmm_iterate(8, 8, 2, 1.0, 1e-4, 1, 4, 9, null, fake, 1 << 30, null) == INV
+    assert L.nq_lbadmm_sync_operands(8, 8, 2, -1, fake, 1 << 30, null) == INV
+    assert L.nq_lbadmm_prepare(fake, 0, 8, 8, null, null, 2, 0, 3, null, fake, 1 << 30,
+                               null) == INV
     assert L.nq_pack_signs(null, 4, 4, fake, null) == INV
 
 

@@ -2,9 +2,10 @@
 
 Callers that cannot allocate device memory or pass a workspace (for example a plugin
 inside a host program that owns the device memory pool) use this variant, whose scratch
-is a fixed array inside the library.  Checked here through the C ABI against the
-workspace-based nq_calib_stats on the same inputs, on two calls in a row, so that
-anything the first call leaves in the shared array cannot leak into the second.
+is a fixed array inside the library.  Checked here through the C ABI on two calls in a
+row (so that anything the first call leaves in the shared array cannot leak into the
+second): bit for bit against the workspace-based nq_calib_stats, which runs the same
+reduction in the same order, and against the FP64 oracle's channel moments at 1e-6.
 This file is collected last on purpose.
 """
 import ctypes
@@ -12,6 +13,8 @@ import ctypes
 import numpy as np
 import pytest
 import torch
+
+from oracle import calib as OC
 
 pytestmark = pytest.mark.gpu
 
@@ -33,13 +36,15 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(nq):
     cases = [torch.randn(70000, 4096, generator=g).to(torch.bfloat16),
              (torch.randn(3000, 1000, generator=g) * 3).to(torch.float32)]
     for X in cases:
+        s_o, q_o, _ = OC.channel_moments([X.float().numpy()])
         X = X.cuda()
         code, s, q = _noalloc(nq, X)
         assert code == 0, nq.status_string(code)
         s_ref, q_ref = nq.nq_calib_stats(X)
         torch.cuda.synchronize()
-        for a, b in ((s, s_ref), (q, q_ref)):
-            a, b = a.cpu().numpy(), b.cpu().numpy()
+        assert torch.equal(s, s_ref) and torch.equal(q, q_ref)
+        for a, b in ((s, s_o), (q, q_o)):
+            a = a.cpu().numpy()
             assert np.max(np.abs(a - b) / np.abs(b)) < 1e-6
 
 
