@@ -209,6 +209,35 @@ nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,
                         nq_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
+/* 3. Inference with the packed factors.  NanoQuant summary page, "Technical    */
+/* novelty" (技术新颖性) and "Limitations" (局限与改进): the compressed layer     */
+/* is applied by binary GEMV/GEMM kernels that read the packed signs.          */
+/* ------------------------------------------------------------------------- */
+
+/* Batches of at most this many rows take the packed-bit (GEMV) path. */
+#define NQ_BINARY_GEMV_MAX_BATCH 16
+
+/* Workspace bytes of nq_binary_matmul for an m x n layer at rank r and batch B. */
+size_t nq_binary_workspace_size(int64_t m, int64_t n, int32_t r, int64_t B);
+
+/*
+ * Y = X diag(s2) V+- U+-^T diag(s1), i.e. for each of the B input rows x (length n)
+ *     y_i = s1_i sum_k U+-[i][k] sum_j V+-[j][k] s2_j x_j      (i < m)
+ * with U+-, V+- decoded from the packed words of nq_lbadmm (bit 1 = -1, LSB-first).
+ * Apply it to W~-space inputs; for the raw layer pass s1/d_out and s2/d_in as scales.
+ *   U_packed [m][(r+31)/32], V_packed [n][(r+31)/32] (uint32), s1 (m), s2 (n) float,
+ *   X [B][n] (dtype dt, row stride n), Y [B][m] float: all device.
+ * B <= NQ_BINARY_GEMV_MAX_BATCH: SIMT kernels on the packed bits (FP32 sums, fixed
+ * order).  Larger B: the signs are expanded once per call into BF16 +-1 tensor-core
+ * operands in the workspace and both products run as tcgen05 GEMMs with split (hi + lo)
+ * BF16 operands for the scaled inputs, FP32 accumulation.  Enqueue only.
+ */
+nq_status nq_binary_matmul(const uint32_t *U_packed, const uint32_t *V_packed, const float *s1,
+                           const float *s2, int64_t m, int64_t n, int32_t r, const void *X,
+                           nq_dtype dt, int64_t B, float *Y, void *ws, size_t ws_bytes,
+                           nq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
 /* Step-level interface over the ADMM state held in the workspace.             */
 /* nq_lbadmm is nq_lbadmm_prepare + nq_lbadmm_iterate + nq_lbadmm_finish.      */
 /* The state fields can be read and written (checkpoint / resume, tests).      */
@@ -290,7 +319,8 @@ typedef enum {
     NQ_K_FINISH = 9,    /* balancing, scales, packing                                */
     NQ_K_RECON = 10,    /* tcgen05 +-1 reconstruction error                          */
     NQ_K_GINV = 11,     /* tcgen05 G^-1 = L^-T L^-1 (symmetric, split BF16)          */
-    NQ_K_COUNT = 12
+    NQ_K_BINARY = 12,   /* binary GEMV/GEMM on the packed factors                    */
+    NQ_K_COUNT = 13
 } nq_kernel_class;
 
 /* Number of kernel launches the library has issued in this process. */

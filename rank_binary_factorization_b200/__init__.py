@@ -21,7 +21,8 @@ from ._lib import (FIELDS, NQ_BF16, NQ_F32, NQ_PREC_BF16, NQ_PREC_FP32, NQError,
 
 __all__ = [
     "nq_bpw", "nq_rank_for_bpw", "nq_calib_stats", "nq_calib_precond", "nq_lbadmm",
-    "nq_recon_error", "nq_pack_signs", "LBState", "NQError", "status_string", "lib",
+    "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "LBState", "NQError",
+    "status_string", "lib",
     "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
 ]
 
@@ -129,6 +130,22 @@ def nq_recon_error(W, U_packed, V_packed, r, s1, s2, d_in=None, d_out=None, ws=N
         _ptr(W), _dtype(W), m, n, _ptr(d_in), _ptr(d_out), _ptr(U_packed), _ptr(V_packed), r,
         _ptr(s1), _ptr(s2), ctypes.byref(out), _ptr(ws), ws.numel(), _stream()))
     return out.value
+
+
+def nq_binary_matmul(U_packed, V_packed, s1, s2, r, X, ws=None):
+    """Y = X diag(s2) V+- U+-^T diag(s1) for X of shape (B, n) or (n,); returns float32 Y."""
+    _cuda(X, "X")
+    vec = X.dim() == 1
+    X2 = X.unsqueeze(0) if vec else X
+    B, n = X2.shape
+    m = s1.shape[0]
+    need = lib.nq_binary_workspace_size(m, n, r, B)
+    ws = ws if ws is not None else workspace(need, X.device)
+    Y = torch.empty(B, m, dtype=torch.float32, device=X.device)
+    check("nq_binary_matmul", lib.nq_binary_matmul(
+        _ptr(U_packed), _ptr(V_packed), _ptr(s1), _ptr(s2), m, n, r, _ptr(X2), _dtype(X2), B,
+        _ptr(Y), _ptr(ws), ws.numel(), _stream()))
+    return Y[0] if vec else Y
 
 
 def nq_pack_signs(X):

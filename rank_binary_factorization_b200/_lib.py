@@ -45,6 +45,9 @@ SIGNATURES = {
     "nq_recon_error": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp,
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_pack_signs": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_vp]),
+    "nq_binary_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i64]),
+    "nq_binary_matmul": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_vp, c_i32, c_i64,
+                                 c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_prepare": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_u64, c_i32,
                                   c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_iterate": (c_i32, [c_i64, c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_i32, c_vp,
@@ -66,7 +69,7 @@ SIGNATURES = {
 }
 NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
-                  "objective", "finish", "recon", "ginv"]
+                  "objective", "finish", "recon", "ginv", "binary"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

@@ -9,7 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnq.so")
-SOURCES = ["api.cu", "gemm_tc.cu", "kernels.cu", "chol.cu", "calib_noalloc.cu", "selftest.cu"]
+SOURCES = ["api.cu", "gemm_tc.cu", "kernels.cu", "chol.cu", "binary.cu", "calib_noalloc.cu",
+           "selftest.cu"]
 HEADERS = ["common.cuh", "gemm_tc.cuh", "kernels.cuh", "layout.h",
            os.path.join("..", "..", "include", "nq.h")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

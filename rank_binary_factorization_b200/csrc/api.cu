@@ -71,7 +71,7 @@ bool g_prof_on = false;
 // NVTX range names of the kernel classes (nq_kernel_class order)
 const char *const kClassNames[NQ_K_COUNT] = {
     "nq.calib", "nq.calib_finalize", "nq.prep", "nq.gram", "nq.chol", "nq.rhs",
-    "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv"};
+    "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv", "nq.binary"};
 
 // Scope of one kernel class's launches: an NVTX range on the host timeline (seen by
 // profilers; inert otherwise) and, when recording is on, a CUDA event pair on the stream.
@@ -186,6 +186,41 @@ nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s
     return NQ_OK;
 }
 
+// ---- side stream of the r x r factorisation ---------------------------------------
+// Per host thread and device: a library-owned stream on which the Cholesky + inverse and
+// the G^-1 GEMM of a half step run beside the RHS GEMM, and the two events that fork it
+// from, and join it back into, the caller's stream.  Created by the first call of a host
+// thread on a device; never destroyed (they live until the process exits).
+struct SideCtx {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+nq_status side_ctx(SideCtx **out) {
+    thread_local SideCtx ctx[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return NQ_ERR_CUDA;
+    SideCtx &c = ctx[dev];
+    if (!c.side) {
+        NQ_CK(cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking));
+        NQ_CK(cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming));
+        NQ_CK(cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming));
+    }
+    *out = &c;
+    return NQ_OK;
+}
+
+// CTAs given to the factorisation while the RHS GEMM runs on the others (0: no overlap,
+// the factorisation takes the whole GPU before the GEMM).  Overlap pays only when the
+// factorisation on a fraction of the SMs is about as short as the GEMM; measured on
+// B200 it is not yet (r = 1000: 305 us on 148 CTAs, 522 us on 23 CTAs, against a
+// ~100 us GEMM), so the factorisation keeps the whole GPU.
+int chol_ctas(int32_t r, int sms) {
+    (void)r;
+    (void)sms;
+    return 0;
+}
+
 // ---- LB-ADMM internals ------------------------------------------------------------
 struct Lb {
     LbLayout L;
@@ -236,7 +271,18 @@ nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s)
     ep.out = lb.p<float>(L.g[other]);
     ep.ldo = L.r;
     ep.diag = diag;
+    // few tiles (small r): split K so that the (tile, part) units fill the SMs; the parts
+    // are summed in a fixed order by gram_reduce
+    const int S = gram_ksplit(L.r, K, nseg, device_sm_count());
     ProfScope ps(NQ_K_GRAM, s);
+    if (S > 1) {
+        ep.ksplit = S;
+        ep.out = lb.p<float>(L.gpart);
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
+        NQ_CK(gram_reduce(lb.p<float>(L.gpart), gram_tiles(L.r), S, L.r, diag,
+                          lb.p<float>(L.g[other]), s));
+        return NQ_OK;
+    }
     NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
     return NQ_OK;
 }
@@ -249,15 +295,28 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     const int BN = pick_bn(L.r);
     nq_status st = lb_gram(lb, other, lambda + rho, prec, s);
     if (st) return st;
+    // The factorisation of G and the G^-1 GEMM depend only on the Gram; the RHS GEMM only
+    // on the other side's operand and this side's dual state.  With overlap they run at
+    // once: the factorisation on ``cc`` CTAs of a side stream, the RHS GEMM on the rest.
+    const int sms = device_sm_count();
+    const int cc = chol_ctas(L.r, sms);
+    SideCtx *sc = nullptr;
+    if (cc > 0 && (st = side_ctx(&sc))) return st;
+    cudaStream_t fs = s;   // stream of the factorisation
+    if (cc > 0) {
+        NQ_CK(cudaEventRecord(sc->fork, s));
+        NQ_CK(cudaStreamWaitEvent(sc->side, sc->fork, 0));
+        fs = sc->side;
+    }
     {
-        ProfScope ps(NQ_K_CHOL, s);
+        ProfScope ps(NQ_K_CHOL, fs);
         NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
-                           &lb.sc->err, lb.sc->bar, s));
+                           &lb.sc->err, lb.sc->bar, cc, fs));
     }
     {
-        ProfScope ps(NQ_K_GINV, s);
+        ProfScope ps(NQ_K_GINV, fs);
         // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo; G^-1 is
         // symmetric, so only its lower-triangular tiles are computed and mirrored
         tc::Maps maps;
@@ -279,12 +338,14 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
         ep.tri_k = 1;
         ep.sym = 1;
+        ep.max_ctas = cc;
         ep.err = &lb.sc->err;
         ep.Rhi = lb.p<__nv_bfloat16>(L.gih);
         ep.Rlo = lb.p<__nv_bfloat16>(L.gil);
         ep.ldr = L.ldr;
-        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, s));
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, fs));
     }
+    if (cc > 0) NQ_CK(cudaEventRecord(sc->join, fs));
 
     // R = W^ X_other + rho (Z - L), split into hi + lo bf16.  FP32-accurate mode: both
     // operands split, three passes [W^_hi, W^_lo, W^_hi] . [X_hi, X_hi, X_lo].
@@ -316,9 +377,11 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ep.Rhi = lb.p<__nv_bfloat16>(L.rhi);
         ep.Rlo = lb.p<__nv_bfloat16>(L.rlo);
         ep.ldr = L.ldr;
+        ep.max_ctas = cc > 0 ? sms - cc : 0;
         ProfScope ps(NQ_K_RHS, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RHS, BN, s));
     }
+    if (cc > 0) NQ_CK(cudaStreamWaitEvent(s, sc->join, 0));
     // X = R G^-1 = [R_hi, R_lo, R_hi] [Gi_hi; Gi_hi; Gi_lo]; S <- X + L; Xt = bf16(X)^T
     {
         tc::Maps maps;
@@ -732,6 +795,94 @@ nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const
     NQ_CK(recon_finalize(part, (int)tc::num_tiles((int)m, (int)n, BN), sc, &sc->recon2, s));
     NQ_CK(cudaMemcpyAsync(rel_err, &sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
     return read_err(&sc->err, s, false);
+}
+
+static bool binary_args_ok(int64_t m, int64_t n, int32_t r, int64_t B) {
+    return m >= 1 && n >= 1 && m <= kMaxDim && n <= kMaxDim && r >= 1 && r <= kMaxRank &&
+           B >= 1 && B <= kMaxDim;
+}
+
+size_t nq_binary_workspace_size(int64_t m, int64_t n, int32_t r, int64_t B) {
+    if (!binary_args_ok(m, n, r, B)) return 0;
+    BinLayout L;
+    L.build(m, n, r, B, NQ_BINARY_GEMV_MAX_BATCH, bin_gemv_chunks(n, r, B));
+    return L.total;
+}
+
+nq_status nq_binary_matmul(const uint32_t *U_packed, const uint32_t *V_packed, const float *s1,
+                           const float *s2, int64_t m, int64_t n, int32_t r, const void *X,
+                           nq_dtype dt, int64_t B, float *Y, void *ws, size_t ws_bytes,
+                           nq_stream_t stream) {
+    if (!U_packed || !V_packed || !s1 || !s2 || !X || !Y || (dt != NQ_F32 && dt != NQ_BF16) ||
+        !binary_args_ok(m, n, r, B))
+        return NQ_ERR_INVALID_ARG;
+    BinLayout L;
+    L.build(m, n, r, B, NQ_BINARY_GEMV_MAX_BATCH, bin_gemv_chunks(n, r, B));
+    nq_status st = check_ws(ws, ws_bytes, L.total);
+    if (st) return st;
+    if ((st = check_device())) return st;
+    cudaStream_t s = cs(stream);
+    const int xb = dt == NQ_BF16;
+    Scalars *sc = at<Scalars>(ws, L.scal);
+    ProfScope ps(NQ_K_BINARY, s);
+    if (B <= NQ_BINARY_GEMV_MAX_BATCH) {
+        NQ_CK(bin_gemv(U_packed, V_packed, s1, s2, m, n, r, X, xb, B, Y, at<float>(ws, L.P),
+                       at<float>(ws, L.z), s));
+        return NQ_OK;
+    }
+    __nv_bfloat16 *vh = at<__nv_bfloat16>(ws, L.vh), *vl = at<__nv_bfloat16>(ws, L.vl),
+                  *um = at<__nv_bfloat16>(ws, L.um), *xh = at<__nv_bfloat16>(ws, L.xh),
+                  *xl = at<__nv_bfloat16>(ws, L.xl), *zh = at<__nv_bfloat16>(ws, L.zh),
+                  *zl = at<__nv_bfloat16>(ws, L.zl);
+    NQ_CK(cudaMemsetAsync(sc, 0, sizeof(Scalars), s));
+    NQ_CK(bin_expand(U_packed, V_packed, s2, m, n, r, X, xb, B, vh, vl, L.ldt, um, L.ldr, xh, xl,
+                     L.ldt, s));
+    // Z = X diag(s2) V+- (B x r) with split operands, written as BF16 hi + lo
+    {
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int nseg = xb ? 2 : 3;
+        const void *as[3] = {xh, xb ? xh : xl, xh}, *bs[3] = {vh, xb ? vl : vh, vl};
+        const int BN = pick_bn(r);
+        for (int g = 0; g < nseg; ++g)
+            if (!tc::make_map_bf16(&maps.a[g], as[g], B, n, L.ldt, tc::BM) ||
+                !tc::make_map_bf16(&maps.b[g], bs[g], r, n, L.ldt, BN))
+                return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = (int)B;
+        ep.N = r;
+        ep.nseg = nseg;
+        for (int g = 0; g < nseg; ++g) ep.kblocks[g] = (int)ceil_div(n, tc::BK);
+        ep.err = &sc->err;
+        ep.Rhi = zh;
+        ep.Rlo = zl;
+        ep.ldr = L.ldr;
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BN, s));
+    }
+    // Y = (Z_hi + Z_lo) U+-^T diag(s1) (B x m)
+    {
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int BN = pick_bn(m);
+        if (!tc::make_map_bf16(&maps.a[0], zh, B, r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[1], zl, B, r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[0], um, m, r, L.ldr, BN) ||
+            !tc::make_map_bf16(&maps.b[1], um, m, r, L.ldr, BN))
+            return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = (int)B;
+        ep.N = (int)m;
+        ep.nseg = 2;
+        ep.kblocks[0] = ep.kblocks[1] = (int)ceil_div(r, tc::BK);
+        ep.err = &sc->err;
+        ep.out = Y;
+        ep.ldo = m;
+        ep.s1 = s1;
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SCALE, BN, s));
+    }
+    return NQ_OK;
 }
 
 nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,

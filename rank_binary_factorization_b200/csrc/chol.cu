@@ -85,12 +85,11 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ int blk_a0() { return (threadIdx.x >> 4) * 4; }
 __device__ __forceinline__ int blk_b0() { return (threadIdx.x & 15) * 4; }
 
-// acc[i][j] += sum_{c in [c0, c1)} XT[c][a0+i] * Y[c][b0+j]
-__device__ __forceinline__ void mac(float (&acc)[4][4], const Tile &XT, const Tile &Y,
-                                   int c0 = 0, int c1 = TB) {
+// acc[i][j] += sum_c XT[c][a0+i] * Y[c][b0+j]
+__device__ __forceinline__ void mac(float (&acc)[4][4], const Tile &XT, const Tile &Y) {
     const int a0 = blk_a0(), b0 = blk_b0();
 #pragma unroll 4
-    for (int c = c0; c < c1; ++c) {
+    for (int c = 0; c < TB; ++c) {
         const float4 x = *reinterpret_cast<const float4 *>(&XT[c][a0]);
         const float4 y = *reinterpret_cast<const float4 *>(&Y[c][b0]);
         const float xs[4] = {x.x, x.y, x.z, x.w};
@@ -166,16 +165,33 @@ __device__ __forceinline__ void put_t(float *M, int64_t ld, int ti, int tj,
 // 16b + l + 32).  Column k's multipliers of the block's diagonal rows are broadcast by
 // shuffles; every lane also keeps the 16 diagonal entries of the block and updates them
 // from those broadcasts, so the next pivot needs no shuffle.  rdiag[c] = 1 / L_cc.
-__device__ void chol_tile(Tile &s, float *rdiag, int *err) {
+// With FUSE the tile's pending rank-64 update s -= P P^T (P: natural layout) is folded
+// into the block-column updates (only the lower triangle is ever formed; measured slower
+// than a separate register-blocked product, so the chain does not use it).  Only the
+// lower triangle of s is read or written; its upper part keeps whatever it held, except
+// inside the 16 x 16 diagonal blocks, which are zero above the diagonal afterwards.
+template <bool FUSE>
+__device__ void chol_tile(Tile &s, const Tile &P, float *rdiag, int *err) {
     const int t = threadIdx.x, lane = t & 31;
     bool bad = false;
 #pragma unroll 1
     for (int b = 0; b < 4; ++b) {
         const int c0 = 16 * b;
-        if (b > 0) {
+        if (FUSE || b > 0) {
             const int c = c0 + (t & 15);
             for (int i = c0 + (t >> 4); i < TB; i += 16) {
                 float acc = 0.f;
+                if (FUSE) {
+#pragma unroll 4
+                    for (int m = 0; m < TB; m += 4) {
+                        const float4 x = *reinterpret_cast<const float4 *>(&P[i][m]);
+                        const float4 y = *reinterpret_cast<const float4 *>(&P[c][m]);
+                        acc = fmaf(x.x, y.x, acc);
+                        acc = fmaf(x.y, y.y, acc);
+                        acc = fmaf(x.z, y.z, acc);
+                        acc = fmaf(x.w, y.w, acc);
+                    }
+                }
                 for (int m = 0; m < c0; m += 4) {
                     const float4 x = *reinterpret_cast<const float4 *>(&s[i][m]);
                     const float4 y = *reinterpret_cast<const float4 *>(&s[c][m]);
@@ -199,12 +215,9 @@ __device__ void chol_tile(Tile &s, float *rdiag, int *err) {
             }
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                float piv = d[k];
-                if (!(piv > 0.f)) {
-                    bad = true;
-                    piv = 1e-30f;
-                }
-                const float il = rsqrtf(piv);
+                // a non-positive pivot is recorded and replaced, without a branch
+                bad |= !(d[k] > 0.f);
+                const float il = rsqrtf(fmaxf(d[k], 1e-30f));
                 if (lane == 0) rdiag[c0 + k] = il;
                 const float l0 = a0[k] * il, l1 = a1[k] * il;
                 a0[k] = l0;
@@ -225,12 +238,7 @@ __device__ void chol_tile(Tile &s, float *rdiag, int *err) {
         }
         __syncthreads();
     }
-    for (int e = t; e < TB * TB; e += blockDim.x) {
-        const int i = e >> 6, c = e & 63;
-        if (i < (c & ~15)) s[i][c] = 0.f;
-    }
     if (bad) raise_error(err, NQ_ERR_NOT_SPD);
-    __syncthreads();
 }
 
 // ---- inverse of a lower-triangular 64 x 64 tile ------------------------------------
@@ -278,8 +286,14 @@ __device__ __forceinline__ void inv_level(const Tile &s, Tile &li, Tile &tmp) {
 
 __device__ void inverse_tile(const Tile &s, const float *rdiag, Tile &li, Tile &lit, Tile &tmp) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    for (int e = t; e < TB * TB; e += blockDim.x) li[e >> 6][e & 63] = 0.f;
-    __syncthreads();
+    if (warp >= 4) {  // zero the six 16 x 16 blocks above the diagonal blocks
+        for (int e = t - 128; e < 6 * 256; e += 128) {
+            const int blk = e >> 8, w = e & 255;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);           // (0,1..3), (1,2..3), (2,3)
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            li[16 * bi + (w >> 4)][16 * bj + (w & 15)] = 0.f;
+        }
+    }
     if (warp < 4 && lane < 16) {  // diagonal 16 x 16 blocks: column `lane` of each inverse
         const int o = 16 * warp;
         float x[16];
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
         // t2: L_jj, t3: L_jj^-1, t4: (L_jj^-1)^T, t0: panel operand, t1: panel^T
         load_n(t2, p.A, rp, 0, 0);
         __syncthreads();
-        chol_tile(t2, rdiag, p.err);
+        chol_tile<false>(t2, t1, rdiag, p.err);
         inverse_tile(t2, rdiag, t3, t4, t1);
         store_n(p.A, rp, 0, 0, t2);
         store_n(p.Li, rp, 0, 0, t3);
@@ -409,7 +423,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                     for (int q = 0; q < 4; ++q) t2[a0 + i][b0 + q] -= acc[i][q];
             }
             __syncthreads();
-            chol_tile(t2, rdiag, p.err);
+            chol_tile<false>(t2, t1, rdiag, p.err);
             inverse_tile(t2, rdiag, t3, t4, t1);
             store_n(p.A, rp, j + 1, j + 1, t2);
             store_n(p.Li, rp, j + 1, j + 1, t3);
@@ -620,7 +634,8 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
 
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
-                         unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s) {
+                         unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
+                         cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
     constexpr int smem = (5 * TB * LDS + TB) * sizeof(float);
     // grid of the cooperative launch (one CTA per SM), per device
@@ -640,6 +655,7 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
         if (grid < 3) return cudaErrorLaunchOutOfResources;
         grids[dev].store(grid);
     }
+    if (max_ctas > 0 && max_ctas < grid) grid = max_ctas < 3 ? 3 : max_ctas;
     cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
     const int nb = (int)(rp / TB);

@@ -186,6 +186,9 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
             for (int j = 0; j < 16; ++j)
                 if (full || col0 + j < p.N) o[j] = w[j];
         }
+    } else if constexpr (EPI == EPI_SCALE) {
+        float *o = p.out + (int64_t)row * p.ldo + col0;
+        for (int j = 0; j < 16 && col0 + j < p.N; ++j) o[j] = v[j] * p.s1[col0 + j];
     } else if constexpr (EPI == EPI_SPLIT) {
         __nv_bfloat16 *hi = p.Rhi + (int64_t)row * p.ldr + col0;
         __nv_bfloat16 *lo = p.Rlo + (int64_t)row * p.ldr + col0;
@@ -367,6 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_tiles = p.sym ? num_m * (num_m + 1) / 2 : num_m * (int)ceil_div(p.N, BN);
     const int total_kb = p.kblocks[0] + (p.nseg > 1 ? p.kblocks[1] : 0) +
                          (p.nseg > 2 ? p.kblocks[2] : 0);
+    // split-K: work unit u = (split u / num_tiles, tile u % num_tiles); split s covers the
+    // k-blocks [s * kchunk, (s + 1) * kchunk) of the concatenated segments
+    const int ksplit = p.ksplit > 1 ? p.ksplit : 1;
+    const int num_units = num_tiles * ksplit;
+    const int kchunk = (total_kb + ksplit - 1) / ksplit;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -396,10 +404,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // TMA producer
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+                const int tile = unit % num_tiles, ks = unit / num_tiles;
+                const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
                 int m0, n0;
                 tile_origin<BN>(p, tile, num_m, m0, n0);
-                for (int kb = 0; kb < total_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     int seg = 0, k = kb;
                     while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
                     if (p.tri_k && k < (m0 > n0 ? m0 : n0) / BK) continue;
@@ -424,7 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             int lt = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+            for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x, ++lt) {
+                const int tile = unit % num_tiles, ks = unit / num_tiles;
+                const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
                 const int as = lt & 1;
                 int m0, n0;
                 tile_origin<BN>(p, tile, num_m, m0, n0);
@@ -432,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(as * BN);
                 bool first = true;
-                for (int kb = 0; kb < total_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (p.tri_k) {
                         int seg = 0, k = kb;
                         while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
@@ -463,7 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         int lt = 0;
         bool dead = false;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+        for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++lt) {
+            const int tile = unit % num_tiles;
             const int as = lt & 1;
             int m0, n0;
             tile_origin<BN>(p, tile, num_m, m0, n0);
@@ -484,7 +497,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BN; c += 16) {
                     float v[16];
                     tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
-                    if (row < p.M && n0 + c < p.N) {
+                    if (EPI == EPI_GRAM && ksplit > 1) {
+                        // split-K partial: the unit's raw 128 x 128 tile, reduced later
+                        st16(p.out + ((int64_t)unit * BM + 32 * q + lane) * BM + c, v);
+                    } else if (row < p.M && n0 + c < p.N) {
                         epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
                         if constexpr (EPI == EPI_SPLIT)
                             if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
@@ -561,8 +577,9 @@ static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s
     if (e != cudaSuccess) return e;
     int sms = device_sm_count();
     if (p.max_ctas > 0 && p.max_ctas < sms) sms = p.max_ctas;
-    const int64_t tiles = p.sym ? ceil_div(p.M, BM) * (ceil_div(p.M, BM) + 1) / 2
-                                : num_tiles(p.M, p.N, BN);
+    const int64_t tiles = (p.sym ? ceil_div(p.M, BM) * (ceil_div(p.M, BM) + 1) / 2
+                                 : num_tiles(p.M, p.N, BN)) *
+                          (p.ksplit > 1 ? p.ksplit : 1);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
     kern<<<grid, kThreads, smem, s>>>(maps, p);
     count_launch();
@@ -587,6 +604,7 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_SOLVE: return launch_bn<EPI_SOLVE>(maps, p, BN, s);
         case EPI_RECON: return launch_bn<EPI_RECON>(maps, p, BN, s);
         case EPI_SPLIT: return launch_bn<EPI_SPLIT>(maps, p, BN, s);
+        case EPI_SCALE: return launch_bn<EPI_SCALE>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
 }

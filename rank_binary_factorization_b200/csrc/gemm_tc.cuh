@@ -24,7 +24,8 @@ constexpr int A_TILE_BYTES = BM * BK * 2;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
-enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4 };
+enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4,
+                 EPI_SCALE = 5 };
 
 struct Maps {
     CUtensorMap a[3];
@@ -40,6 +41,10 @@ struct EpiParams {
                         // triangular tiles only, each off-diagonal tile also written mirrored
     int max_ctas;       // 0: one CTA per SM; else at most this many CTAs (SMs left free for
                         // kernels running beside this one on another stream)
+    int ksplit;         // EPI_GRAM only: > 1 splits the K range into ksplit parts; unit u
+                        // (tile u % T, part u / T) writes its raw 128 x 128 tile to
+                        // out + u * 128 * 128 (row-major, ld 128) for a later reduction.
+                        // Every part must get at least one k-block.
     int *err;
     // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
     float *out;
@@ -62,6 +67,7 @@ struct EpiParams {
     int64_t ldxt;
     int objective;             // also sum (R - rho (2Z - S_old)) . X into part[tile]
     double *part;              // per-tile partial sums (EPI_SOLVE objective, EPI_RECON)
+    // EPI_SCALE: out[row * ldo + col] = acc * s1[col]
     // EPI_RECON: sum_ij (d_out_i W_ij d_in_j - s1_i acc s2_j)^2
     const void *W;
     int w_bf16;

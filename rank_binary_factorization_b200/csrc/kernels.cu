@@ -488,48 +488,80 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 // steps from b = 1.  One pass over S per power step: t = |S| b row by row and
 // b' = |S|^T t / ||t|| column by column, from the same shared-memory copy of S.
 // =================================================================================
-// One CTA tile = kSvidRows rows of |S| staged in shared memory with 16-byte loads; warp w
+// Each CTA stages tiles of rows of S in shared memory (16-byte cp.async copies); warp w
 // forms the row dot t_w = |S_w.| b, then every thread accumulates its columns' share of
-// |S|^T t.  Small tiles keep several CTAs per SM in flight (the loads of one overlap the
-// arithmetic of another).  Partial sums per CTA go to partb / partn (fixed order).
+// |S|^T t.  Partial sums per CTA go to partb / partn (fixed order).
+// Each CTA walks its tiles of ROWS rows with a two-buffer cp.async ring, so the copy of
+// the next tile overlaps the arithmetic on the current one.
+__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(float *dst, const float *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+
+template <int ROWS>
 __global__ void __launch_bounds__(256)
-    svid_pass_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
-                     const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
-                     double *partn) {
+    svid_pass2_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
+                      const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
+                      double *partn) {
     extern __shared__ __align__(16) float sm[];
-    float *sA = sm;                      // kSvidRows x ldf
-    float *sb = sm + kSvidRows * ldf;    // r
-    __shared__ float st[kSvidRows];
-    __shared__ double sn[kSvidRows];
+    float *sb = sm + 2 * ROWS * ldf;     // b (r)
+    __shared__ float st[ROWS];
+    __shared__ double sn[ROWS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int k = threadIdx.x; k < r; k += blockDim.x) sb[k] = b_in ? b_in[k] : 1.f;
     float acc[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) acc[u] = 0.f;
     double nacc = 0.0;
-    const int r4 = r >> 2;
-    const int64_t ntile = ceil_div(rows, kSvidRows);
-    for (int64_t tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
-        const int64_t row0 = tile * kSvidRows;
-        __syncthreads();
-        // rows x r4 float4 loads, then the scalar tail
-        for (int e = threadIdx.x; e < kSvidRows * r4; e += blockDim.x) {
+    const int r4 = r >> 2, rt = r - 4 * r4;
+    const int64_t ntile = ceil_div(rows, ROWS);
+    // copy tile `tile` (ROWS rows of S, zero rows past the end) into buffer `buf`
+    auto issue = [&](int64_t tile, float *buf) {
+        const int64_t row0 = tile * ROWS;
+        for (int e = threadIdx.x; e < ROWS * r4; e += blockDim.x) {
             const int w = e / r4, k4 = e - w * r4;
             const int64_t i = row0 + w;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < rows) v = __ldcg(reinterpret_cast<const float4 *>(S + i * ldf) + k4);
-            *reinterpret_cast<float4 *>(sA + w * ldf + 4 * k4) =
-                make_float4(fabsf(v.x), fabsf(v.y), fabsf(v.z), fabsf(v.w));
+            float *dst = buf + w * ldf + 4 * k4;
+            if (i < rows)
+                cp_async16(dst, S + i * ldf + 4 * k4);
+            else
+                *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int e = threadIdx.x; e < kSvidRows * (r - 4 * r4); e += blockDim.x) {
-            const int w = e / (r - 4 * r4), k = 4 * r4 + e % (r - 4 * r4);
+        for (int e = threadIdx.x; e < ROWS * rt; e += blockDim.x) {
+            const int w = e / rt, k = 4 * r4 + e % rt;
             const int64_t i = row0 + w;
-            sA[w * ldf + k] = i < rows ? fabsf(S[i * ldf + k]) : 0.f;
+            if (i < rows)
+                cp_async4(buf + w * ldf + k, S + i * ldf + k);
+            else
+                buf[w * ldf + k] = 0.f;
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int64_t tile = blockIdx.x;
+    if (tile < ntile) issue(tile, sm);
+    int cur = 0;
+    for (; tile < ntile; tile += gridDim.x, cur ^= 1) {
+        float *bc = sm + cur * ROWS * ldf;
+        const int64_t next = tile + gridDim.x;
+        if (next < ntile) {
+            issue(next, sm + (cur ^ 1) * ROWS * ldf);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
-        if (warp < kSvidRows) {
+        const int64_t row0 = tile * ROWS;
+        if (warp < ROWS) {
             float t = 0.f;
-            for (int k = lane; k < r; k += 32) t = fmaf(sA[warp * ldf + k], sb[k], t);
+            for (int k = lane; k < r; k += 32) t = fmaf(fabsf(bc[warp * ldf + k]), sb[k], t);
             t = warp_sum(t);
             if (lane == 0) {
                 st[warp] = t;
@@ -544,21 +576,22 @@ __global__ void __launch_bounds__(256)
             if (k < r) {
                 float v = 0.f;
 #pragma unroll
-                for (int w = 0; w < kSvidRows; ++w) v = fmaf(sA[w * ldf + k], st[w], v);
+                for (int w = 0; w < ROWS; ++w) v = fmaf(fabsf(bc[w * ldf + k]), st[w], v);
                 acc[u] += v;
             }
         }
+        __syncthreads();   // bc may be refilled by the next-but-one tile's copy
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
         const int k = threadIdx.x + 256 * u;
         if (k < r) partb[(int64_t)blockIdx.x * r + k] = acc[u];
     }
-    if (lane == 0 && warp < kSvidRows) sn[warp] = nacc;
+    if (lane == 0 && warp < ROWS) sn[warp] = nacc;
     __syncthreads();
     if (threadIdx.x == 0) {
         double v = 0.0;
-        for (int w = 0; w < kSvidRows; ++w) v += sn[w];
+        for (int w = 0; w < ROWS; ++w) v += sn[w];
         partn[blockIdx.x] = v;
     }
 }
@@ -604,16 +637,21 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
-                 float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
-                 cudaStream_t s) {
-    const size_t smem = (size_t)(kSvidRows * ldf + r) * sizeof(float);
+// Rows per pipelined tile: two buffers of ROWS x ldf floats stay near 64 KB, so that
+// several CTAs fit on an SM.
+static int svid_tile_rows(int64_t ldf) { return ldf <= 1024 ? 8 : (ldf <= 2048 ? 4 : 2); }
+
+template <int ROWS>
+static cudaError_t svid_passes(const float *S, int64_t rows, int32_t r, int64_t ldf, int K,
+                               int nsv, float *bcur, float *tvec, float *partb, double *partn,
+                               float *a, float *b, cudaStream_t s) {
+    const size_t smem = (size_t)(2 * ROWS * ldf + r) * sizeof(float);
     // largest dynamic shared-memory limit set so far, per device
     static std::atomic<size_t> configured[kMaxDevices];
     const int dev = current_device();
     if (dev < 0) return cudaErrorInvalidDevice;
     if (smem > 48 * 1024 && smem > configured[dev].load()) {
-        cudaError_t e = cudaFuncSetAttribute(svid_pass_kernel,
+        cudaError_t e = cudaFuncSetAttribute(svid_pass2_kernel<ROWS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
@@ -621,17 +659,73 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
         while (prev < smem && !configured[dev].compare_exchange_weak(prev, smem)) {
         }
     }
+    // two CTAs per SM (the partial arrays hold nsv >= this many rows)
+    int64_t grid = ceil_div(rows, ROWS);
+    const int64_t cap = 2 * (int64_t)device_sm_count();
+    if (grid > cap) grid = cap;
+    if (grid > nsv) grid = nsv;
     for (int pass = 1; pass <= K; ++pass) {
         const float *b_in = pass == 1 ? nullptr : bcur + (size_t)((pass - 1) & 1) * r;
         const bool last = pass == K;
         float *b_out = last ? b : bcur + (size_t)(pass & 1) * r;
-        svid_pass_kernel<<<nsv, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec, last ? 1 : 0, partb,
-                                                partn);
+        svid_pass2_kernel<ROWS><<<(unsigned)grid, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec,
+                                                                 last ? 1 : 0, partb, partn);
         count_launch();
         svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 256, 0, s>>>(
-            partb, partn, nsv, r, rows, last ? 1 : 0, tvec, b_out, a);
+            partb, partn, (int)grid, r, rows, last ? 1 : 0, tvec, b_out, a);
         count_launch();
     }
+    return cudaGetLastError();
+}
+
+cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
+                 float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
+                 cudaStream_t s) {
+    switch (svid_tile_rows(ldf)) {
+        case 8: return svid_passes<8>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
+        case 4: return svid_passes<4>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
+        default: return svid_passes<2>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
+    }
+}
+
+// =================================================================================
+// Split-K Gram: G = sum over the parts of the raw 128 x 128 tiles + diag I, mirrored.
+// Unit u = part * T + t of the partial array holds lower-triangular tile t (row by row:
+// (0,0), (1,0), (1,1), ...) of one K part.  Parts are summed in index order, so the
+// result does not depend on the order in which the GEMM's CTAs finished.
+// =================================================================================
+__global__ void __launch_bounds__(256)
+    gram_reduce_kernel(const float *__restrict__ P, int T, int S, int r, float diag, float *G) {
+    __shared__ float tr[32][33];
+    const int t = blockIdx.x;
+    int a = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((a + 1) * (a + 2) / 2 <= t) ++a;
+    while (a * (a + 1) / 2 > t) --a;
+    const int b = t - a * (a + 1) / 2;
+    const int m0 = a * 128, n0 = b * 128;
+    const int si = (blockIdx.y >> 2) * 32, sj = (blockIdx.y & 3) * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int k = ty; k < 32; k += 8) {
+        const int li = si + k, lj = sj + tx;
+        float v = 0.f;
+        for (int sp = 0; sp < S; ++sp) v += P[((int64_t)(sp * T + t) * 128 + li) * 128 + lj];
+        const int gi = m0 + li, gj = n0 + lj;
+        if (gi == gj) v += diag;
+        if (gi < r && gj < r) G[(int64_t)gi * r + gj] = v;
+        tr[k][tx] = v;
+    }
+    if (a != b) {
+        __syncthreads();
+        for (int k = ty; k < 32; k += 8) {
+            const int gi = n0 + sj + k, gj = m0 + si + tx;   // mirror of tile entry (si+tx, sj+k)
+            if (gi < r && gj < r) G[(int64_t)gi * r + gj] = tr[tx][k];
+        }
+    }
+}
+
+cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G, cudaStream_t s) {
+    gram_reduce_kernel<<<dim3((unsigned)T, 16), 256, 0, s>>>(P, T, S, r, diag, G);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -47,15 +47,38 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 // ---- Cholesky + inverse (cooperative, FP32) -------------------------------------
 // G = L L^T for the SPD r x r matrix G (row stride r); writes (L^-1)^T as hi + lo bf16
 // [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: 2 (rp/64)^2 counters.
+// max_ctas > 0 limits the cooperative grid (at least 3 CTAs); 0: one CTA per SM.
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *LiT_hi, __nv_bfloat16 *LiT_lo, int64_t ldr,
-                         unsigned int *flags, int *err, unsigned int *bar, cudaStream_t s);
+                         unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
+                         cudaStream_t s);
 
 // ---- SVID -------------------------------------------------------------------------
 // K power steps on |S| (S rows x r, row stride ldf): a = t/||t||, b = A^T t / ||t||.
 cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
                  float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
                  cudaStream_t s);
+
+// ---- inference with the packed factors (binary.cu) --------------------------------
+// Row chunks of the GEMV path's z pass (partials: chunks x B x r floats).
+int bin_gemv_chunks(int64_t n, int32_t r, int64_t B);
+// Y = X diag(s2) V+- U+-^T diag(s1) for B <= NQ_BINARY_GEMV_MAX_BATCH on the packed bits;
+// P: partials, z: B x r floats.
+cudaError_t bin_gemv(const uint32_t *Up, const uint32_t *Vp, const float *s1, const float *s2,
+                     int64_t m, int64_t n, int32_t r, const void *X, int x_bf16, int64_t B,
+                     float *Y, float *P, float *z, cudaStream_t s);
+// Tensor-path operands: Vt hi/lo [r][ldt] (scaled signs of V), Um [m][ldr] (+-1), X split
+// into BF16 hi (and lo for FP32 X) rows of stride ldx.
+cudaError_t bin_expand(const uint32_t *Up, const uint32_t *Vp, const float *s2, int64_t m,
+                       int64_t n, int32_t r, const void *X, int x_bf16, int64_t B,
+                       __nv_bfloat16 *Vh, __nv_bfloat16 *Vl, int64_t ldt, __nv_bfloat16 *Um,
+                       int64_t ldr, __nv_bfloat16 *Xh, __nv_bfloat16 *Xl, int64_t ldx,
+                       cudaStream_t s);
+
+// ---- split-K Gram reduction ------------------------------------------------------
+// G (r x r) = sum_{s < S} P[s * T + t] (raw 128 x 128 lower-triangular tiles t < T) +
+// diag I, each off-diagonal tile also stored mirrored.
+cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G, cudaStream_t s);
 
 // ---- objective --------------------------------------------------------------------
 // obj[slot] = (what_n2 - 2 sum(px) + <GU - cI, GV - cI>) / what_n2

@@ -13,6 +13,25 @@ constexpr int kSvidCtas = 4 * 148;     // CTAs of an SVID pass (4 per SM)
 constexpr int kRedBlocks = 592;       // CTAs of grid-stride reduction kernels (4 per SM)
 constexpr int kObjRing = 4096;        // per-iteration objective slots kept on the device
 constexpr int kMaxRank = 4096;
+constexpr int kGramMaxUnits = 2 * 148;  // split-K Gram: most (tile, part) work units
+
+// Lower-triangular 128 x 128 tiles of an r x r Gram.
+inline int gram_tiles(int32_t r) {
+    const int nm = (r + 127) / 128;
+    return nm * (nm + 1) / 2;
+}
+// Split-K parts of a Gram over K rows (nseg concatenated K segments) on ``sms`` SMs: enough
+// (tile, part) units to fill the SMs, at most 8 parts, at least 8 k-blocks of 64 per part.
+inline int gram_ksplit(int32_t r, int64_t K, int nseg, int sms) {
+    const int T = gram_tiles(r);
+    if (T >= sms) return 1;
+    int S = sms / T;
+    if (S > 8) S = 8;
+    const int64_t kb = nseg * ((K + 63) / 64);
+    if (S > kb / 8) S = (int)(kb / 8);
+    if (S * T > kGramMaxUnits) S = kGramMaxUnits / T;
+    return S < 1 ? 1 : S;
+}
 constexpr int64_t kMaxDim = 65536;
 
 // Scalars block at the start of every workspace.
@@ -38,7 +57,7 @@ struct LbLayout {
     size_t scal = 0, what = 0, whatT = 0, whatL = 0, whatTL = 0, x[2] = {0, 0}, s[2] = {0, 0},
            a[2] = {0, 0}, b[2] = {0, 0}, xt[2] = {0, 0}, xtl[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
            gih = 0, gil = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
-           partb = 0, obj = 0, total = 0;
+           partb = 0, obj = 0, gpart = 0, total = 0;
     size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
 
     int64_t rows(int side) const { return side == 0 ? m : n; }
@@ -101,6 +120,9 @@ struct LbLayout {
         partg = take((size_t)kRedBlocks * 8); // Gram dot-product partials
         partb = take((size_t)2 * nsv * r * 4);  // column partials (SVID; U and V norms)
         obj = take((size_t)kObjRing * 4);
+        // split-K Gram partial tiles (128 x 128 FP32 per unit)
+        const int gu = gram_tiles(r) * 8 < kGramMaxUnits ? gram_tiles(r) * 8 : kGramMaxUnits;
+        gpart = take((size_t)gu * 128 * 128 * 4);
         total = off;
     }
 };
@@ -124,6 +146,38 @@ struct CalibLayout {
         pq = take((size_t)nslab * C * 8);
         s = take((size_t)C * 8);
         q = take((size_t)C * 8);
+        total = off;
+    }
+};
+
+// Workspace of nq_binary_matmul.  B <= gemv_max: partials of the z pass (chunks x B x r)
+// and z (B x r); larger B: the expanded tensor-core operands.
+struct BinLayout {
+    int64_t ldt = 0, ldr = 0;   // leading dims (elements) of the n- and r-long BF16 rows
+    size_t scal = 0, P = 0, z = 0, vh = 0, vl = 0, um = 0, xh = 0, xl = 0, zh = 0, zl = 0,
+           total = 0;
+    void build(int64_t m, int64_t n, int32_t r, int64_t B, int gemv_max, int chunks) {
+        ldt = (n + 7) / 8 * 8;
+        ldr = (r + 7) / 8 * 8;
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off = align_up(off + bytes);
+            return o;
+        };
+        scal = take(sizeof(Scalars));
+        if (B <= gemv_max) {
+            P = take((size_t)chunks * B * r * 4);
+            z = take((size_t)B * r * 4);
+        } else {
+            vh = take((size_t)r * ldt * 2);
+            vl = take((size_t)r * ldt * 2);
+            um = take((size_t)m * ldr * 2);
+            xh = take((size_t)B * ldt * 2);
+            xl = take((size_t)B * ldt * 2);
+            zh = take((size_t)B * ldr * 2);
+            zl = take((size_t)B * ldr * 2);
+        }
         total = off;
     }
 };
