@@ -15,8 +15,10 @@
 //     (j+2, j+2)); CTAs 2.. take the other panel tiles and the trailing updates
 //     round-robin in a topological order, so every wait ends;
 //   * the 64 x 64 tile Cholesky works in 16-column blocks factored by one warp with
-//     shuffles (no CTA barrier per column); the tile inverse takes 16 x 16 diagonal blocks
-//     in four warps at once and two doubling levels;
+//     shuffles (no CTA barrier per column); while that warp sweeps a block, three warps
+//     prepare the next block's update (including its share of the look-ahead update) and
+//     four warps invert the blocks already finished, so the tile's inverse and update
+//     cost little beyond the column sweeps;
 //   * L^-1 in the same dataflow: block column m is a forward substitution advanced one
 //     block row per factorisation step (X_jm = -L_jj^-1 sum_k L_jk X_km), so the inverse
 //     trails the factorisation instead of following it;
@@ -85,22 +87,6 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ int blk_a0() { return (threadIdx.x >> 4) * 4; }
 __device__ __forceinline__ int blk_b0() { return (threadIdx.x & 15) * 4; }
 
-// acc[i][j] += sum_c XT[c][a0+i] * Y[c][b0+j]
-__device__ __forceinline__ void mac(float (&acc)[4][4], const Tile &XT, const Tile &Y) {
-    const int a0 = blk_a0(), b0 = blk_b0();
-#pragma unroll 4
-    for (int c = 0; c < TB; ++c) {
-        const float4 x = *reinterpret_cast<const float4 *>(&XT[c][a0]);
-        const float4 y = *reinterpret_cast<const float4 *>(&Y[c][b0]);
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-        const float ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xs[i], ys[j], acc[i][j]);
-    }
-}
-
 // acc[i][j] += sum_c X[a0+i][c] * Y[c][b0+j]  (both tiles in plain layout)
 __device__ __forceinline__ void mac_n(float (&acc)[4][4], const Tile &X, const Tile &Y) {
     const int a0 = blk_a0(), b0 = blk_b0();
@@ -159,52 +145,103 @@ __device__ __forceinline__ void put_t(float *M, int64_t ld, int ti, int tj,
                make_float4(acc[0][q], acc[1][q], acc[2][q], acc[3][q]));
 }
 
-// ---- 64 x 64 tile Cholesky: four 16-column blocks -----------------------------------
-// Block b: all threads subtract the finished columns from block column b (rows 16b ..
-// 63), then warp 0 factors it column by column (lane l holds rows 16b + l and
-// 16b + l + 32).  Column k's multipliers of the block's diagonal rows are broadcast by
-// shuffles; every lane also keeps the 16 diagonal entries of the block and updates them
-// from those broadcasts, so the next pivot needs no shuffle.  rdiag[c] = 1 / L_cc.
-// With FUSE the tile's pending rank-64 update s -= P P^T (P: natural layout) is folded
-// into the block-column updates (only the lower triangle is ever formed; measured slower
-// than a separate register-blocked product, so the chain does not use it).  Only the
-// lower triangle of s is read or written; its upper part keeps whatever it held, except
-// inside the 16 x 16 diagonal blocks, which are zero above the diagonal afterwards.
+// ---- the chain CTA's tile step: factorisation, look-ahead update and inverse ----------
+// The column sweep of a 16-column block (warp 0) is a latency chain; the update of the
+// next block column that does not depend on the block being swept - including its share
+// of the pending rank-64 update with the panel P when FUSE - is formed meanwhile by warps
+// 1-3 and 5-7 (warps share an SM sub-partition by warp % 4, so warp 4 stays idle and
+// leaves warp 0's sub-partition to it).  After the sweeps, L^-1 is formed block-wise in
+// four levels by all warps and lit = li^T.
+//   warp 0        factors block b column by column (lane l holds rows 16b + l and
+//                 16b + l + 32; column k's multipliers are broadcast by shuffles; every
+//                 lane tracks the block's diagonal, so the next pivot needs no shuffle; a
+//                 non-positive pivot is recorded and replaced, without a branch);
+//   warps 1-3,5-7 sum_m P[i][m] P[c][m] + sum over finished blocks < b of s[i][m] s[c][m]
+//                 for block b+1's entries (four pairs at a time), then, after the sweep,
+//                 block b's share, and store block b+1's updated columns.
+// s: the tile (lower triangle read; L on return); P: the panel L_{j+1,j} in natural layout
+// (FUSE only); tmp: scratch of the inverse's block products.
+// Warp-level 16 x 16 x 16 product c (+)= A_blk B_blk: lane = row (lane & 15), 8 columns.
+__device__ __forceinline__ void blk_acc(float (&c)[8], const Tile &A, int ar, int ac,
+                                        const Tile &B, int br, int bc) {
+    const int lane = threadIdx.x & 31, row = lane & 15, col0 = (lane >> 4) * 8;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float a = A[ar + row][ac + k];
+        const float4 y0 = *reinterpret_cast<const float4 *>(&B[br + k][bc + col0]);
+        const float4 y1 = *reinterpret_cast<const float4 *>(&B[br + k][bc + col0 + 4]);
+        c[0] = fmaf(a, y0.x, c[0]);
+        c[1] = fmaf(a, y0.y, c[1]);
+        c[2] = fmaf(a, y0.z, c[2]);
+        c[3] = fmaf(a, y0.w, c[3]);
+        c[4] = fmaf(a, y1.x, c[4]);
+        c[5] = fmaf(a, y1.y, c[5]);
+        c[6] = fmaf(a, y1.z, c[6]);
+        c[7] = fmaf(a, y1.w, c[7]);
+    }
+}
+
+__device__ __forceinline__ void blk_store(Tile &D, int dr, int dc, const float (&c)[8], float sgn) {
+    const int lane = threadIdx.x & 31, row = lane & 15, col0 = (lane >> 4) * 8;
+    *reinterpret_cast<float4 *>(&D[dr + row][dc + col0]) =
+        make_float4(sgn * c[0], sgn * c[1], sgn * c[2], sgn * c[3]);
+    *reinterpret_cast<float4 *>(&D[dr + row][dc + col0 + 4]) =
+        make_float4(sgn * c[4], sgn * c[5], sgn * c[6], sgn * c[7]);
+}
+
+// Dot products of four (row i_u, row c_u) pairs over columns [m0, m1) of one tile, summed
+// into acc[u] (four independent chains).
+__device__ __forceinline__ void dot4(float (&acc)[4], const Tile &X, const int (&i)[4],
+                                     const int (&c)[4], int m0, int m1) {
+#pragma unroll 2
+    for (int m = m0; m < m1; m += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float4 x = *reinterpret_cast<const float4 *>(&X[i[u]][m]);
+            const float4 y = *reinterpret_cast<const float4 *>(&X[c[u]][m]);
+            acc[u] = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc[u]))));
+        }
+    }
+}
+
 template <bool FUSE>
-__device__ void chol_tile(Tile &s, const Tile &P, float *rdiag, int *err) {
-    const int t = threadIdx.x, lane = t & 31;
+__device__ void chain_tile(Tile &s, const Tile &P, float *rdiag, Tile &li, Tile &lit, Tile &tmp,
+                           int *err) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // update workers: warps 1-3 and 5-7, thread index tw in [0, 192)
+    const bool upd = warp != 0 && warp != 4;
+    const int tw = (warp < 4 ? warp - 1 : warp - 2) * 32 + lane;
     bool bad = false;
+    // block 0's share of the pending update, by all warps: pairs (i, c), i < 64, c < 16
+    if (FUSE) {
+        int ii[4], cc[4];
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int pr = u * 256 + t;
+            ii[u] = pr >> 4;
+            cc[u] = pr & 15;
+        }
+        dot4(acc, P, ii, cc, 0, TB);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s[ii[u]][cc[u]] -= acc[u];
+    }
+    __syncthreads();
 #pragma unroll 1
     for (int b = 0; b < 4; ++b) {
         const int c0 = 16 * b;
-        if (FUSE || b > 0) {
-            const int c = c0 + (t & 15);
-            for (int i = c0 + (t >> 4); i < TB; i += 16) {
-                float acc = 0.f;
-                if (FUSE) {
-#pragma unroll 4
-                    for (int m = 0; m < TB; m += 4) {
-                        const float4 x = *reinterpret_cast<const float4 *>(&P[i][m]);
-                        const float4 y = *reinterpret_cast<const float4 *>(&P[c][m]);
-                        acc = fmaf(x.x, y.x, acc);
-                        acc = fmaf(x.y, y.y, acc);
-                        acc = fmaf(x.z, y.z, acc);
-                        acc = fmaf(x.w, y.w, acc);
-                    }
-                }
-                for (int m = 0; m < c0; m += 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(&s[i][m]);
-                    const float4 y = *reinterpret_cast<const float4 *>(&s[c][m]);
-                    acc = fmaf(x.x, y.x, acc);
-                    acc = fmaf(x.y, y.y, acc);
-                    acc = fmaf(x.z, y.z, acc);
-                    acc = fmaf(x.w, y.w, acc);
-                }
-                s[i][c] -= acc;
-            }
-            __syncthreads();
+        // block b+1's pairs: (i, c), i in [c0+16, 64), c in [c0+16, c0+32); pair
+        // pr = u * 192 + tw, u < 4 (pairs past np are clamped onto a valid one, not stored)
+        const int np = (48 - c0) * 16;
+        int ii[4], cc[4];
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int pr = min(u * 192 + tw, np - 1);
+            ii[u] = c0 + 16 + (pr >> 4);
+            cc[u] = c0 + 16 + (pr & 15);
         }
-        if (t < 32) {
+        if (warp == 0) {
             const int r0 = c0 + lane, r1 = r0 + 32;
             float a0[16], a1[16], d[16];
 #pragma unroll
@@ -215,7 +252,6 @@ __device__ void chol_tile(Tile &s, const Tile &P, float *rdiag, int *err) {
             }
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                // a non-positive pivot is recorded and replaced, without a branch
                 bad |= !(d[k] > 0.f);
                 const float il = rsqrtf(fmaxf(d[k], 1e-30f));
                 if (lane == 0) rdiag[c0 + k] = il;
@@ -235,66 +271,24 @@ __device__ void chol_tile(Tile &s, const Tile &P, float *rdiag, int *err) {
                 if (r0 < TB) s[r0][c0 + c] = (lane >= c) ? a0[c] : 0.f;
                 if (r1 < TB) s[r1][c0 + c] = a1[c];
             }
+        } else if (upd && b < 3) {
+            if (FUSE) dot4(part, P, ii, cc, 0, TB);
+            dot4(part, s, ii, cc, 0, c0);
         }
         __syncthreads();
-    }
-    if (bad) raise_error(err, NQ_ERR_NOT_SPD);
-}
-
-// ---- inverse of a lower-triangular 64 x 64 tile ------------------------------------
-// li = L^-1 (plain, zero above the diagonal), lit = (L^-1)^T.  The four 16 x 16 diagonal
-// blocks are inverted by four warps at once (lane = column, forward substitution with the
-// reciprocal diagonal rdiag); two doubling levels then form the off-diagonal blocks,
-// Li21 = -Li22 (L21 Li11), with tmp as scratch.
-template <int H>
-__device__ __forceinline__ void inv_level(const Tile &s, Tile &li, Tile &tmp) {
-    // thread job: one pair pr, one row a, four columns b .. b+3; entries above the
-    // diagonal of li are zero, so the K loops run over the full block (no predicates)
-    constexpr int NP = TB / (2 * H), G = H / 4;
-    for (int e = threadIdx.x; e < NP * H * G; e += blockDim.x) {  // tmp = L21 Li11
-        const int pr = e / (H * G), a = (e / G) % H, b = 4 * (e % G), o = 2 * H * pr;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (b < 3) {
+            if (upd) {   // block b's share; store block b+1's columns
+                dot4(part, s, ii, cc, c0, c0 + 16);
 #pragma unroll
-        for (int c = 0; c < H; ++c) {
-            const float l = s[o + H + a][o + c];
-            const float4 y = *reinterpret_cast<const float4 *>(&li[o + c][o + b]);
-            acc.x = fmaf(l, y.x, acc.x);
-            acc.y = fmaf(l, y.y, acc.y);
-            acc.z = fmaf(l, y.z, acc.z);
-            acc.w = fmaf(l, y.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(&tmp[o + a][b]) = acc;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < NP * H * G; e += blockDim.x) {  // Li21 = -Li22 tmp
-        const int pr = e / (H * G), a = (e / G) % H, b = 4 * (e % G), o = 2 * H * pr;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < H; ++c) {
-            const float l = li[o + H + a][o + H + c];
-            const float4 y = *reinterpret_cast<const float4 *>(&tmp[o + c][b]);
-            acc.x = fmaf(l, y.x, acc.x);
-            acc.y = fmaf(l, y.y, acc.y);
-            acc.z = fmaf(l, y.z, acc.z);
-            acc.w = fmaf(l, y.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(&li[o + H + a][o + b]) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-    __syncthreads();
-}
-
-__device__ void inverse_tile(const Tile &s, const float *rdiag, Tile &li, Tile &lit, Tile &tmp) {
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    if (warp >= 4) {  // zero the six 16 x 16 blocks above the diagonal blocks
-        for (int e = t - 128; e < 6 * 256; e += 128) {
-            const int blk = e >> 8, w = e & 255;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);           // (0,1..3), (1,2..3), (2,3)
-            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            li[16 * bi + (w >> 4)][16 * bj + (w & 15)] = 0.f;
+                for (int u = 0; u < 4; ++u)
+                    if (u * 192 + tw < np) s[ii[u]][cc[u]] -= part[u];
+            }
+            __syncthreads();
         }
     }
-    if (warp < 4 && lane < 16) {  // diagonal 16 x 16 blocks: column `lane` of each inverse
+    // L^-1 by 16 x 16 blocks: X_aa by forward substitution, then
+    // X_ak = -X_aa sum_{l=k}^{a-1} L_al X_lk by distance a - k = 1, 2, 3
+    if (warp < 4 && lane < 16) {
         const int o = 16 * warp;
         float x[16];
 #pragma unroll
@@ -307,15 +301,38 @@ __device__ void inverse_tile(const Tile &s, const float *rdiag, Tile &li, Tile &
         }
 #pragma unroll
         for (int k = 0; k < 16; ++k) li[o + k][o + lane] = x[k];
+    } else if (warp >= 4) {   // zero the six blocks above the diagonal blocks
+        for (int e = t - 128; e < 6 * 256; e += 128) {
+            const int blk = e >> 8, q = e & 255;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);           // (0,1..3), (1,2..3), (2,3)
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            li[16 * bi + (q >> 4)][16 * bj + (q & 15)] = 0.f;
+        }
     }
     __syncthreads();
-    inv_level<16>(s, li, tmp);
-    inv_level<32>(s, li, tmp);
+#pragma unroll 1
+    for (int dist = 1; dist < 4; ++dist) {
+        const int a = dist + warp, k = warp;   // warp w < 4 - dist: block (dist + w, w)
+        const bool act = warp < 4 - dist;
+        if (act) {
+            float c[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int l = k; l < a; ++l) blk_acc(c, s, 16 * a, 16 * l, li, 16 * l, 16 * k);
+            blk_store(tmp, 16 * a, 16 * k, c, 1.f);
+        }
+        __syncthreads();
+        if (act) {
+            float c[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            blk_acc(c, li, 16 * a, 16 * a, tmp, 16 * a, 16 * k);
+            blk_store(li, 16 * a, 16 * k, c, -1.f);
+        }
+        __syncthreads();
+    }
     for (int e = t; e < TB * TB; e += blockDim.x) {
         const int c = e >> 6, b = e & 63;
         lit[b][c] = li[c][b];
     }
     __syncthreads();
+    if (bad) raise_error(err, NQ_ERR_NOT_SPD);
 }
 
 // lower-triangular enumeration idx -> (ii >= kk)
@@ -386,8 +403,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
         // t2: L_jj, t3: L_jj^-1, t4: (L_jj^-1)^T, t0: panel operand, t1: panel^T
         load_n(t2, p.A, rp, 0, 0);
         __syncthreads();
-        chol_tile<false>(t2, t1, rdiag, p.err);
-        inverse_tile(t2, rdiag, t3, t4, t1);
+        chain_tile<false>(t2, t1, rdiag, t3, t4, t0, p.err);
         store_n(p.A, rp, 0, 0, t2);
         store_n(p.Li, rp, 0, 0, t3);
         if (nb > 1) store_n(p.Li, rp, 0, 1, t4);      // L_00^-T in an unused upper tile
@@ -407,24 +423,15 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
                 const int a0 = blk_a0(), b0 = blk_b0();
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) t1[b0 + q][a0 + i] = acc[i][q];
+                    *reinterpret_cast<float4 *>(&t1[a0 + i][b0]) =
+                        make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
             }
             signal_count(CNT(j + 1, j), 1);
             cp_async_wait<0>();
             __syncthreads();
-            zero(acc);
-            mac(acc, t1, t1);                          // L_{j+1,j} L_{j+1,j}^T
-            {
-                const int a0 = blk_a0(), b0 = blk_b0();
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) t2[a0 + i][b0 + q] -= acc[i][q];
-            }
-            __syncthreads();
-            chol_tile<false>(t2, t1, rdiag, p.err);
-            inverse_tile(t2, rdiag, t3, t4, t1);
+            // factorisation of the next diagonal tile with its look-ahead update
+            // t2 -= L_{j+1,j} L_{j+1,j}^T and its inverse, in one pass
+            chain_tile<true>(t2, t1, rdiag, t3, t4, t0, p.err);
             store_n(p.A, rp, j + 1, j + 1, t2);
             store_n(p.Li, rp, j + 1, j + 1, t3);
             if (j + 2 < nb) store_n(p.Li, rp, j + 1, j + 2, t4);  // L^-T, unused upper tile
