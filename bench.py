@@ -189,6 +189,47 @@ def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
                 share_of_step=None, peak_kind=peak_kind)
 
 
+def time_binary_matmul(nq, res, m, n, r, peaks, reps=10):
+    """Device time of nq_binary_matmul on the packed result: batch 1 (packed-bit GEMV path)
+    and batch 256 (tensor-core path, sign expansion included).  L2 is flushed before each
+    timed call (the packed factors of a layer fit in L2)."""
+    import torch
+    flush = torch.empty(320 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    nw = (r + 31) // 32
+    out = {}
+    for B in (1, 256):
+        X = torch.randn(B, n, device="cuda").to(torch.bfloat16)
+        ws = nq.workspace(nq.lib.nq_binary_workspace_size(m, n, r, B))
+        for _ in range(3):
+            nq.nq_binary_matmul(res["U_packed"], res["V_packed"], res["s1"], res["s2"], r, X, ws=ws)
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            nq.nq_binary_matmul(res["U_packed"], res["V_packed"], res["s1"], res["s2"], r, X, ws=ws)
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1) / 1e3
+        t = tot / reps
+        if B == 1:
+            # packed signs + scales + input + output, bytes that must come from HBM
+            nbytes = (m + n) * nw * 4 + (m + n) * 4 + n * 2 + m * 4
+            gbs = nbytes / t / 1e9
+            out["gemv"] = dict(batch=1, us=round(t * 1e6, 2), bytes=nbytes, gbs=round(gbs, 1),
+                               frac_hbm=round(gbs / peaks["hbm_gbs"], 4))
+        else:
+            flops = 2.0 * B * (n * r + r * m)   # the two products
+            tf = flops / t / 1e12
+            out["gemm"] = dict(batch=B, us=round(t * 1e6, 2), flops=flops, tflops=round(tf, 2),
+                               frac_bf16=round(tf / peaks["bf16_tflops"], 4),
+                               note="per call, including the expansion of the signs into "
+                                    "BF16 operands; products run with split operands")
+    del flush
+    return out
+
+
 # ---------------------------------------------------------------------------------------
 # oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------------------
@@ -411,6 +452,8 @@ def run_ours(args):
         e2e=dict(value=round(world * iters * e2e_steps / t_e2e, 3), unit=UNIT,
                  h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h)),
         rel_err=res["rel_err"])
+    if not args.no_binary:
+        line["binary_matmul"] = time_binary_matmul(nq, res, m, n, r, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_sample(W_h, acts_h, grads_h, r, iters, T)
         info["value"] = round(v, 5)
@@ -432,6 +475,8 @@ def main():
     ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-binary", action="store_true",
+                    help="skip the timing of nq_binary_matmul on the packed result")
     ap.add_argument("--workload", choices=["gate_proj", "q_proj", "profile", "q_proj_profile"],
                     default="gate_proj",
                     help="gate_proj (default): the 11008x4096 Llama-2-7B gate/up shape at "

@@ -166,7 +166,8 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  *     S = U + L_U;  A = |S|;  b = 1;  K times { a = A b / ||A b||;  b = A^T a }
  *     Z_U = sign(S) * a b^T;   L_U = L_U + U - Z_U
  *     the same for V with W^^T and U
- *     objective[t] = ||W^ - U V^T||_F^2 / ||W^||_F^2
+ *     objective[t] = ||W^ - U V^T||_F^2 / ||W^||_F^2   (of W^ and the latents as the
+ *                    tensor-core operands hold them: BF16, or split BF16 for FP32)
  *   g_k = sqrt(||V_:k|| / ||U_:k||);  U_:k *= g_k;  V_:k /= g_k
  *   s1_i = gamma mean_k |U_ik|,  s2_j = mean_k |V_jk|
  *   sign bit = (latent < 0), LSB-first along k, row-major uint32[rows][(r+31)/32]

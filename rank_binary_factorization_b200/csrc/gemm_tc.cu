@@ -265,18 +265,19 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
                 bad |= !isfinite(x);
                 const float z = sgn(so[j]) * ai * bb[j];
                 sn[j] = x + so[j] - z;
-                if (p.objective) part += (rr[j] - p.rho * (2.f * z - so[j])) * x;
+                // the latent as the next contractions see it: bf16(x) (+ its low part)
+                const __nv_bfloat16 h = __float2bfloat16_rn(x);
+                float xo = __bfloat162float(h);
+                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = h;
+                if (p.XtL) {
+                    const __nv_bfloat16 l = __float2bfloat16_rn(x - xo);
+                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] = l;
+                    xo += __bfloat162float(l);
+                }
+                if (p.objective) part += (rr[j] - p.rho * (2.f * z - so[j])) * xo;
             }
             st16(Xrow, v);
             st16(Srow, sn);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-                p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = h;
-                if (p.XtL)
-                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] =
-                        __float2bfloat16_rn(v[j] - __bfloat162float(h));
-            }
         } else {
             for (int j = 0; j < 16 && col0 + j < p.N; ++j) {
                 const float x = v[j];
@@ -286,14 +287,17 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
                 Xrow[j] = x;
                 Srow[j] = x + sold - z;
                 const __nv_bfloat16 h = __float2bfloat16_rn(x);
+                float xo = __bfloat162float(h);
                 p.Xt[(int64_t)(col0 + j) * p.ldxt + row] = h;
-                if (p.XtL)
-                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] =
-                        __float2bfloat16_rn(x - __bfloat162float(h));
+                if (p.XtL) {
+                    const __nv_bfloat16 l = __float2bfloat16_rn(x - xo);
+                    p.XtL[(int64_t)(col0 + j) * p.ldxt + row] = l;
+                    xo += __bfloat162float(l);
+                }
                 if (p.objective) {
                     const int64_t o = (int64_t)row * p.ldr + col0 + j;
                     const float r = __bfloat162float(p.Rhi[o]) + __bfloat162float(p.Rlo[o]);
-                    part += (r - p.rho * (2.f * z - sold)) * x;
+                    part += (r - p.rho * (2.f * z - sold)) * xo;
                 }
             }
         }

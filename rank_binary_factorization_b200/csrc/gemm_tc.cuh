@@ -61,7 +61,9 @@ struct EpiParams {
     __nv_bfloat16 *Rhi, *Rlo;  // [M][ldr]
     int64_t ldr;
     // EPI_SOLVE: X = acc; S <- X + S - sign(S) a b^T; Xt[col][row] = bf16(X) and, when XtL
-    // is set, XtL[col][row] = bf16(X - Xt) (the low part of a split-BF16 operand)
+    // is set, XtL[col][row] = bf16(X - Xt) (the low part of a split-BF16 operand).  The
+    // objective partial takes X as the operands hold it (Xt, + XtL), so that it belongs
+    // to the same latents as the Grams of the operands.
     float *X;                  // [M][ldf]
     __nv_bfloat16 *Xt, *XtL;   // [N][ldxt]
     int64_t ldxt;

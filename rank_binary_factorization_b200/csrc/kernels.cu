@@ -732,7 +732,9 @@ cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *
 // =================================================================================
 // Objective ||W^ - U V^T||^2 / ||W^||^2 = (||W^||^2 - 2 <W^^T U, V> + <U^T U, V^T V>)
 // / ||W^||^2 from by-products: <W^^T U, V> from the V-step epilogue, the Gram
-// matrices (less the ridge) of both steps.
+// matrices (less the ridge) of both steps.  All three terms are of the latents as the
+// tensor-core operands hold them (BF16, or split BF16 at NQ_PREC_FP32), so the identity
+// is exact for those matrices and only accumulation rounding enters the difference.
 // =================================================================================
 __global__ void __launch_bounds__(256)
     gram_dot_kernel(const float *__restrict__ GU, const float *__restrict__ GV, int r, float c,

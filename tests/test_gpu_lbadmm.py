@@ -124,6 +124,12 @@ def _single_step_case(nq, m, n, r, side, seed, rho=1.0, lam=1e-4, K=4, prec="bf1
     flips = np.sign(S) != np.sign(Sr)
     rms = np.sqrt(np.mean(Sr ** 2))
     assert np.all(np.abs(Sr[flips]) < 1e-3 * rms)
+    # normal-equation residual of the GPU's solve: ||X G - R|| / ||R|| with the exact
+    # G = Y^T Y + (lambda + rho) I and R of these inputs (the solve's own accuracy)
+    G = Y.T @ Y + (lam + rho) * np.eye(r)
+    R = A @ Y + rho * (Z - Lam)
+    resid = float(np.linalg.norm(X @ G - R) / np.linalg.norm(R))
+    assert resid <= 1e-4, resid
     # the transposed BF16 operand the other side will read
     xt_ref = bf16_exact(Xr)
     return max_rel(X, Xr), st, xt_ref
@@ -141,6 +147,15 @@ def test_single_step_matches_oracle(nq, m, n, r, side):
 @pytest.mark.parametrize("side", [0, 1])
 def test_single_step_fp32_precision_matches_oracle(nq, m, n, r, side):
     _single_step_case(nq, m, n, r, side, seed=3 * m + n + r + side, prec="fp32")
+
+
+@pytest.mark.parametrize("m,n,r", [(11008, 4096, 1000), (8192, 8192, 4080), (28672, 8192, 3488)])
+@pytest.mark.parametrize("side", [0, 1])
+def test_single_step_large_shapes(nq, m, n, r, side):
+    # the 11008 x 4096 r = 1000 target layer, config 5's largest rank (64 Cholesky block
+    # steps) and config 4's 70B gate/up shape (non-square, r = 3488)
+    err, _, _ = _single_step_case(nq, m, n, r, side, seed=m + r + side)
+    assert err < TOL_STEP
 
 
 def test_single_step_full_size_q_proj(nq):
@@ -292,3 +307,111 @@ def test_full_size_q_proj_pipeline_properties(nq):
                            d_in, d_out)
     assert abs(e2 - e) <= 1e-5 * e
     assert torch.all(res["s1"] > 0) and torch.all(res["s2"] > 0)
+
+
+def _late_state(m, n, r, seed, eps, cast):
+    """A state late in a run: W^ = c (A B^T + eps sqrt(r) N) with ||W^|| = 2 sqrt(r) (the
+    library's normalisation), latents U = sqrt(c) A, V = sqrt(c) B (U V^T fits W^ up to
+    the noise, a relative residual of about eps^2), S = latent + 0.05 N, positive a, b."""
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((m, r))
+    B = rng.standard_normal((n, r))
+    M = A @ B.T + eps * np.sqrt(r) * rng.standard_normal((m, n))
+    c = 2 * np.sqrt(r) / np.linalg.norm(M)
+    Wh = cast(c * M)
+    U, V = cast(np.sqrt(c) * A).astype(np.float64), cast(np.sqrt(c) * B).astype(np.float64)
+    SU = (U + 0.05 * rng.standard_normal((m, r))).astype(np.float32)
+    SV = (V + 0.05 * rng.standard_normal((n, r))).astype(np.float32)
+    aU, aV = [np.abs(rng.standard_normal(k)).astype(np.float32) / np.sqrt(k) for k in (m, n)]
+    bU, bV = [0.1 * np.abs(rng.standard_normal(r)).astype(np.float32) for _ in range(2)]
+    return Wh, U, V, SU, aU, bU, SV, aV, bV
+
+
+def _oracle_iteration(Wh, U, V, SU, aU, bU, SV, aV, bV, rho=1.0, lam=1e-4, operand=None):
+    """The U and V steps of one iteration from the loaded state; ``operand`` (if given)
+    rounds U before the V step takes it as its contraction operand, as the BF16 mode
+    defines it."""
+    W = Wh.astype(np.float64)
+    ZU = O.sign_pm(SU) * np.outer(aU, bU)
+    LU = SU.astype(np.float64) - ZU
+    ZV = O.sign_pm(SV) * np.outer(aV, bV)
+    LV = SV.astype(np.float64) - ZV
+    U1, _, _, _ = O.latent_update(W, V, ZU, LU, rho, lam)
+    if operand is not None:
+        U1 = operand(U1).astype(np.float64)
+    V1, _, _, _ = O.latent_update(W.T, U1, ZV, LV, rho, lam)
+    return U1, V1
+
+
+@pytest.mark.parametrize("prec,m,n,r,eps", [("fp32", 2048, 2048, 1008, 0.05),
+                                            ("bf16", 4096, 4096, 2032, 0.05),
+                                            ("bf16", 4096, 4096, 2032, 0.3)])
+def test_objective_on_identical_late_state(nq, prec, m, n, r, eps):
+    # The per-iteration objective (||W^||^2 - 2 <W^T U, V> + <U^T U, V^T V>) / ||W^||^2
+    # subtracts terms near ||W^||^2 when the residual is small (eps = 0.05: ~6e-4 after
+    # one step).  From an identical late state (rho = 1e-3, so that the step fits W^):
+    # one iteration on the GPU, then its objective (i) against the explicit residual of
+    # W^ and the GPU's U, V as its operands hold them (BF16-rounded in the BF16 mode):
+    # 1e-4 relative, the formula's own accuracy; (ii) against the oracle's iteration
+    # from the same state, with the latents rounded where the BF16 mode rounds them:
+    # 1e-3 relative.
+    rho, lam = 1e-3, 1e-4
+    cast = bf16_exact if prec == "bf16" else (lambda a: np.asarray(a, dtype=np.float32))
+    Wh, U, V, SU, aU, bU, SV, aV, bV = _late_state(m, n, r, 5, eps, cast)
+    st = nq.LBState(m, n, r, prec=prec)
+    # prepare on W^ itself: ||W^|| = 2 sqrt(r), so gamma = 1 and W^ and its norm are
+    # formed as they will be loaded
+    Wt = torch.from_numpy(Wh).to(torch.bfloat16 if prec == "bf16" else torch.float32)
+    st.prepare(Wt.cuda(), seed=0)
+    _load_state(st, m, n, r, Wh, U, V, SU, aU, bU, SV, aV, bV)
+    obj = st.iterate(1, rho=rho, lam=lam)[0]
+    assert st.check_device_error() == 0
+    U1 = st.field("U")[:, :r].cpu().double().numpy()
+    V1 = st.field("V")[:, :r].cpu().double().numpy()
+    Wd = Wh.astype(np.float64)
+    op = bf16_exact if prec == "bf16" else (lambda a: a)
+    explicit = O.relative_residual(Wd, op(U1).astype(np.float64), op(V1).astype(np.float64))
+    assert abs(obj - explicit) <= 1e-4 * explicit, (obj, explicit)
+    U1r, V1r = _oracle_iteration(Wh, U, V, SU, aU, bU, SV, aV, bV, rho=rho, lam=lam,
+                                 operand=bf16_exact if prec == "bf16" else None)
+    ref = O.relative_residual(Wd, U1r, op(V1r).astype(np.float64))
+    assert abs(obj - ref) <= 1e-3 * ref, (obj, ref)
+
+
+@pytest.mark.parametrize("m,n,r", [(300, 500, 40), (4096, 4096, 2032), (777, 1000, 33)])
+def test_finish_scales_and_bits_on_loaded_latents(nq, m, n, r):
+    # balancing, scale extraction and packing on identical latents: s1, s2 within 1e-5 of
+    # the oracle, packed words bit for bit
+    rng = np.random.default_rng(m + r)
+    W = torch.randn(m, n, generator=torch.Generator().manual_seed(r)) * 0.02
+    st = nq.LBState(m, n, r, prec="fp32")
+    gamma = st.prepare(W.cuda(), seed=0)
+    U = (rng.standard_normal((m, r)) * np.exp(rng.standard_normal(r))).astype(np.float32)
+    V = (rng.standard_normal((n, r)) * np.exp(rng.standard_normal(r))).astype(np.float32)
+    U[3, 5 % r] = 0.0
+    st.field("U")[:, :r].copy_(torch.from_numpy(U).cuda())
+    st.field("V")[:, :r].copy_(torch.from_numpy(V).cuda())
+    res = st.finish(W.cuda())
+    Ub, Vb, _ = O.balance(U.astype(np.float64), V.astype(np.float64))
+    s1, s2 = O.extract_scales(Ub, Vb, gamma)
+    assert max_rel(res["s1"].cpu().numpy(), s1) <= 1e-5
+    assert max_rel(res["s2"].cpu().numpy(), s2) <= 1e-5
+    np.testing.assert_array_equal(res["U_packed"].cpu().numpy().view(np.uint32), O.pack_signs(Ub))
+    np.testing.assert_array_equal(res["V_packed"].cpu().numpy().view(np.uint32), O.pack_signs(Vb))
+    Wt, _, _ = O.precondition(W.double().numpy(), None, None, r)
+    ref = O.recon_error(Wt, s1, O.sign_pm(Ub), O.sign_pm(Vb), s2)
+    assert abs(res["rel_err"] - ref) <= 1e-5 * ref
+
+
+@pytest.mark.parametrize("shape,r,seed", [((4, 4), 1, 0), ((4, 4), 2, 1), ((6, 6), 1, 2),
+                                          ((6, 6), 2, 3), ((6, 6), 2, 4)])
+def test_brute_force_lower_bounds_the_gpu_result(nq, shape, r, seed):
+    # Exhaustive search over every sign pattern with least-squares scales lower-bounds
+    # the squared error of any factorisation of this family, the GPU's included.
+    from oracle import brute
+    W = np.random.default_rng(seed).standard_normal(shape)
+    res = nq.nq_lbadmm(torch.from_numpy(W.astype(np.float32)).cuda(), r, iters=50)
+    Wt, _, _ = O.precondition(W.astype(np.float32).astype(np.float64), None, None, r)
+    e2_gpu = res["rel_err"] ** 2 * np.sum(Wt * Wt)
+    bf, *_ = brute.min_sq_error(Wt, r)
+    assert bf <= e2_gpu * (1 + 1e-6) + 1e-12, (bf, e2_gpu)
