@@ -154,7 +154,10 @@ def kernel_units(cls, m, n, r, K, T):
     if cls == "ginv":
         return float(r) ** 3 / 3.0, "FLOP", "tensor"         # L^-T L^-1
     if cls == "svid":
-        return 4.0 * K * (m + n) / 2 * r, "B", "hbm"         # K reads of S (FP32)
+        # K reads of S (FP32).  Inside nq_lbadmm the SVID passes run on an auxiliary
+        # stream beside the next RHS GEMM and solve, so this class's time is elapsed time
+        # while overlapped, not the passes' own duration.
+        return 4.0 * K * (m + n) / 2 * r, "B", "hbm"
     return None
 
 
@@ -418,8 +421,11 @@ def run_ours(args):
         e = roofline_entry(cls, nl, ms, m, n, r, K, T, peaks)
         if e is not None:
             e["share_of_step"] = round(ms / (t_local * 1e3), 4)
+            if cls == "svid":
+                e["overlapped"] = "runs beside the RHS GEMM and solve on an auxiliary stream"
             entries[cls] = e
-    dominant = max(entries.values(), key=lambda e: e["launches"] * e["ms_per_launch"])
+    dominant = max((e for e in entries.values() if "overlapped" not in e),
+                   key=lambda e: e["launches"] * e["ms_per_launch"])
     value = world * iters * args.steps / t
     tflops = 4.0 * m * n * r * iters * world * args.steps / t / 1e12
     ms_iter = (step_ms - (prof["calib"][1] + prof["calib_finalize"][1]) / args.steps) / iters

@@ -139,6 +139,15 @@ int pick_bn(int64_t N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
 
 inline bool valid_prec(int prec) { return prec == NQ_PREC_BF16 || prec == NQ_PREC_FP32; }
 
+// Tile width for skinny products (few 128-row tiles): the widest BN whose tile count still
+// fills the SMs, else the narrowest.
+int pick_bn_fill(int64_t M, int64_t N, int sms) {
+    for (int bn : {256, 128}) {
+        if (N > bn / 2 && ceil_div(M, 128) * ceil_div(N, bn) >= sms) return bn;
+    }
+    return N <= 64 ? 64 : (ceil_div(M, 128) * ceil_div(N, 128) >= sms ? 128 : 64);
+}
+
 nq_status read_err(int *dev_err, cudaStream_t s, bool reset) {
     int h = 0;
     NQ_CK(cudaMemcpyAsync(&h, dev_err, sizeof(int), cudaMemcpyDeviceToHost, s));
@@ -191,9 +200,11 @@ nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s
 // the G^-1 GEMM of a half step run beside the RHS GEMM, and the two events that fork it
 // from, and join it back into, the caller's stream.  Created by the first call of a host
 // thread on a device; never destroyed (they live until the process exits).
+// The same context also holds the auxiliary stream of the SVID passes, which run beside
+// the next half step's RHS GEMM and solve (see lb_iterate), with its events.
 struct SideCtx {
-    cudaStream_t side = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaStream_t side = nullptr, aux = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, pre_rhs = nullptr, svid_done[2] = {nullptr, nullptr};
 };
 
 nq_status side_ctx(SideCtx **out) {
@@ -203,8 +214,9 @@ nq_status side_ctx(SideCtx **out) {
     SideCtx &c = ctx[dev];
     if (!c.side) {
         NQ_CK(cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking));
-        NQ_CK(cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming));
-        NQ_CK(cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming));
+        NQ_CK(cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking));
+        for (cudaEvent_t *e : {&c.fork, &c.join, &c.pre_rhs, &c.svid_done[0], &c.svid_done[1]})
+            NQ_CK(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     }
     *out = &c;
     return NQ_OK;
@@ -287,8 +299,25 @@ nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s)
     return NQ_OK;
 }
 
+nq_status lb_svid(const Lb &lb, int side, int K, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    ProfScope ps(NQ_K_SVID, s);
+    NQ_CK(svid(lb.p<float>(L.s[side]), L.rows(side), L.r, L.ldr, K, L.nsv, lb.p<float>(L.bcur),
+               lb.p<float>(L.tvec), lb.p<float>(L.partb), lb.p<double>(L.partn),
+               lb.p<float>(L.a[side]), lb.p<float>(L.b[side]), s));
+    return NQ_OK;
+}
+
+// One half step: X_side from X_other (Gram, factorisation, G^-1, RHS, solve), then the
+// SVID of this side on ``s`` when ``ov`` is null.  Inside lb_iterate ``ov`` is the side
+// context and the SVIDs run on its auxiliary stream instead: ``pending`` (>= 0) is the
+// side solved by the previous half step, whose SVID is started once this half step's
+// G^-1 is formed, beside its RHS GEMM and solve; ``wait_own`` makes the RHS GEMM wait for
+// the SVID of ``side`` started by the previous half step (the RHS and the solve read the
+// dual state a, b it writes).
 nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, int prec,
-                       cudaStream_t s) {
+                       cudaStream_t s, SideCtx *ov = nullptr, int pending = -1,
+                       bool wait_own = false) {
     const LbLayout &L = lb.L;
     const int other = 1 - side;
     const int64_t rows = L.rows(side), Kd = L.rows(other);
@@ -346,6 +375,13 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, fs));
     }
     if (cc > 0) NQ_CK(cudaEventRecord(sc->join, fs));
+    if (ov && pending >= 0) {   // the previous half step's SVID, beside this RHS and solve
+        NQ_CK(cudaEventRecord(ov->pre_rhs, s));
+        NQ_CK(cudaStreamWaitEvent(ov->aux, ov->pre_rhs, 0));
+        if ((st = lb_svid(lb, pending, K, ov->aux))) return st;
+        NQ_CK(cudaEventRecord(ov->svid_done[pending], ov->aux));
+    }
+    if (ov && wait_own) NQ_CK(cudaStreamWaitEvent(s, ov->svid_done[side], 0));
 
     // R = W^ X_other + rho (Z - L), split into hi + lo bf16.  FP32-accurate mode: both
     // operands split, three passes [W^_hi, W^_lo, W^_hi] . [X_hi, X_hi, X_lo].
@@ -419,11 +455,8 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ProfScope ps(NQ_K_SOLVE, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BN, s));
     }
-    ProfScope ps(NQ_K_SVID, s);
-    NQ_CK(svid(lb.p<float>(L.s[side]), rows, L.r, L.ldr, K, L.nsv, lb.p<float>(L.bcur),
-               lb.p<float>(L.tvec), lb.p<float>(L.partb), lb.p<double>(L.partn),
-               lb.p<float>(L.a[side]), lb.p<float>(L.b[side]), s));
-    return NQ_OK;
+    if (ov) return NQ_OK;
+    return lb_svid(lb, side, K, s);
 }
 
 nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
@@ -468,13 +501,21 @@ nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
     return NQ_OK;
 }
 
+// The iterations.  The SVID of the side just solved is needed only by that side's next
+// RHS GEMM, one half step later, so it runs on the auxiliary stream beside the next half
+// step's RHS GEMM and solve; the last one runs on ``s`` before returning.
 nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, int prec,
                      float *objective_h, cudaStream_t s) {
+    SideCtx *ov = nullptr;
+    nq_status st = side_ctx(&ov);
+    if (st) return st;
     for (int t = 0; t < iters; ++t) {
-        nq_status st = lb_half_step(lb, 0, rho, lambda, K, prec, s);
+        // U side: starts the SVID of V (solved by the previous half step, none at t = 0)
+        st = lb_half_step(lb, 0, rho, lambda, K, prec, s, ov, t > 0 ? 1 : -1, t > 0);
         if (st) return st;
         if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
-        if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s))) return st;
+        // V side: starts the SVID of U, waits for its own from the previous iteration
+        if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s, ov, 0, t > 0))) return st;
         if (objective_h && t > 0 && (t % kObjRing) == 0) {
             // the ring holds the objectives of iterations t - kObjRing .. t - 1; the copy is
             // stream-ordered before the next write to slot 0
@@ -482,8 +523,12 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
                                   (size_t)kObjRing * 4, cudaMemcpyDeviceToHost, s));
         }
     }
+    // join the auxiliary stream (the last SVID of U; the SVID scratch is shared), then the
+    // last SVID of V
+    NQ_CK(cudaStreamWaitEvent(s, ov->svid_done[0], 0));
+    if ((st = lb_svid(lb, 1, K, s))) return st;
     // objective of the last iteration needs the Gram of the last V
-    nq_status st = lb_gram(lb, 1, lambda + rho, prec, s);
+    st = lb_gram(lb, 1, lambda + rho, prec, s);
     if (st) return st;
     if ((st = lb_objective(lb, lambda + rho, (iters - 1) % kObjRing, s))) return st;
     if (objective_h) {
@@ -843,7 +888,7 @@ nq_status nq_binary_matmul(const uint32_t *U_packed, const uint32_t *V_packed, c
         memset(&maps, 0, sizeof(maps));
         const int nseg = xb ? 2 : 3;
         const void *as[3] = {xh, xb ? xh : xl, xh}, *bs[3] = {vh, xb ? vl : vh, vl};
-        const int BN = pick_bn(r);
+        const int BN = pick_bn_fill(B, r, device_sm_count());
         for (int g = 0; g < nseg; ++g)
             if (!tc::make_map_bf16(&maps.a[g], as[g], B, n, L.ldt, tc::BM) ||
                 !tc::make_map_bf16(&maps.b[g], bs[g], r, n, L.ldt, BN))
@@ -864,7 +909,7 @@ nq_status nq_binary_matmul(const uint32_t *U_packed, const uint32_t *V_packed, c
     {
         tc::Maps maps;
         memset(&maps, 0, sizeof(maps));
-        const int BN = pick_bn(m);
+        const int BN = pick_bn_fill(B, m, device_sm_count());
         if (!tc::make_map_bf16(&maps.a[0], zh, B, r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.a[1], zl, B, r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.b[0], um, m, r, L.ldr, BN) ||

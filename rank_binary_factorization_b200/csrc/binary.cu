@@ -14,94 +14,117 @@
 namespace nq {
 
 // ---- GEMV path ----------------------------------------------------------------------
-// grid (ceil(nw / 8), chunks); warp w of the CTA owns packed word wd = 8 blockIdx.x + w,
-// i.e. rank columns 32 wd .. 32 wd + 31 (lane = bit); rows j of chunk blockIdx.y.
+// z pass: CTA = one chunk of rows of V; its packed words (contiguous in memory) and the
+// scaled inputs s2_j X[b][j] are staged in shared memory with coalesced copies, then warp
+// w takes words w, w + 8, ... (lane = bit) and walks the chunk's rows.
 __global__ void __launch_bounds__(256)
     bin_z_kernel(const uint32_t *__restrict__ Vp, const float *__restrict__ s2,
                  const void *__restrict__ X, int x_bf16, int64_t n, int r, int64_t B,
                  int64_t rows_per_chunk, float *__restrict__ P) {
-    extern __shared__ float xs[];   // [B][rows_per_chunk]: s2_j X[b][j] of the chunk's rows
+    extern __shared__ __align__(16) float smz[];
     const int nw = (r + 31) >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j0 = (int64_t)blockIdx.y * rows_per_chunk;
+    const int64_t j0 = (int64_t)blockIdx.x * rows_per_chunk;
     const int64_t j1 = min(n, j0 + rows_per_chunk);
     const int64_t nj = j1 - j0;
+    float *xs = smz;                                                   // [B][rows_per_chunk]
+    uint32_t *vw = reinterpret_cast<uint32_t *>(smz + B * rows_per_chunk);  // [nj][nw]
     for (int64_t e = threadIdx.x; e < B * nj; e += blockDim.x) {
         const int64_t b = e / nj, jj = e % nj, j = j0 + jj;
         const float x = x_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(X)[b * n + j])
                                : reinterpret_cast<const float *>(X)[b * n + j];
         xs[b * rows_per_chunk + jj] = s2[j] * x;
     }
+    const uint32_t *src = Vp + j0 * nw;
+    for (int64_t e = threadIdx.x; e < nj * nw; e += blockDim.x) vw[e] = __ldg(src + e);
     __syncthreads();
-    const int wd = blockIdx.x * 8 + warp;
-    if (wd >= nw) return;
-    float z[NQ_BINARY_GEMV_MAX_BATCH];
+    for (int wd = warp; wd < nw; wd += 8) {
+        float z[NQ_BINARY_GEMV_MAX_BATCH];
 #pragma unroll
-    for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) z[b] = 0.f;
-    for (int64_t jj = 0; jj < nj; ++jj) {
-        const uint32_t word = __ldg(Vp + (j0 + jj) * nw + wd);
-        const bool neg = (word >> lane) & 1u;
+        for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) z[b] = 0.f;
+        for (int64_t jj = 0; jj < nj; ++jj) {
+            const bool neg = (vw[jj * nw + wd] >> lane) & 1u;
 #pragma unroll
-        for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) {
-            if (b >= B) break;
-            const float w = xs[b * rows_per_chunk + jj];
-            z[b] += neg ? -w : w;
+            for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) {
+                if (b >= B) break;
+                const float w = xs[b * rows_per_chunk + jj];
+                z[b] += neg ? -w : w;
+            }
         }
+        const int k = 32 * wd + lane;
+        if (k < r)
+            for (int b = 0; b < B; ++b) P[((int64_t)blockIdx.x * B + b) * r + k] = z[b];
     }
-    const int k = 32 * wd + lane;
-    if (k < r)
-        for (int b = 0; b < B; ++b) P[((int64_t)blockIdx.y * B + b) * r + k] = z[b];
 }
 
-// z[b][k] = sum over chunks of P[chunk][b][k], in chunk order.
+// z[b][k] = sum over chunks of P[chunk][b][k]: four interleaved partial sums (chunks
+// c = 4q + u into sum u), combined in a fixed order, so the loads stay in flight.
 __global__ void bin_zreduce_kernel(const float *__restrict__ P, int chunks, int64_t Br,
                                    float *__restrict__ z) {
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < Br;
          e += (int64_t)gridDim.x * blockDim.x) {
-        float v = 0.f;
-        for (int c = 0; c < chunks; ++c) v += P[(int64_t)c * Br + e];
-        z[e] = v;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        int c = 0;
+#pragma unroll 2
+        for (; c + 4 <= chunks; c += 4) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] += P[(int64_t)(c + u) * Br + e];
+        }
+        for (; c < chunks; ++c) v[c & 3] += P[(int64_t)c * Br + e];
+        z[e] = (v[0] + v[1]) + (v[2] + v[3]);
     }
 }
 
-// One warp per output row i: lane = bit of each packed word of U's row i.
+// y pass: CTA = 32 output rows; their packed words and (when it fits) z are staged in
+// shared memory; warp w takes rows w, w + 8, ... with lane = bit of each word.
+constexpr int kBinRowsPerCta = 32;
 __global__ void __launch_bounds__(256)
     bin_y_kernel(const uint32_t *__restrict__ Up, const float *__restrict__ s1,
-                 const float *__restrict__ z, int64_t m, int r, int64_t B, float *__restrict__ Y) {
+                 const float *__restrict__ z, int64_t m, int r, int64_t B, int z_in_smem,
+                 float *__restrict__ Y) {
+    extern __shared__ __align__(16) float smy[];
     const int nw = (r + 31) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (i >= m) return;
-    float acc[NQ_BINARY_GEMV_MAX_BATCH];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t i0 = (int64_t)blockIdx.x * kBinRowsPerCta;
+    const int64_t ni = min((int64_t)kBinRowsPerCta, m - i0);
+    uint32_t *uw = reinterpret_cast<uint32_t *>(smy);              // [ni][nw]
+    float *zs = smy + kBinRowsPerCta * nw;                           // [B][r] when staged
+    const uint32_t *src = Up + i0 * nw;
+    for (int64_t e = threadIdx.x; e < ni * nw; e += blockDim.x) uw[e] = __ldg(src + e);
+    if (z_in_smem)
+        for (int64_t e = threadIdx.x; e < B * r; e += blockDim.x) zs[e] = __ldg(z + e);
+    __syncthreads();
+    const float *zz = z_in_smem ? zs : z;
+    for (int ii = warp; ii < ni; ii += 8) {
+        float acc[NQ_BINARY_GEMV_MAX_BATCH];
 #pragma unroll
-    for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) acc[b] = 0.f;
-    for (int wd = 0; wd < nw; ++wd) {
-        const uint32_t word = __ldg(Up + i * nw + wd);
-        const int k = 32 * wd + lane;
-        if (k >= r) break;
-        const bool neg = (word >> lane) & 1u;
+        for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) acc[b] = 0.f;
+        for (int wd = 0; wd < nw; ++wd) {
+            const int k = 32 * wd + lane;
+            if (k >= r) break;
+            const bool neg = (uw[ii * nw + wd] >> lane) & 1u;
 #pragma unroll
-        for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) {
-            if (b >= B) break;
-            const float v = __ldg(z + (int64_t)b * r + k);
-            acc[b] += neg ? -v : v;
+            for (int b = 0; b < NQ_BINARY_GEMV_MAX_BATCH; ++b) {
+                if (b >= B) break;
+                const float v = zz[(int64_t)b * r + k];
+                acc[b] += neg ? -v : v;
+            }
         }
-    }
-    const float sc = s1[i];
-    for (int b = 0; b < B; ++b) {
-        const float t = warp_sum(acc[b]);
-        if (lane == 0) Y[(int64_t)b * m + i] = sc * t;
+        const float sc = s1[i0 + ii];
+        for (int b = 0; b < B; ++b) {
+            const float t = warp_sum(acc[b]);
+            if (lane == 0) Y[(int64_t)b * m + i0 + ii] = sc * t;
+        }
     }
 }
 
 // Row chunks of the z pass: about two CTAs per SM, at least 32 rows per chunk, and the
-// chunk's scaled inputs (B x rows floats) within 192 KB of shared memory.
+// chunk's staged inputs and words within 192 KB of shared memory.
 int bin_gemv_chunks(int64_t n, int32_t r, int64_t B) {
     const int64_t nw = (r + 31) / 32;
-    const int64_t cx = (nw + 7) / 8;
-    int64_t c = (2 * kNumSMsB200) / cx;
+    int64_t c = 2 * kNumSMsB200;
     if (c > (n + 31) / 32) c = (n + 31) / 32;
-    const int64_t max_rows = (192 * 1024) / (4 * (B > 0 ? B : 1));
+    const int64_t max_rows = (192 * 1024) / (4 * ((B > 0 ? B : 1) + nw));
     if (c < (n + max_rows - 1) / max_rows) c = (n + max_rows - 1) / max_rows;
     return c < 1 ? 1 : (int)c;
 }
@@ -112,18 +135,27 @@ cudaError_t bin_gemv(const uint32_t *Up, const uint32_t *Vp, const float *s1, co
     const int chunks = bin_gemv_chunks(n, r, B);
     const int64_t rpc = (n + chunks - 1) / chunks;
     const int nw = (r + 31) / 32;
-    const size_t smem = (size_t)B * rpc * sizeof(float);
-    if (smem > 48 * 1024) {
+    const size_t smem_z = (size_t)rpc * (B + nw) * sizeof(float);
+    if (smem_z > 48 * 1024) {
         static std::atomic<uint64_t> configured{0};
         cudaError_t e = ensure_smem_limit((const void *)bin_z_kernel, 192 * 1024, configured);
         if (e != cudaSuccess) return e;
     }
-    bin_z_kernel<<<dim3((unsigned)((nw + 7) / 8), (unsigned)chunks), 256, smem, s>>>(
-        Vp, s2, X, x_bf16, n, r, B, rpc, P);
+    bin_z_kernel<<<(unsigned)chunks, 256, smem_z, s>>>(Vp, s2, X, x_bf16, n, r, B, rpc, P);
     count_launch();
     bin_zreduce_kernel<<<(unsigned)ceil_div(B * r, 256), 256, 0, s>>>(P, chunks, B * r, z);
     count_launch();
-    bin_y_kernel<<<(unsigned)ceil_div(m * 32, 256), 256, 0, s>>>(Up, s1, z, m, r, B, Y);
+    // z staged in shared memory when it fits beside the words (at most 96 KB)
+    const int z_in_smem = (size_t)B * r * sizeof(float) <= 96 * 1024;
+    const size_t smem_y = (size_t)kBinRowsPerCta * nw * sizeof(uint32_t) +
+                          (z_in_smem ? (size_t)B * r * sizeof(float) : 0);
+    if (smem_y > 48 * 1024) {
+        static std::atomic<uint64_t> configured{0};
+        cudaError_t e = ensure_smem_limit((const void *)bin_y_kernel, 192 * 1024, configured);
+        if (e != cudaSuccess) return e;
+    }
+    bin_y_kernel<<<(unsigned)ceil_div(m, kBinRowsPerCta), 256, smem_y, s>>>(Up, s1, z, m, r, B,
+                                                                           z_in_smem, Y);
     count_launch();
     return cudaGetLastError();
 }

@@ -596,6 +596,63 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Row-streaming pass for r <= 32 NPL: lane l of a warp holds columns l, l + 32, ... of one
+// row of S in registers; the warp forms t = |S_i.| b with a shuffle sum and adds
+// |S_i.| t to its column partials, row after row, with no CTA barrier per row.  At the
+// end the 8 warps' partials are summed in a fixed order.
+template <int NPL>
+__global__ void __launch_bounds__(256, 2)
+    svid_rows_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
+                     const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
+                     double *partn) {
+    __shared__ float red[8][32 * NPL];
+    __shared__ double sn[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float bl[NPL], acc[NPL];
+#pragma unroll
+    for (int u = 0; u < NPL; ++u) {
+        const int k = lane + 32 * u;
+        bl[u] = k < r ? (b_in ? b_in[k] : 1.f) : 0.f;
+        acc[u] = 0.f;
+    }
+    double nacc = 0.0;
+    const int64_t nw = (int64_t)gridDim.x * 8;
+    for (int64_t i = (int64_t)blockIdx.x * 8 + warp; i < rows; i += nw) {
+        const float *row = S + i * ldf;
+        float sv[NPL];
+#pragma unroll
+        for (int u = 0; u < NPL; ++u) {
+            const int k = lane + 32 * u;
+            sv[u] = k < r ? fabsf(__ldcg(row + k)) : 0.f;
+        }
+        float t = 0.f;
+#pragma unroll
+        for (int u = 0; u < NPL; ++u) t = fmaf(sv[u], bl[u], t);
+        t = warp_sum(t);
+#pragma unroll
+        for (int u = 0; u < NPL; ++u) acc[u] = fmaf(sv[u], t, acc[u]);
+        if (lane == 0) {
+            nacc += (double)t * (double)t;
+            if (write_t) tvec[i] = t;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < NPL; ++u) red[warp][lane + 32 * u] = acc[u];
+    if (lane == 0) sn[warp] = nacc;
+    __syncthreads();
+    for (int k = threadIdx.x; k < r; k += blockDim.x) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += red[w][k];
+        partb[(int64_t)blockIdx.x * r + k] = v;
+    }
+    if (threadIdx.x == 0) {
+        double v = 0.0;
+        for (int w = 0; w < 8; ++w) v += sn[w];
+        partn[blockIdx.x] = v;
+    }
+}
+
 // b'_k = sum over CTAs of partb[.][k] / ||t||: CTA = 32 columns x 8 groups of partial rows;
 // each group walks every 8th partial row, then the 8 group sums are combined in a fixed
 // order (deterministic).  The last pass also writes a = t / ||t||.
@@ -618,8 +675,11 @@ __global__ void __launch_bounds__(256)
     const int64_t col = (int64_t)blockIdx.x * 32 + c;
     double v = 0.0;
     if (col < r) {
-#pragma unroll 8
-        for (int k = grp; k < nblk; k += 8) v += partb[(int64_t)k * r + col];
+        double w[4] = {0.0, 0.0, 0.0, 0.0};   // interleaved sums keep the loads in flight
+        int k = grp, u = 0;
+#pragma unroll 4
+        for (; k < nblk; k += 8, u = (u + 1) & 3) w[u] += partb[(int64_t)k * r + col];
+        v = (w[0] + w[1]) + (w[2] + w[3]);
     }
     sg[grp][c] = v;
     __syncthreads();
@@ -678,9 +738,35 @@ static cudaError_t svid_passes(const float *S, int64_t rows, int32_t r, int64_t 
     return cudaGetLastError();
 }
 
+template <int NPL>
+static cudaError_t svid_row_passes(const float *S, int64_t rows, int32_t r, int64_t ldf, int K,
+                                   int nsv, float *bcur, float *tvec, float *partb,
+                                   double *partn, float *a, float *b, cudaStream_t s) {
+    int64_t grid = ceil_div(rows, 8);
+    const int64_t cap = 2 * (int64_t)device_sm_count();
+    if (grid > cap) grid = cap;
+    if (grid > nsv) grid = nsv;
+    for (int pass = 1; pass <= K; ++pass) {
+        const float *b_in = pass == 1 ? nullptr : bcur + (size_t)((pass - 1) & 1) * r;
+        const bool last = pass == K;
+        float *b_out = last ? b : bcur + (size_t)(pass & 1) * r;
+        svid_rows_kernel<NPL><<<(unsigned)grid, 256, 0, s>>>(S, rows, r, ldf, b_in, tvec,
+                                                            last ? 1 : 0, partb, partn);
+        count_launch();
+        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 256, 0, s>>>(
+            partb, partn, (int)grid, r, rows, last ? 1 : 0, tvec, b_out, a);
+        count_launch();
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, int nsv,
                  float *bcur, float *tvec, float *partb, double *partn, float *a, float *b,
                  cudaStream_t s) {
+    // rows of at most 1024 columns stream through registers; longer rows through tiles
+    if (r <= 256) return svid_row_passes<8>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
+    if (r <= 512) return svid_row_passes<16>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
+    if (r <= 1024) return svid_row_passes<32>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
     switch (svid_tile_rows(ldf)) {
         case 8: return svid_passes<8>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
         case 4: return svid_passes<4>(S, rows, r, ldf, K, nsv, bcur, tvec, partb, partn, a, b, s);
