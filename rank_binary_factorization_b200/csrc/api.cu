@@ -223,14 +223,14 @@ nq_status side_ctx(SideCtx **out) {
 }
 
 // CTAs given to the factorisation while the RHS GEMM runs on the others (0: no overlap,
-// the factorisation takes the whole GPU before the GEMM).  Overlap pays only when the
-// factorisation on a fraction of the SMs is about as short as the GEMM; measured on
-// B200 it is not yet (r = 1000: 305 us on 148 CTAs, 522 us on 23 CTAs, against a
-// ~100 us GEMM), so the factorisation keeps the whole GPU.
+// the factorisation takes the whole GPU before the GEMM).  The factorisation is a chain
+// of nb = r/64 dependent tile steps plus ~nb^3/3 tile tasks for its workers; up to
+// nb = 24 half of the SMs keep the workers ahead of the chain, so the chain's latency,
+// not the SM count, sets its time, and the GEMM runs on the other half meanwhile.
+// Beyond that the workers need the whole GPU.
 int chol_ctas(int32_t r, int sms) {
-    (void)r;
-    (void)sms;
-    return 0;
+    const int nb = (r + 63) / 64;
+    return nb <= 24 ? sms / 2 : 0;
 }
 
 // ---- LB-ADMM internals ------------------------------------------------------------
