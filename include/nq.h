@@ -209,6 +209,26 @@ nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const
 nq_status nq_pack_signs(const float *X, int64_t rows, int32_t r, uint32_t *bits,
                         nq_stream_t stream);
 
+/*
+ * Least-squares refit of the channel scales with the signs fixed.  NanoQuant summary
+ * page, "Method steps" stage two and "Technical novelty": the scales s1, s2 of
+ * W~ ~ diag(s1) U+- V+-^T diag(s2) are extracted after magnitude balancing; this refines
+ * them for the fixed packed signs by alternating exact minimisations (P = U+- V+-^T):
+ *     s1_i <- sum_j W~_ij P_ij s2_j / sum_j P_ij^2 s2_j^2,   then
+ *     s2_j <- sum_i W~_ij P_ij s1_i / sum_i P_ij^2 s1_i^2,   ``sweeps`` times
+ * (a scale whose denominator vanishes keeps its value), so the error never increases.
+ * Each half sweep is one +-1 tensor-core GEMM (exact) with the sums fused into its
+ * epilogue (FP32 within a 64-256 column tile, FP64 across tiles).  W, d_in, d_out,
+ * U_packed, V_packed as for nq_recon_error; s1 (m), s2 (n): device float, updated in
+ * place.  rel_err: host, or NULL: the reconstruction error after the refit
+ * (synchronises when non-NULL).  sweeps >= 1.
+ */
+size_t nq_ls_refit_workspace_size(int64_t m, int64_t n, int32_t r);
+nq_status nq_ls_refit(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                      const float *d_out, const uint32_t *U_packed, const uint32_t *V_packed,
+                      int32_t r, float *s1, float *s2, int32_t sweeps, double *rel_err,
+                      void *ws, size_t ws_bytes, nq_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* 3. Inference with the packed factors.  NanoQuant summary page, "Technical    */
 /* novelty" (技术新颖性) and "Limitations" (局限与改进): the compressed layer     */
@@ -321,7 +341,8 @@ typedef enum {
     NQ_K_RECON = 10,    /* tcgen05 +-1 reconstruction error                          */
     NQ_K_GINV = 11,     /* tcgen05 G^-1 = L^-T L^-1 (symmetric, split BF16)          */
     NQ_K_BINARY = 12,   /* binary GEMV/GEMM on the packed factors                    */
-    NQ_K_COUNT = 13
+    NQ_K_REFIT = 13,    /* least-squares scale refit                                 */
+    NQ_K_COUNT = 14
 } nq_kernel_class;
 
 /* Number of kernel launches the library has issued in this process. */

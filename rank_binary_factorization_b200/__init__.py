@@ -21,7 +21,7 @@ from ._lib import (FIELDS, NQ_BF16, NQ_F32, NQ_PREC_BF16, NQ_PREC_FP32, NQError,
 
 __all__ = [
     "nq_bpw", "nq_rank_for_bpw", "nq_calib_stats", "nq_calib_precond", "nq_lbadmm",
-    "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "LBState", "NQError",
+    "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "nq_ls_refit", "LBState", "NQError",
     "status_string", "lib",
     "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
 ]
@@ -146,6 +146,21 @@ def nq_binary_matmul(U_packed, V_packed, s1, s2, r, X, ws=None):
         _ptr(U_packed), _ptr(V_packed), _ptr(s1), _ptr(s2), m, n, r, _ptr(X2), _dtype(X2), B,
         _ptr(Y), _ptr(ws), ws.numel(), _stream()))
     return Y[0] if vec else Y
+
+
+def nq_ls_refit(W, U_packed, V_packed, r, s1, s2, d_in=None, d_out=None, sweeps=3, ws=None,
+                want_error=True):
+    """Least-squares refit of s1, s2 (updated in place) for the fixed packed signs; returns
+    the reconstruction error after the refit (or None)."""
+    _cuda(W, "W")
+    m, n = W.shape
+    ws = ws if ws is not None else workspace(lib.nq_ls_refit_workspace_size(m, n, r), W.device)
+    out = ctypes.c_double(0.0)
+    check("nq_ls_refit", lib.nq_ls_refit(
+        _ptr(W), _dtype(W), m, n, _ptr(d_in), _ptr(d_out), _ptr(U_packed), _ptr(V_packed), r,
+        _ptr(s1), _ptr(s2), sweeps, ctypes.byref(out) if want_error else None, _ptr(ws),
+        ws.numel(), _stream()))
+    return out.value if want_error else None
 
 
 def nq_pack_signs(X):

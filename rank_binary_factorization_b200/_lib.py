@@ -46,6 +46,9 @@ SIGNATURES = {
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_pack_signs": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_vp]),
     "nq_binary_workspace_size": (c_sz, [c_i64, c_i64, c_i32, c_i64]),
+    "nq_ls_refit_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
+    "nq_ls_refit": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp,
+                            c_i32, c_vp, c_vp, c_sz, c_vp]),
     "nq_binary_matmul": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_vp, c_i32, c_i64,
                                  c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_prepare": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_u64, c_i32,
@@ -69,7 +72,7 @@ SIGNATURES = {
 }
 NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
-                  "objective", "finish", "recon", "ginv", "binary"]
+                  "objective", "finish", "recon", "ginv", "binary", "refit"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

@@ -71,7 +71,8 @@ bool g_prof_on = false;
 // NVTX range names of the kernel classes (nq_kernel_class order)
 const char *const kClassNames[NQ_K_COUNT] = {
     "nq.calib", "nq.calib_finalize", "nq.prep", "nq.gram", "nq.chol", "nq.rhs",
-    "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv", "nq.binary"};
+    "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv", "nq.binary",
+    "nq.refit"};
 
 // Scope of one kernel class's launches: an NVTX range on the host timeline (seen by
 // profilers; inert otherwise) and, when recording is on, a CUDA event pair on the stream.
@@ -121,6 +122,8 @@ nq_status check_device() {
 }
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+// a vector that is absent (identity) or starts on a 16-byte boundary
+inline bool vec16(const void *p) { return !p || aligned(p, 16); }
 
 nq_status check_lb_args(int64_t m, int64_t n, int32_t r) {
     if (m < 1 || n < 1 || m > kMaxDim || n > kMaxDim) return NQ_ERR_INVALID_ARG;
@@ -579,6 +582,7 @@ nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, co
     ep.d_out = d_out;
     ep.s1 = s1;
     ep.s2 = s2;
+    ep.cvec = vec16(d_in) && vec16(s2);
     NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RECON, BN, s));
     NQ_CK(recon_finalize(lb.p<double>(L.part), (int)tc::num_tiles((int)L.m, (int)L.n, BN), lb.sc,
                          &lb.sc->recon2, s));
@@ -792,6 +796,42 @@ size_t nq_recon_workspace_size(int64_t m, int64_t n, int32_t r) {
     return L.total;
 }
 
+// ||W~ - diag(s1) U+- V+-^T diag(s2)|| / ||W~|| into sc->recon2 from the +-1 BF16
+// operands up (m x r) and vp (n x r), row stride ldr.
+static nq_status enqueue_recon(const void *W, nq_dtype dt, int64_t m, int64_t n,
+                               const float *d_in, const float *d_out, const __nv_bfloat16 *up,
+                               const __nv_bfloat16 *vp, int64_t ldr, int32_t r, const float *s1,
+                               const float *s2, Scalars *sc, double *part, cudaStream_t s) {
+    NQ_CK(wt_norm_partials(W, dt == NQ_BF16, m, n, d_in, d_out, part, &sc->err, s));
+    NQ_CK(reduce_partials(part, kRedBlocks, &sc->wt_norm2, nullptr, r, s));
+    const int BN = pick_bn(n);
+    tc::Maps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!tc::make_map_bf16(&maps.a[0], up, m, r, ldr, tc::BM) ||
+        !tc::make_map_bf16(&maps.b[0], vp, n, r, ldr, BN))
+        return NQ_ERR_CUDA;
+    tc::EpiParams ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.M = (int)m;
+    ep.N = (int)n;
+    ep.nseg = 1;
+    ep.kblocks[0] = (int)ceil_div(r, tc::BK);
+    ep.err = &sc->err;
+    ep.part = part;
+    ep.W = W;
+    ep.w_bf16 = dt == NQ_BF16;
+    ep.w_vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) && ((n * (dt == NQ_BF16 ? 2 : 4)) % 16 == 0);
+    ep.ldw = n;
+    ep.d_in = d_in;
+    ep.d_out = d_out;
+    ep.s1 = s1;
+    ep.s2 = s2;
+    ep.cvec = vec16(d_in) && vec16(s2);
+    NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RECON, BN, s));
+    NQ_CK(recon_finalize(part, (int)tc::num_tiles((int)m, (int)n, BN), sc, &sc->recon2, s));
+    return NQ_OK;
+}
+
 nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
                          const float *d_out, const uint32_t *U_packed, const uint32_t *V_packed,
                          int32_t r, const float *s1, const float *s2, double *rel_err, void *ws,
@@ -812,32 +852,78 @@ nq_status nq_recon_error(const void *W, nq_dtype dt, int64_t m, int64_t n, const
     NQ_CK(cudaMemsetAsync(sc, 0, sizeof(Scalars), s));
     NQ_CK(unpack_pm(U_packed, m, r, up, L.ldr, s));
     NQ_CK(unpack_pm(V_packed, n, r, vp, L.ldr, s));
-    NQ_CK(wt_norm_partials(W, dt == NQ_BF16, m, n, d_in, d_out, part, &sc->err, s));
-    NQ_CK(reduce_partials(part, kRedBlocks, &sc->wt_norm2, nullptr, r, s));
-    const int BN = pick_bn(n);
-    tc::Maps maps;
-    memset(&maps, 0, sizeof(maps));
-    if (!tc::make_map_bf16(&maps.a[0], up, m, r, L.ldr, tc::BM) ||
-        !tc::make_map_bf16(&maps.b[0], vp, n, r, L.ldr, BN))
-        return NQ_ERR_CUDA;
-    tc::EpiParams ep;
-    memset(&ep, 0, sizeof(ep));
-    ep.M = (int)m;
-    ep.N = (int)n;
-    ep.nseg = 1;
-    ep.kblocks[0] = (int)ceil_div(r, tc::BK);
-    ep.err = &sc->err;
-    ep.part = part;
-    ep.W = W;
-    ep.w_bf16 = dt == NQ_BF16;
-    ep.w_vec = (reinterpret_cast<uintptr_t>(W) % 16 == 0) && ((n * (dt == NQ_BF16 ? 2 : 4)) % 16 == 0);
-    ep.ldw = n;
-    ep.d_in = d_in;
-    ep.d_out = d_out;
-    ep.s1 = s1;
-    ep.s2 = s2;
-    NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RECON, BN, s));
-    NQ_CK(recon_finalize(part, (int)tc::num_tiles((int)m, (int)n, BN), sc, &sc->recon2, s));
+    if ((st = enqueue_recon(W, dt, m, n, d_in, d_out, up, vp, L.ldr, r, s1, s2, sc, part, s)))
+        return st;
+    NQ_CK(cudaMemcpyAsync(rel_err, &sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
+    return read_err(&sc->err, s, false);
+}
+
+size_t nq_ls_refit_workspace_size(int64_t m, int64_t n, int32_t r) {
+    if (check_lb_args(m, n, r)) return 0;
+    RefitLayout L;
+    L.build(m, n, r);
+    return L.total;
+}
+
+nq_status nq_ls_refit(const void *W, nq_dtype dt, int64_t m, int64_t n, const float *d_in,
+                      const float *d_out, const uint32_t *U_packed, const uint32_t *V_packed,
+                      int32_t r, float *s1, float *s2, int32_t sweeps, double *rel_err,
+                      void *ws, size_t ws_bytes, nq_stream_t stream) {
+    if (!W || !U_packed || !V_packed || !s1 || !s2 || sweeps < 1 ||
+        (dt != NQ_F32 && dt != NQ_BF16))
+        return NQ_ERR_INVALID_ARG;
+    nq_status st = check_lb_args(m, n, r);
+    if (st) return st;
+    RefitLayout L;
+    L.build(m, n, r);
+    if ((st = check_ws(ws, ws_bytes, L.total))) return st;
+    if ((st = check_device())) return st;
+    cudaStream_t s = cs(stream);
+    Scalars *sc = at<Scalars>(ws, L.scal);
+    __nv_bfloat16 *up = at<__nv_bfloat16>(ws, L.up), *vp = at<__nv_bfloat16>(ws, L.vp);
+    double *num = at<double>(ws, L.num), *den = at<double>(ws, L.den);
+    ProfScope ps(NQ_K_REFIT, s);
+    NQ_CK(cudaMemsetAsync(sc, 0, sizeof(Scalars), s));
+    NQ_CK(unpack_pm(U_packed, m, r, up, L.ldr, s));
+    NQ_CK(unpack_pm(V_packed, n, r, vp, L.ldr, s));
+    const bool wv = (reinterpret_cast<uintptr_t>(W) % 16 == 0) && ((n * (dt == NQ_BF16 ? 2 : 4)) % 16 == 0);
+    for (int sw = 0; sw < sweeps; ++sw) {
+        for (int pass = 0; pass < 2; ++pass) {
+            // pass 0: rows i of W (s1, sums over j with s2); pass 1: columns j (s2, over i)
+            const int64_t M = pass == 0 ? m : n, N = pass == 0 ? n : m;
+            const __nv_bfloat16 *A = pass == 0 ? up : vp, *Bm = pass == 0 ? vp : up;
+            const int BN = pick_bn(N) < 64 ? 64 : pick_bn(N);
+            tc::Maps maps;
+            memset(&maps, 0, sizeof(maps));
+            if (!tc::make_map_bf16(&maps.a[0], A, M, r, L.ldr, tc::BM) ||
+                !tc::make_map_bf16(&maps.b[0], Bm, N, r, L.ldr, BN))
+                return NQ_ERR_CUDA;
+            tc::EpiParams ep;
+            memset(&ep, 0, sizeof(ep));
+            ep.M = (int)M;
+            ep.N = (int)N;
+            ep.nseg = 1;
+            ep.kblocks[0] = (int)ceil_div(r, tc::BK);
+            ep.err = &sc->err;
+            ep.W = W;
+            ep.w_bf16 = dt == NQ_BF16;
+            ep.w_vec = wv;
+            ep.ldw = n;
+            ep.d_in = d_in;
+            ep.d_out = d_out;
+            ep.refit_trans = pass;
+            ep.sv = pass == 0 ? s2 : s1;
+            ep.cvec = vec16(pass == 0 ? d_in : d_out) && vec16(ep.sv);
+            ep.num = num;
+            ep.den = den;
+            NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_REFIT, BN, s));
+            NQ_CK(refit_scales(num, den, (int)ceil_div(N, BN), M, pass == 0 ? s1 : s2, s));
+        }
+    }
+    if (!rel_err) return NQ_OK;
+    if ((st = enqueue_recon(W, dt, m, n, d_in, d_out, up, vp, L.ldr, r, s1, s2, sc,
+                            at<double>(ws, L.part), s)))
+        return st;
     NQ_CK(cudaMemcpyAsync(rel_err, &sc->recon2, sizeof(double), cudaMemcpyDeviceToHost, s));
     return read_err(&sc->err, s, false);
 }

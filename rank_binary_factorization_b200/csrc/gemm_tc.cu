@@ -172,7 +172,8 @@ __device__ __forceinline__ void gram_mirror(const EpiParams &p, int row, int col
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int col0,
-                                               const float (&v)[16], float &acc_sum) {
+                                               const float (&v)[16], float &acc_sum,
+                                               float &acc_aux) {
     const bool full = (col0 + 16 <= p.N);
     if constexpr (EPI == EPI_GRAM) {
         float *o = p.out + (int64_t)row * p.ldo + col0;
@@ -303,6 +304,41 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
         }
         if (bad) raise_error(p.err, NQ_ERR_NONFINITE);
         acc_sum += part;
+    } else if constexpr (EPI == EPI_REFIT) {
+        float pn = 0.f, pd = 0.f;
+        const float *dcol = p.refit_trans ? p.d_out : p.d_in;
+        const float *drow = p.refit_trans ? p.d_in : p.d_out;
+        const float dr = drow ? drow[row] : 1.f;
+        float dc[16], sv[16], w[16];
+        const bool cv = full && p.cvec;
+        if (cv) {
+            if (dcol) ld16(dc, dcol + col0);
+            ld16(sv, p.sv + col0);
+        }
+        if (full && !p.refit_trans && p.w_vec) {
+            if (p.w_bf16)
+                ld16_bf16(w, reinterpret_cast<const __nv_bfloat16 *>(p.W) + (int64_t)row * p.ldw + col0);
+            else
+                ld16(w, reinterpret_cast<const float *>(p.W) + (int64_t)row * p.ldw + col0);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int c = col0 + j;
+                w[j] = (full || c < p.N) ? (p.refit_trans ? load_w(p, c, row) : load_w(p, row, c)) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int c = col0 + j;
+            if (!(full || c < p.N)) continue;
+            const float dcj = cv ? (dcol ? dc[j] : 1.f) : (dcol ? dcol[c] : 1.f);
+            const float svj = cv ? sv[j] : p.sv[c];
+            const float sc = svj * v[j];
+            pn = fmaf(dr * dcj * w[j], sc, pn);
+            pd = fmaf(sc, sc, pd);
+        }
+        acc_sum += pn;
+        acc_aux += pd;
     } else if constexpr (EPI == EPI_RECON) {
         const float dro = p.d_out ? p.d_out[row] : 1.f;
         const float s1 = p.s1[row];
@@ -317,12 +353,20 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
             for (int j = 0; j < 16; ++j) w[j] = (full || col0 + j < p.N) ? load_w(p, row, col0 + j) : 0.f;
         }
         float part = 0.f;
+        float di[16], s2v[16];
+        const bool cv = full && p.cvec;
+        if (cv) {
+            if (p.d_in) ld16(di, p.d_in + col0);
+            ld16(s2v, p.s2 + col0);
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int c = col0 + j;
             if (!(full || c < p.N)) continue;
-            const float wt = dro * w[j] * (p.d_in ? p.d_in[c] : 1.f);
-            const float d = wt - s1 * v[j] * p.s2[c];
+            const float dij = cv ? (p.d_in ? di[j] : 1.f) : (p.d_in ? p.d_in[c] : 1.f);
+            const float s2j = cv ? s2v[j] : p.s2[c];
+            const float wt = dro * w[j] * dij;
+            const float d = wt - s1 * v[j] * s2j;
             part += d * d;
         }
         acc_sum += part;
@@ -485,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int m0, n0;
             tile_origin<BN>(p, tile, num_m, m0, n0);
             const int row = m0 + 32 * q + lane;
-            float acc_sum = 0.f;
+            float acc_sum = 0.f, acc_aux = 0.f;
             if (!dead) {
                 // one lane waits; the outcome is broadcast so that the warp-collective
                 // tcgen05.ld below is executed by all 32 lanes or by none
@@ -505,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // split-K partial: the unit's raw 128 x 128 tile, reduced later
                         st16(p.out + ((int64_t)unit * BM + 32 * q + lane) * BM + c, v);
                     } else if (row < p.M && n0 + c < p.N) {
-                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum);
+                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum, acc_aux);
                         if constexpr (EPI == EPI_SPLIT)
                             if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
                         if constexpr (EPI == EPI_GRAM)
@@ -515,6 +559,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[as]);
+            }
+            if constexpr (EPI == EPI_REFIT) {
+                // one thread owns (row, this tile's columns): its sums are the partials
+                if (!dead && row < p.M) {
+                    const int64_t o = (int64_t)(n0 / BN) * p.M + row;
+                    p.num[o] = (double)acc_sum;
+                    p.den[o] = (double)acc_aux;
+                }
             }
             if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
                 if (p.part && (EPI == EPI_RECON || p.objective)) {
@@ -609,6 +661,7 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_RECON: return launch_bn<EPI_RECON>(maps, p, BN, s);
         case EPI_SPLIT: return launch_bn<EPI_SPLIT>(maps, p, BN, s);
         case EPI_SCALE: return launch_bn<EPI_SCALE>(maps, p, BN, s);
+        case EPI_REFIT: return launch_bn<EPI_REFIT>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
 }

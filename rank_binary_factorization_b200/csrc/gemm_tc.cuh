@@ -25,7 +25,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4,
-                 EPI_SCALE = 5 };
+                 EPI_SCALE = 5, EPI_REFIT = 6 };
 
 struct Maps {
     CUtensorMap a[3];
@@ -74,8 +74,17 @@ struct EpiParams {
     const void *W;
     int w_bf16;
     int w_vec;                 // W rows 16-byte aligned: vector loads in the epilogue
+    int cvec;                  // EPI_RECON / EPI_REFIT: the per-column vectors (d_in or d_out,
+                               // s2 or sv) start 16-byte aligned: vector loads
     int64_t ldw;
     const float *d_in, *d_out, *s1, *s2;
+    // EPI_REFIT: acc = P (row, col) of the +-1 product; with w = W~ of the pair (W read as
+    // W[col][row] when refit_trans, i.e. the GEMM's rows are W's columns), accumulate
+    // num[tn][row] = sum_col w acc sv[col] and den[tn][row] = sum_col acc^2 sv[col]^2 over
+    // the tile's BN columns (tn = the tile's column index)
+    int refit_trans;
+    const float *sv;
+    double *num, *den;
 };
 
 // Host: encode a 2-D BF16 tensor map over rows x cols (row stride ld elements) with

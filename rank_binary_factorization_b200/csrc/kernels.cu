@@ -989,6 +989,28 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Least-squares scale update: s_i = sum_t num[t][i] / sum_t den[t][i] (tiles in order);
+// a scale whose denominator vanishes keeps its value.
+__global__ void refit_scales_kernel(const double *__restrict__ num, const double *__restrict__ den,
+                                    int ntiles, int64_t M, float *s) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < M;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        double a = 0.0, b = 0.0;
+        for (int t = 0; t < ntiles; ++t) {
+            a += num[(int64_t)t * M + i];
+            b += den[(int64_t)t * M + i];
+        }
+        if (b > 0.0) s[i] = (float)(a / b);
+    }
+}
+
+cudaError_t refit_scales(const double *num, const double *den, int ntiles, int64_t M, float *s,
+                         cudaStream_t st) {
+    refit_scales_kernel<<<(unsigned)ceil_div(M, 256), 256, 0, st>>>(num, den, ntiles, M, s);
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t recon_finalize(const double *part, int count, const Scalars *sc, double *out,
                            cudaStream_t s) {
     recon_finalize_kernel<<<1, 256, 0, s>>>(part, count, sc, out);

@@ -100,6 +100,9 @@ cudaError_t pack_signs(const float *X, int64_t rows, int32_t r, int64_t ldx, uin
 // +-1 bf16 [rows][ldpm] from packed bits.
 cudaError_t unpack_pm(const uint32_t *bits, int64_t rows, int32_t r, __nv_bfloat16 *pm,
                       int64_t ldpm, cudaStream_t s);
+// s_i = sum_t num[t][i] / sum_t den[t][i] over ntiles partial rows (kept when den = 0)
+cudaError_t refit_scales(const double *num, const double *den, int ntiles, int64_t M, float *s,
+                         cudaStream_t st);
 // *out = sqrt(sum(part) / wt_norm2) (0 when both vanish)
 cudaError_t recon_finalize(const double *part, int count, const Scalars *sc, double *out,
                            cudaStream_t s);

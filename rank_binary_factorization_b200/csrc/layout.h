@@ -182,6 +182,34 @@ struct BinLayout {
     }
 };
 
+// Workspace of nq_ls_refit: the +-1 operands, the per-(row, tile) partial sums of both
+// passes (tiles of 64 columns at most: the narrowest tile width) and the reduction
+// partials of the final reconstruction error.
+struct RefitLayout {
+    int64_t ldr = 0;
+    size_t scal = 0, up = 0, vp = 0, num = 0, den = 0, part = 0, total = 0;
+    void build(int64_t m, int64_t n, int32_t r) {
+        ldr = (r + 7) / 8 * 8;
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            size_t o = off;
+            off = align_up(off + bytes);
+            return o;
+        };
+        const int64_t a = ((n + 63) / 64) * m, b = ((m + 63) / 64) * n;
+        const int64_t np = a > b ? a : b;
+        scal = take(sizeof(Scalars));
+        up = take((size_t)m * ldr * 2);
+        vp = take((size_t)n * ldr * 2);
+        num = take((size_t)np * 8);
+        den = take((size_t)np * 8);
+        int64_t t_rec = ((m + 127) / 128) * ((n + 63) / 64);
+        if (t_rec < kRedBlocks) t_rec = kRedBlocks;
+        part = take((size_t)t_rec * 8);
+        total = off;
+    }
+};
+
 struct ReconLayout {
     int64_t m = 0, n = 0;
     int32_t r = 0;

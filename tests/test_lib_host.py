@@ -126,6 +126,15 @@ def test_argument_errors_are_reported_before_any_device_work():
     assert L.nq_lbadmm_prepare(fake, 0, 8, 8, null, null, 2, 0, 3, null, fake, 1 << 30,
                                null) == INV
     assert L.nq_pack_signs(null, 4, 4, fake, null) == INV
+    # refit: zero sweeps, null scales; binary matmul: empty batch, null input
+    assert L.nq_ls_refit(fake, 0, 8, 8, null, null, fake, fake, 2, fake, fake, 0, null, fake,
+                         1 << 30, null) == INV
+    assert L.nq_ls_refit(fake, 0, 8, 8, null, null, fake, fake, 2, null, fake, 1, null, fake,
+                         1 << 30, null) == INV
+    assert L.nq_binary_matmul(fake, fake, fake, fake, 8, 8, 2, fake, 0, 0, fake, fake, 1 << 30,
+                              null) == INV
+    assert L.nq_binary_matmul(fake, fake, fake, fake, 8, 8, 2, null, 0, 1, fake, fake, 1 << 30,
+                              null) == INV
 
 
 @pytest.mark.parametrize("m,n,r", [(300, 200, 40), (256, 512, 16), (4096, 4096, 2032),
