@@ -140,7 +140,9 @@ def kernel_units(cls, m, n, r, K, T):
     Per launch scope, averaged over the two sides where they differ.  "chol" counts the
     method's own work, one Cholesky factorisation (r^3 / 3); the triangular inverse the
     library also forms there is executed work beyond it.  "ginv" is the product
-    L^-T L^-1 of two triangular factors (r^3 / 3)."""
+    L^-T L^-1 of two triangular factors (r^3 / 3).  "newton" (the Newton-Schulz update
+    of G^-1 that replaces the factorisation once G changes little) is credited with the
+    explicit inverse it replaces (r^3)."""
     if cls == "calib":
         return T * (m + n), "B", "hbm"   # per launch: mean of the two BF16 streams (T x n, T x m)
     if cls == "rhs":
@@ -153,6 +155,11 @@ def kernel_units(cls, m, n, r, K, T):
         return float(r) ** 3 / 3.0, "FLOP", "alu"            # Cholesky of the r x r system
     if cls == "ginv":
         return float(r) ** 3 / 3.0, "FLOP", "tensor"         # L^-T L^-1
+    if cls == "newton":
+        # the update stands in for forming G^-1 explicitly (Cholesky r^3/3, triangular
+        # inverse r^3/3, L^-T L^-1 r^3/3); its own steps execute 4 r^3 each (two r x r
+        # products), in BF16 or split BF16
+        return float(r) ** 3, "FLOP", "tensor"
     if cls == "svid":
         # K reads of S (FP32).  Inside nq_lbadmm the SVID passes run on an auxiliary
         # stream beside the next RHS GEMM and solve, so this class's time is elapsed time

@@ -154,6 +154,26 @@ nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void
 size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
 
 /*
+ * How the inverse G^-1 = (X^T X + (lambda + rho) I)^-1 of each half step is formed.
+ * NQ_INV_CHOLESKY: the Cholesky factorisation and triangular inverse (FP32), then
+ *   G^-1 = L^-T L^-1 (split-BF16 tensor-core GEMM).
+ * NQ_INV_NEWTON: first a Newton-Schulz update of the inverse this side used in its
+ *   previous half step, X_{k+1} = X_k + (I - X_k G) X_k (two r x r tensor-core GEMMs per
+ *   step; the first two steps with BF16 operands, the later ones split BF16), at most 6
+ *   steps; the iterate after the step whose ||I - X_k G||_F is <= 1e-2 is taken (so
+ *   ||I - X G||_2 <= 1e-4 up to rounding).  An update whose residual does not shrink,
+ *   or that reaches no such step, is dropped and the Cholesky path runs instead, decided
+ *   on the device (no synchronisation).
+ * NQ_INV_AUTO (default): NQ_INV_NEWTON for r >= 256 once the workspace has run 3
+ *   iterations since its nq_lbadmm_prepare (the first iterations move G too far),
+ *   NQ_INV_CHOLESKY otherwise.
+ * Process-wide; read when a half step is enqueued.  Returns NQ_ERR_INVALID_ARG for an
+ * unknown mode.
+ */
+typedef enum { NQ_INV_AUTO = 0, NQ_INV_CHOLESKY = 1, NQ_INV_NEWTON = 2 } nq_inverse_mode;
+nq_status nq_set_inverse_mode(nq_inverse_mode mode);
+
+/*
  * Full LB-ADMM initialisation of one layer.
  *
  * Form of the iteration (the pages give no equations; this is the concrete form
@@ -162,7 +182,7 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  *   V_0[j][k] = sqrt(2/n) * (-1 if bit 63 of SplitMix64(seed, j*r+k) else +1);
  *   Z_U = L_U = Z_V = L_V = 0;
  *   repeat iters times:
- *     U = (W^ V + rho (Z_U - L_U)) (V^T V + (lambda + rho) I)^-1      (Cholesky)
+ *     U = (W^ V + rho (Z_U - L_U)) (V^T V + (lambda + rho) I)^-1
  *     S = U + L_U;  A = |S|;  b = 1;  K times { a = A b / ||A b||;  b = A^T a }
  *     Z_U = sign(S) * a b^T;   L_U = L_U + U - Z_U
  *     the same for V with W^^T and U
@@ -174,6 +194,9 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  * Tensor-core operands (W^ and the latent factor of the contraction) are BF16 for BF16
  * weights and split BF16 (FP32-accurate, see nq_precision) for FP32 weights;
  * accumulation and every other quantity is FP32 (reductions FP64 where noted).
+ * (V^T V + (lambda + rho) I)^-1 is formed explicitly and applied as a split-BF16 GEMM;
+ * how it is formed is set by nq_set_inverse_mode (Cholesky, or a Newton-Schulz update
+ * of the previous iteration's inverse that falls back to Cholesky on the device).
  *
  * W: device, m x n, dtype dt.  d_in (n), d_out (m): device float, or NULL for 1.
  * U_packed: device uint32 [m][(r+31)/32];  V_packed: device uint32 [n][(r+31)/32].
@@ -295,11 +318,17 @@ nq_status nq_lbadmm_finish(const void *W, nq_dtype dt, int64_t m, int64_t n, con
  * SVID input, from which the dual state is Z = sign(S) a b^T, L = S - Z (rows x r,
  * float); A = a (rows, float); B = b (r, float); WHAT = W^ (m x n, bf16, row
  * stride ld elements); WHAT_LO = its low part in NQ_PREC_FP32 (zero otherwise);
- * GAMMA = gamma (1 double). */
+ * GAMMA = gamma (1 double); INV_STATS = the inverse update's counters (11 x 8 bytes:
+ * [0] half steps whose G^-1 came from the Newton-Schulz update, [1] attempts that fell
+ * back to Cholesky (uint64), [2] steps of the last accepted update (int64), [3..10]
+ * ||I - X_k G||_F of the last attempt's steps (double)); GINV_U / GINV_V = G^-1 of the
+ * last U / V solve, hi part (r x r, bf16, row stride ld), GINV_U_LO / GINV_V_LO its low
+ * part (G^-1 = hi + lo). */
 typedef enum {
     NQ_FIELD_U = 0, NQ_FIELD_V = 1, NQ_FIELD_SU = 2, NQ_FIELD_SV = 3, NQ_FIELD_AU = 4,
     NQ_FIELD_AV = 5, NQ_FIELD_BU = 6, NQ_FIELD_BV = 7, NQ_FIELD_WHAT = 8, NQ_FIELD_GAMMA = 9,
-    NQ_FIELD_WHAT_LO = 10
+    NQ_FIELD_WHAT_LO = 10, NQ_FIELD_INV_STATS = 11, NQ_FIELD_GINV_U = 12,
+    NQ_FIELD_GINV_U_LO = 13, NQ_FIELD_GINV_V = 14, NQ_FIELD_GINV_V_LO = 15
 } nq_field;
 
 /* Device address, element count, element size and row stride (elements) of a
@@ -342,7 +371,8 @@ typedef enum {
     NQ_K_GINV = 11,     /* tcgen05 G^-1 = L^-T L^-1 (symmetric, split BF16)          */
     NQ_K_BINARY = 12,   /* binary GEMV/GEMM on the packed factors                    */
     NQ_K_REFIT = 13,    /* least-squares scale refit                                 */
-    NQ_K_COUNT = 14
+    NQ_K_NEWTON = 14,   /* tcgen05 Newton-Schulz update of G^-1                      */
+    NQ_K_COUNT = 15
 } nq_kernel_class;
 
 /* Number of kernel launches the library has issued in this process. */

@@ -24,6 +24,7 @@ __all__ = [
     "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "nq_ls_refit", "LBState", "NQError",
     "status_string", "lib",
     "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
+    "nq_set_inverse_mode",
 ]
 
 
@@ -171,6 +172,13 @@ def nq_pack_signs(X):
     return bits
 
 
+def nq_set_inverse_mode(mode):
+    """How each half step forms G^-1: "auto", "cholesky" or "newton" (process-wide)."""
+    code = {"auto": _lib.NQ_INV_AUTO, "cholesky": _lib.NQ_INV_CHOLESKY,
+            "newton": _lib.NQ_INV_NEWTON}[mode]
+    check("nq_set_inverse_mode", lib.nq_set_inverse_mode(code))
+
+
 def nq_launch_count():
     """Kernel launches issued by the library so far in this process."""
     return lib.nq_launch_count()
@@ -264,6 +272,20 @@ class LBState:
         if ld.value > 1:
             return flat.view(-1, ld.value)
         return flat
+
+    def inv_stats(self):
+        """Counters of the Newton-Schulz inverse update: accepted half steps, fallbacks to
+        Cholesky, steps of the last accepted update, ||I - X_k G||_F of the last attempt."""
+        w = self.field("INV_STATS").cpu()
+        i = w.view(torch.int64)
+        return dict(accepted=int(i[0]), fallbacks=int(i[1]), steps=int(i[2]),
+                    residuals=[float(x) for x in w[3:]])
+
+    def ginv(self, side):
+        """G^-1 (hi + lo, FP32, r x r) of the last solve of ``side`` (0: U, 1: V)."""
+        nm = "GINV_U" if side == 0 else "GINV_V"
+        r = self.r
+        return self.field(nm)[:r, :r].float() + self.field(nm + "_LO")[:r, :r].float()
 
     def sync_operands(self):
         check("nq_lbadmm_sync_operands", lib.nq_lbadmm_sync_operands(

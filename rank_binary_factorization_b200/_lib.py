@@ -25,7 +25,9 @@ NQ_OK, NQ_ERR_INVALID_ARG, NQ_ERR_WORKSPACE, NQ_ERR_CUDA, NQ_ERR_NONFINITE, NQ_E
     NQ_ERR_TIMEOUT, NQ_ERR_UNSUPPORTED = range(8)
 NQ_F32, NQ_BF16 = 0, 1
 NQ_PREC_BF16, NQ_PREC_FP32 = 0, 1
-FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9, WHAT_LO=10)
+FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9, WHAT_LO=10,
+              INV_STATS=11, GINV_U=12, GINV_U_LO=13, GINV_V=14, GINV_V_LO=15)
+NQ_INV_AUTO, NQ_INV_CHOLESKY, NQ_INV_NEWTON = 0, 1, 2
 
 # name -> (restype, argtypes); the list is the full set of exported entry points
 SIGNATURES = {
@@ -39,6 +41,7 @@ SIGNATURES = {
     "nq_calib_precond": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_i32, c_f64, c_vp,
                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_lbadmm_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
+    "nq_set_inverse_mode": (c_i32, [c_i32]),
     "nq_lbadmm": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_f32, c_f32, c_i32,
                           c_i32, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_recon_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
@@ -72,7 +75,7 @@ SIGNATURES = {
 }
 NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
-                  "objective", "finish", "recon", "ginv", "binary", "refit"]
+                  "objective", "finish", "recon", "ginv", "binary", "refit", "newton"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

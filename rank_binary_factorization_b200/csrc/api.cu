@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "gemm_tc.cuh"
@@ -72,7 +73,7 @@ bool g_prof_on = false;
 const char *const kClassNames[NQ_K_COUNT] = {
     "nq.calib", "nq.calib_finalize", "nq.prep", "nq.gram", "nq.chol", "nq.rhs",
     "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv", "nq.binary",
-    "nq.refit"};
+    "nq.refit", "nq.newton"};
 
 // Scope of one kernel class's launches: an NVTX range on the host timeline (seen by
 // profilers; inert otherwise) and, when recording is on, a CUDA event pair on the stream.
@@ -261,7 +262,10 @@ nq_status lb_open(Lb &lb, int64_t m, int64_t n, int32_t r, void *ws, size_t ws_b
 // Gram of the operand of side ``other`` (its BF16 transpose) into g[other]; the result is
 // symmetric, so only its lower-triangular 128 x 128 tiles are computed and mirrored.  In
 // the FP32-accurate mode the operand is split (hi + lo) and the Gram takes three passes.
-nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s) {
+// With ``ns_prep`` the Gram is also written split (hi + lo BF16) for the Newton-Schulz
+// update, and the update's gate is opened.
+nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s,
+                  bool ns_prep = false) {
     const LbLayout &L = lb.L;
     const int64_t K = L.rows(other), ld = L.ld_rows(other);
     const __nv_bfloat16 *xt = lb.p<__nv_bfloat16>(L.xt[other]);
@@ -269,33 +273,40 @@ nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s)
     constexpr int BN = tc::BM;
     tc::Maps maps;
     memset(&maps, 0, sizeof(maps));
-    const int nseg = prec == NQ_PREC_FP32 ? 3 : 1;
-    const void *as[3] = {xt, xl, xt}, *bs[3] = {xt, xt, xl};
-    for (int g = 0; g < nseg; ++g)
-        if (!tc::make_map_bf16(&maps.a[g], as[g], L.r, K, ld, tc::BM) ||
-            !tc::make_map_bf16(&maps.b[g], bs[g], L.r, K, ld, BN))
+    const int split = prec == NQ_PREC_FP32 ? 1 : 0;
+    const void *parts[2] = {xt, xl};
+    for (int g = 0; g <= split; ++g)
+        if (!tc::make_map_bf16(&maps.a[g], parts[g], L.r, K, ld, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[g], parts[g], L.r, K, ld, BN))
             return NQ_ERR_CUDA;
     tc::EpiParams ep;
     memset(&ep, 0, sizeof(ep));
     ep.M = L.r;
     ep.N = L.r;
-    ep.nseg = nseg;
-    for (int g = 0; g < nseg; ++g) ep.kblocks[g] = (int)ceil_div(K, tc::BK);
+    ep.nseg = 1;
+    ep.split3 = split;
+    ep.kblocks[0] = (int)ceil_div(K, tc::BK);
     ep.sym = 1;
     ep.err = &lb.sc->err;
     ep.out = lb.p<float>(L.g[other]);
     ep.ldo = L.r;
     ep.diag = diag;
+    __nv_bfloat16 *gh = ns_prep ? lb.p<__nv_bfloat16>(L.gsh) : nullptr;
+    __nv_bfloat16 *gl = ns_prep ? lb.p<__nv_bfloat16>(L.gsl) : nullptr;
+    ep.Rhi = gh;
+    ep.Rlo = gl;
+    ep.ldr = L.ldr;
+    ep.ns = ns_prep ? lb.p<NsState>(L.ns) : nullptr;
     // few tiles (small r): split K so that the (tile, part) units fill the SMs; the parts
     // are summed in a fixed order by gram_reduce
-    const int S = gram_ksplit(L.r, K, nseg, device_sm_count());
+    const int S = gram_ksplit(L.r, K, 1, device_sm_count());
     ProfScope ps(NQ_K_GRAM, s);
     if (S > 1) {
         ep.ksplit = S;
         ep.out = lb.p<float>(L.gpart);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
         NQ_CK(gram_reduce(lb.p<float>(L.gpart), gram_tiles(L.r), S, L.r, diag,
-                          lb.p<float>(L.g[other]), s));
+                          lb.p<float>(L.g[other]), gh, gl, L.ldr, s));
         return NQ_OK;
     }
     NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GRAM, BN, s));
@@ -308,6 +319,120 @@ nq_status lb_svid(const Lb &lb, int side, int K, cudaStream_t s) {
     NQ_CK(svid(lb.p<float>(L.s[side]), L.rows(side), L.r, L.ldr, K, L.nsv, lb.p<float>(L.bcur),
                lb.p<float>(L.tvec), lb.p<float>(L.partb), lb.p<double>(L.partn),
                lb.p<float>(L.a[side]), lb.p<float>(L.b[side]), s));
+    return NQ_OK;
+}
+
+// ---- Newton-Schulz update of G^-1 --------------------------------------------------
+// The Gram of a side changes little from one iteration to the next, so the inverse used
+// by that side's previous solve is a close start for the next one: the Newton-Schulz
+// (Schulz 1933; Ben-Israel 1965) iteration X_{k+1} = X_k (2I - G X_k), written as
+// X_{k+1} = X_k + E_k X_k with E_k = I - X_k G, converges quadratically (E_{k+1} = E_k^2)
+// whenever the spectral radius of E_0 is below 1.  Each step is two r x r tensor-core
+// GEMMs; the first kNsBf16Steps with plain BF16 operands, the rest split (hi + lo).  The
+// device decides: a step whose ||E_k||_F falls to ns_tau makes the next iterate final
+// (written to the side's G^-1); a residual that does not shrink, or no final iterate
+// after kNsMaxSteps, falls back to the Cholesky path, which then runs (gated).
+constexpr int32_t kNsMinRank = 256;  // below this the factorisation is as fast
+constexpr int kNsFirstIter = 3;      // iterations since prepare before the first attempt
+constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E||_2 <= 1e-4)
+
+std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
+
+// Iterations run on each workspace since its last prepare (host side; AUTO mode).
+std::mutex g_iter_mu;
+std::unordered_map<const void *, long long> g_iter_count;
+long long iters_since_prepare(const void *ws) {
+    std::lock_guard<std::mutex> g(g_iter_mu);
+    auto it = g_iter_count.find(ws);
+    return it == g_iter_count.end() ? 0 : it->second;
+}
+void add_iters(const void *ws, long long k) {
+    std::lock_guard<std::mutex> g(g_iter_mu);
+    if (k < 0)
+        g_iter_count[ws] = 0;
+    else
+        g_iter_count[ws] += k;
+}
+
+// Tile width of the r x r products on ``ctas`` CTAs: the fewest waves x tile width.
+int pick_bn_square(int32_t r, int ctas) {
+    int best = 64;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : {256, 128, 64}) {
+        const int64_t tiles = ceil_div(r, 128) * ceil_div(r, bn);
+        const int64_t cost = ceil_div(tiles, ctas) * bn;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    NsState *ns = lb.p<NsState>(L.ns);
+    const int r = L.r;
+    const int ctas = max_ctas > 0 ? max_ctas : device_sm_count();
+    const int BN = pick_bn_square(r, ctas);
+    const int kb = (int)ceil_div(r, tc::BK);
+    const void *gh = lb.p<void>(L.gsh), *gl = lb.p<void>(L.gsl);
+    const void *eh = lb.p<void>(L.nth), *el = lb.p<void>(L.ntl);
+    ProfScope ps(NQ_K_NEWTON, s);
+    for (int k = 0; k < kNsMaxSteps; ++k) {
+        // X_0: the side's previous G^-1; X_k: iterate buffer k % 2
+        const size_t xo_h = k == 0 ? L.gih[side] : L.nqh[k % 2];
+        const size_t xo_l = k == 0 ? L.gil[side] : L.nql[k % 2];
+        const void *xh = lb.p<void>(xo_h), *xl = lb.p<void>(xo_l);
+        const int split = k < kNsBf16Steps ? 0 : 1;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = r;
+        ep.N = r;
+        ep.nseg = 1;
+        ep.split3 = split;
+        ep.kblocks[0] = kb;
+        ep.max_ctas = max_ctas;
+        ep.err = &lb.sc->err;
+        ep.gate = &ns->gate;
+        ep.gate_skip = (1 << NS_DONE) | (1 << NS_FAIL);
+        ep.ns = ns;
+        ep.ns_step = k;
+        ep.ns_last = kNsMaxSteps - 1;
+        ep.ns_min_final = kNsBf16Steps;
+        ep.ns_tau = kNsTau;
+        ep.ldr = L.ldr;
+        {   // E_k = I - X_k G: A = X_k, B = G (symmetric: its rows are its columns)
+            tc::Maps maps;
+            memset(&maps, 0, sizeof(maps));
+            const void *as[2] = {xh, xl}, *bs[2] = {gh, gl};
+            for (int g = 0; g <= split; ++g)
+                if (!tc::make_map_bf16(&maps.a[g], as[g], r, r, L.ldr, tc::BM) ||
+                    !tc::make_map_bf16(&maps.b[g], bs[g], r, r, L.ldr, BN))
+                    return NQ_ERR_CUDA;
+            ep.part = lb.p<double>(L.nspart);
+            ep.Rhi = lb.p<__nv_bfloat16>(L.nth);
+            ep.Rlo = lb.p<__nv_bfloat16>(L.ntl);
+            NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_NS1, BN, s));
+        }
+        {   // X_{k+1} = X_k + E_k X_k: A = E_k, B = X_k (symmetric)
+            tc::Maps maps;
+            memset(&maps, 0, sizeof(maps));
+            const void *as[2] = {eh, el}, *bs[2] = {xh, xl};
+            for (int g = 0; g <= split; ++g)
+                if (!tc::make_map_bf16(&maps.a[g], as[g], r, r, L.ldr, tc::BM) ||
+                    !tc::make_map_bf16(&maps.b[g], bs[g], r, r, L.ldr, BN))
+                    return NQ_ERR_CUDA;
+            ep.part = nullptr;
+            ep.Ph = static_cast<const __nv_bfloat16 *>(xh);
+            ep.Pl = static_cast<const __nv_bfloat16 *>(xl);
+            ep.Rhi = lb.p<__nv_bfloat16>(L.nqh[(k + 1) % 2]);
+            ep.Rlo = lb.p<__nv_bfloat16>(L.nql[(k + 1) % 2]);
+            ep.Fhi = lb.p<__nv_bfloat16>(L.gih[side]);
+            ep.Flo = lb.p<__nv_bfloat16>(L.gil[side]);
+            NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_NS2, BN, s));
+        }
+    }
     return NQ_OK;
 }
 
@@ -325,7 +450,12 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     const int other = 1 - side;
     const int64_t rows = L.rows(side), Kd = L.rows(other);
     const int BN = pick_bn(L.r);
-    nq_status st = lb_gram(lb, other, lambda + rho, prec, s);
+    const int mode = g_inverse_mode.load(std::memory_order_relaxed);
+    const bool newton = mode == NQ_INV_NEWTON ||
+                        (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
+                         iters_since_prepare(lb.ws) >= kNsFirstIter);
+    NsState *ns = lb.p<NsState>(L.ns);
+    nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton);
     if (st) return st;
     // The factorisation of G and the G^-1 GEMM depend only on the Gram; the RHS GEMM only
     // on the other side's operand and this side's dual state.  With overlap they run at
@@ -340,12 +470,16 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         NQ_CK(cudaStreamWaitEvent(sc->side, sc->fork, 0));
         fs = sc->side;
     }
+    if (newton && (st = lb_newton(lb, side, cc, fs))) return st;
+    // with the update, the factorisation and the G^-1 GEMM run only if it failed
+    const int *gate = newton ? &ns->gate : nullptr;
+    const int gate_skip = newton ? (1 << NS_DONE) : 0;
     {
         ProfScope ps(NQ_K_CHOL, fs);
         NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
-                           &lb.sc->err, lb.sc->bar, cc, fs));
+                           &lb.sc->err, lb.sc->bar, cc, gate, gate_skip, fs));
     }
     {
         ProfScope ps(NQ_K_GINV, fs);
@@ -356,24 +490,25 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         const void *th = lb.p<void>(L.lth), *tl = lb.p<void>(L.ltl);
         const int BNg = tc::BM;  // square tiles: only the lower triangle is computed
         if (!tc::make_map_bf16(&maps.a[0], th, L.r, L.r, L.ldr, tc::BM) ||
-            !tc::make_map_bf16(&maps.a[1], th, L.r, L.r, L.ldr, tc::BM) ||
-            !tc::make_map_bf16(&maps.a[2], tl, L.r, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[1], tl, L.r, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.b[0], th, L.r, L.r, L.ldr, BNg) ||
-            !tc::make_map_bf16(&maps.b[1], tl, L.r, L.r, L.ldr, BNg) ||
-            !tc::make_map_bf16(&maps.b[2], th, L.r, L.r, L.ldr, BNg))
+            !tc::make_map_bf16(&maps.b[1], tl, L.r, L.r, L.ldr, BNg))
             return NQ_ERR_CUDA;
         tc::EpiParams ep;
         memset(&ep, 0, sizeof(ep));
         ep.M = L.r;
         ep.N = L.r;
-        ep.nseg = 3;
-        ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
+        ep.nseg = 1;
+        ep.split3 = 1;
+        ep.kblocks[0] = (int)ceil_div(L.r, tc::BK);
         ep.tri_k = 1;
         ep.sym = 1;
         ep.max_ctas = cc;
         ep.err = &lb.sc->err;
-        ep.Rhi = lb.p<__nv_bfloat16>(L.gih);
-        ep.Rlo = lb.p<__nv_bfloat16>(L.gil);
+        ep.gate = gate;
+        ep.gate_skip = gate_skip;
+        ep.Rhi = lb.p<__nv_bfloat16>(L.gih[side]);
+        ep.Rlo = lb.p<__nv_bfloat16>(L.gil[side]);
         ep.ldr = L.ldr;
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SPLIT, BNg, fs));
     }
@@ -395,9 +530,9 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         const void *Al = side == 0 ? lb.p<void>(L.whatL) : lb.p<void>(L.whatTL);
         const int64_t lda = side == 0 ? L.ldn : L.ldm;
         const void *B = lb.p<void>(L.xt[other]), *Bl = lb.p<void>(L.xtl[other]);
-        const int nseg = prec == NQ_PREC_FP32 ? 3 : 1;
-        const void *as[3] = {A, Al, A}, *bs[3] = {B, B, Bl};
-        for (int g = 0; g < nseg; ++g)
+        const int split = prec == NQ_PREC_FP32 ? 1 : 0;
+        const void *as[2] = {A, Al}, *bs[2] = {B, Bl};
+        for (int g = 0; g <= split; ++g)
             if (!tc::make_map_bf16(&maps.a[g], as[g], rows, Kd, lda, tc::BM) ||
                 !tc::make_map_bf16(&maps.b[g], bs[g], L.r, Kd, L.ld_rows(other), BN))
                 return NQ_ERR_CUDA;
@@ -405,8 +540,9 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         memset(&ep, 0, sizeof(ep));
         ep.M = (int)rows;
         ep.N = L.r;
-        ep.nseg = nseg;
-        for (int g = 0; g < nseg; ++g) ep.kblocks[g] = (int)ceil_div(Kd, tc::BK);
+        ep.nseg = 1;
+        ep.split3 = split;
+        ep.kblocks[0] = (int)ceil_div(Kd, tc::BK);
         ep.err = &lb.sc->err;
         ep.S = lb.p<float>(L.s[side]);
         ep.a = lb.p<float>(L.a[side]);
@@ -426,20 +562,19 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         tc::Maps maps;
         memset(&maps, 0, sizeof(maps));
         const void *rh = lb.p<void>(L.rhi), *rl = lb.p<void>(L.rlo);
-        const void *gh = lb.p<void>(L.gih), *gl = lb.p<void>(L.gil);
+        const void *gh = lb.p<void>(L.gih[side]), *gl = lb.p<void>(L.gil[side]);
         if (!tc::make_map_bf16(&maps.a[0], rh, rows, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.a[1], rl, rows, L.r, L.ldr, tc::BM) ||
-            !tc::make_map_bf16(&maps.a[2], rh, rows, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.b[0], gh, L.r, L.r, L.ldr, BN) ||
-            !tc::make_map_bf16(&maps.b[1], gh, L.r, L.r, L.ldr, BN) ||
-            !tc::make_map_bf16(&maps.b[2], gl, L.r, L.r, L.ldr, BN))
+            !tc::make_map_bf16(&maps.b[1], gl, L.r, L.r, L.ldr, BN))
             return NQ_ERR_CUDA;
         tc::EpiParams ep;
         memset(&ep, 0, sizeof(ep));
         ep.M = (int)rows;
         ep.N = L.r;
-        ep.nseg = 3;
-        ep.kblocks[0] = ep.kblocks[1] = ep.kblocks[2] = (int)ceil_div(L.r, tc::BK);
+        ep.nseg = 1;
+        ep.split3 = 1;
+        ep.kblocks[0] = (int)ceil_div(L.r, tc::BK);
         ep.err = &lb.sc->err;
         ep.S = lb.p<float>(L.s[side]);
         ep.a = lb.p<float>(L.a[side]);
@@ -499,6 +634,13 @@ nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
     }
     NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[0]), 0, (size_t)L.m * L.ldr * 4, s));
     NQ_CK(cudaMemsetAsync(lb.p<void>(L.x[1]), 0, (size_t)L.n * L.ldr * 4, s));
+    // no previous G^-1 yet: zero (a Newton-Schulz start of 0 fails at once)
+    for (int sd = 0; sd < 2; ++sd) {
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.gih[sd]), 0, (size_t)L.r * L.ldr * 2, s));
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.gil[sd]), 0, (size_t)L.r * L.ldr * 2, s));
+    }
+    NQ_CK(cudaMemsetAsync(lb.p<void>(L.ns), 0, sizeof(NsState), s));
+    add_iters(lb.ws, -1);
     NQ_CK(init_v0(L.n, L.r, seed, lb.p<float>(L.x[1]), L.ldr, lb.p<__nv_bfloat16>(L.xt[1]),
                   split ? lb.p<__nv_bfloat16>(L.xtl[1]) : nullptr, L.ldn, s));
     return NQ_OK;
@@ -519,6 +661,7 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
         if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
         // V side: starts the SVID of U, waits for its own from the previous iteration
         if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s, ov, 0, t > 0))) return st;
+        add_iters(lb.ws, 1);
         if (objective_h && t > 0 && (t % kObjRing) == 0) {
             // the ring holds the objectives of iterations t - kObjRing .. t - 1; the copy is
             // stream-ordered before the next write to slot 0
@@ -680,6 +823,13 @@ nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void
         alpha_out[1] = h.alpha[1];
         if (h.err) return static_cast<nq_status>(h.err);
     }
+    return NQ_OK;
+}
+
+nq_status nq_set_inverse_mode(nq_inverse_mode mode) {
+    if (mode != NQ_INV_AUTO && mode != NQ_INV_CHOLESKY && mode != NQ_INV_NEWTON)
+        return NQ_ERR_INVALID_ARG;
+    g_inverse_mode.store(mode, std::memory_order_relaxed);
     return NQ_OK;
 }
 
@@ -1049,6 +1199,11 @@ nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, voi
         case NQ_FIELD_WHAT: off = L.what; cnt = m * L.ldn; l = L.ldn; eb = 2; break;
         case NQ_FIELD_WHAT_LO: off = L.whatL; cnt = m * L.ldn; l = L.ldn; eb = 2; break;
         case NQ_FIELD_GAMMA: off = L.scal + offsetof(Scalars, gamma); cnt = 1; l = 1; eb = 8; break;
+        case NQ_FIELD_INV_STATS: off = L.ns; cnt = 3 + kNsMaxSteps + 2; l = 1; eb = 8; break;
+        case NQ_FIELD_GINV_U: off = L.gih[0]; cnt = (int64_t)r * L.ldr; l = L.ldr; eb = 2; break;
+        case NQ_FIELD_GINV_U_LO: off = L.gil[0]; cnt = (int64_t)r * L.ldr; l = L.ldr; eb = 2; break;
+        case NQ_FIELD_GINV_V: off = L.gih[1]; cnt = (int64_t)r * L.ldr; l = L.ldr; eb = 2; break;
+        case NQ_FIELD_GINV_V_LO: off = L.gil[1]; cnt = (int64_t)r * L.ldr; l = L.ldr; eb = 2; break;
         default: return NQ_ERR_INVALID_ARG;
     }
     *dev_ptr = static_cast<char *>(ws) + off;

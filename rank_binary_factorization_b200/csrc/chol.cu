@@ -46,6 +46,8 @@ struct Chol2Args {
     unsigned int *cnt;  // 2 x nb x nb: operations completed on tile (i, k) of L, of L^-1
     int *err;
     unsigned int *bar;
+    const int *gate;    // when set, the launch returns at once if bit (*gate) of
+    int gate_skip;      // gate_skip is set
 };
 
 // ---- tile movement (L2-coherent loads: other CTAs write the tiles between tasks) -----
@@ -372,6 +374,11 @@ __device__ __forceinline__ void signal_count(unsigned int *c, unsigned int inc) 
 }
 
 __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
+    // every CTA reads the same word before any wait: all return, or none
+    if (p.gate) {
+        const int g = *reinterpret_cast<const volatile int *>(p.gate);
+        if ((unsigned)g < 32u && ((p.gate_skip >> g) & 1)) return;
+    }
     extern __shared__ __align__(16) float smem_f[];
     Tile &t0 = *reinterpret_cast<Tile *>(smem_f);
     Tile &t1 = *reinterpret_cast<Tile *>(smem_f + TB * LDS);
@@ -642,7 +649,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
-                         cudaStream_t s) {
+                         const int *gate, int gate_skip, cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
     constexpr int smem = (5 * TB * LDS + TB) * sizeof(float);
     // grid of the cooperative launch (one CTA per SM), per device
@@ -668,7 +675,7 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
     const int nb = (int)(rp / TB);
     e = cudaMemsetAsync(flags, 0, (size_t)2 * nb * nb * sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    Chol2Args args{G, r, nb, rp, A, Li, Gi_hi, Gi_lo, ldr, flags, err, bar};
+    Chol2Args args{G, r, nb, rp, A, Li, Gi_hi, Gi_lo, ldr, flags, err, bar, gate, gate_skip};
     void *params[] = {&args};
     count_launch();
     return cudaLaunchCooperativeKernel((const void *)chol2_kernel, dim3(grid), dim3(256), params,

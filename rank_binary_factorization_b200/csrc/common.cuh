@@ -46,6 +46,13 @@ __device__ __forceinline__ float bf16_round(float x) {
     return __bfloat162float(__float2bfloat16_rn(x));
 }
 
+// x as hi + lo BF16 (hi = RNE of x, lo = RNE of the remainder).
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 *hi, __nv_bfloat16 *lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    *hi = h;
+    *lo = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
 // Warp-level sum.
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

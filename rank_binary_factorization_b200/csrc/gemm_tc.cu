@@ -160,7 +160,8 @@ __device__ __forceinline__ void split_mirror(const EpiParams &p, int row, int co
 }
 
 // Mirrored store of a symmetric Gram tile (EPI_GRAM with sym): entry (row, col0 + j) also
-// goes to (col0 + j, row).  Off-diagonal tiles only, so no ridge term is added here.
+// goes to (col0 + j, row), and to its hi + lo split when Rhi is set.  Off-diagonal tiles
+// only, so no ridge term is added here.
 __device__ __forceinline__ void gram_mirror(const EpiParams &p, int row, int col0,
                                             const float (&v)[16]) {
 #pragma unroll
@@ -168,12 +169,37 @@ __device__ __forceinline__ void gram_mirror(const EpiParams &p, int row, int col
         if (col0 + j >= p.N) break;
         p.out[(int64_t)(col0 + j) * p.ldo + row] = v[j];
     }
+    if (p.Rhi) split_mirror(p, row, col0, v);
+}
+
+// Row segment (row, col0 .. col0 + 15) of a split (hi + lo BF16) output; ``full``: all 16
+// columns are inside the matrix (then two 32-byte stores per part).
+__device__ __forceinline__ void split_store(__nv_bfloat16 *hi, __nv_bfloat16 *lo, bool full,
+                                            int ncols, const float (&v)[16]) {
+    if (full) {
+        __align__(16) __nv_bfloat16 h[16], l[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            h[j] = __float2bfloat16_rn(v[j]);
+            l[j] = __float2bfloat16_rn(v[j] - __bfloat162float(h[j]));
+        }
+        reinterpret_cast<uint4 *>(hi)[0] = reinterpret_cast<uint4 *>(h)[0];
+        reinterpret_cast<uint4 *>(hi)[1] = reinterpret_cast<uint4 *>(h)[1];
+        reinterpret_cast<uint4 *>(lo)[0] = reinterpret_cast<uint4 *>(l)[0];
+        reinterpret_cast<uint4 *>(lo)[1] = reinterpret_cast<uint4 *>(l)[1];
+    } else {
+        for (int j = 0; j < 16 && j < ncols; ++j) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+            hi[j] = h;
+            lo[j] = __float2bfloat16_rn(v[j] - __bfloat162float(h));
+        }
+    }
 }
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int col0,
                                                const float (&v)[16], float &acc_sum,
-                                               float &acc_aux) {
+                                               float &acc_aux, bool fin) {
     const bool full = (col0 + 16 <= p.N);
     if constexpr (EPI == EPI_GRAM) {
         float *o = p.out + (int64_t)row * p.ldo + col0;
@@ -187,6 +213,41 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
             for (int j = 0; j < 16; ++j)
                 if (full || col0 + j < p.N) o[j] = w[j];
         }
+        if (p.Rhi) {
+            const int64_t so = (int64_t)row * p.ldr + col0;
+            split_store(p.Rhi + so, p.Rlo + so, full, p.N - col0, w);
+        }
+    } else if constexpr (EPI == EPI_NS1) {
+        const int64_t so = (int64_t)row * p.ldr + col0;
+        float e[16];
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            e[j] = (row == col0 + j ? 1.f : 0.f) - v[j];
+            if (full || col0 + j < p.N) part += e[j] * e[j];
+        }
+        split_store(p.Rhi + so, p.Rlo + so, full, p.N - col0, e);
+        acc_sum += part;
+    } else if constexpr (EPI == EPI_NS2) {
+        const int64_t so = (int64_t)row * p.ldr + col0;
+        float xh[16], xl[16], xn[16];
+        if (full) {
+            ld16_bf16(xh, p.Ph + so);
+            ld16_bf16(xl, p.Pl + so);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const bool in = col0 + j < p.N;
+                xh[j] = in ? __bfloat162float(p.Ph[so + j]) : 0.f;
+                xl[j] = in ? __bfloat162float(p.Pl[so + j]) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xn[j] = (xh[j] + xl[j]) + v[j];
+        if (fin)
+            split_store(p.Fhi + so, p.Flo + so, full, p.N - col0, xn);
+        else
+            split_store(p.Rhi + so, p.Rlo + so, full, p.N - col0, xn);
     } else if constexpr (EPI == EPI_SCALE) {
         float *o = p.out + (int64_t)row * p.ldo + col0;
         for (int j = 0; j < 16 && col0 + j < p.N; ++j) o[j] = v[j] * p.s1[col0 + j];
@@ -373,6 +434,65 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
     }
 }
 
+// Newton-Schulz bookkeeping, run by one epilogue warp per finished tile.  NS1: the tile's
+// sum of squared residual entries goes to part[tile]; the warp that finishes the last tile
+// of the launch (ticket) sums the partials in a fixed order and moves the gate.  NS2: the
+// last tile closes an accepted update.
+template <int EPI>
+__device__ __forceinline__ void ns_tile_done(const EpiParams &p, int tile, int num_tiles,
+                                             int lane, const double *red, bool fin) {
+    NsState *ns = p.ns;
+    unsigned last = 0;
+    if (lane == 0) {
+        if constexpr (EPI == EPI_NS1) {
+            double t = 0.0;
+            for (int e = 0; e < kEpiWarps; ++e) t += red[e];
+            p.part[tile] = t;
+        }
+        __threadfence();
+        last = atomicAdd(&ns->ticket, 1u) == (unsigned)(num_tiles - 1) ? 1u : 0u;
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence();
+    if constexpr (EPI == EPI_NS1) {
+        double t = 0.0;
+        for (int i = lane; i < num_tiles; i += 32) t += __ldcg(p.part + i);
+        t = warp_sum(t);
+        if (lane == 0) {
+            const int k = p.ns_step;
+            const double ef = t >= 0.0 ? sqrt(t) : -1.0;   // a timed-out tile left NaN/-1
+            ns->ef[k] = ef;
+            // the first split step (k == ns_min_final) starts from an iterate at the BF16
+            // steps' rounding floor, so its residual is not compared with theirs; within
+            // the BF16 steps only growth is a failure (a floor may already be reached)
+            const double prev = k > 0 ? ns->ef[k - 1] : 0.0;
+            int g = NS_RUNNING;
+            if (!(ef >= 0.0 && ef < 1e30))
+                g = NS_FAIL;
+            else if (k >= p.ns_min_final && ef <= (double)p.ns_tau)
+                g = NS_FINAL;
+            else if (k >= p.ns_last || (k > p.ns_min_final && ef > 0.9 * prev) ||
+                     (k > 0 && k < p.ns_min_final && ef > 1.5 * prev))
+                g = NS_FAIL;
+            if (g == NS_FAIL) ns->fallbacks += 1;
+            ns->ticket = 0;
+            __threadfence();
+            *reinterpret_cast<volatile int *>(&ns->gate) = g;
+        }
+    } else {
+        if (lane == 0) {
+            if (fin) {
+                ns->accepted += 1;
+                ns->steps = p.ns_step + 1;
+            }
+            ns->ticket = 0;
+            __threadfence();
+            if (fin) *reinterpret_cast<volatile int *>(&ns->gate) = NS_DONE;
+        }
+    }
+}
+
 // Output tile -> (m0, n0).  Plain: m fastest.  Symmetric (BN == BM): the lower-triangular
 // tiles (tm >= tn) row by row, so tiles come in order of decreasing K range under tri_k.
 template <int BN>
@@ -395,12 +515,26 @@ __device__ __forceinline__ void tile_origin(const EpiParams &p, int tile, int nu
 // consecutive CTAs share the B tile).  Two TMEM accumulator stages let the epilogue
 // of one tile run while the MMAs of the next are issued.
 // ---------------------------------------------------------------------------------
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, bool F3>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ Maps maps, const EpiParams p) {
     constexpr int B_TILE_BYTES = BN * BK * 2;
-    constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+    // F3 (split3): a stage holds A_hi, A_lo, B_hi, B_lo of one k-block and takes the three
+    // products hi.hi, lo.hi, hi.lo; otherwise one A and one B tile of one segment
+    constexpr int STAGE_BYTES = (F3 ? 2 : 1) * (A_TILE_BYTES + B_TILE_BYTES);
     constexpr uint32_t TMEM_COLS = 2 * BN;
+
+    // gate: the whole launch is skipped on the gate values in gate_skip
+    int gate_v = 0;
+    if (p.gate) {
+        gate_v = *reinterpret_cast<const volatile int *>(p.gate);
+        if ((unsigned)gate_v < 32u && ((p.gate_skip >> gate_v) & 1)) return;
+    }
+    const bool fin = (EPI == EPI_NS2) && gate_v == NS_FINAL;
+    if (EPI == EPI_GRAM && p.ns && blockIdx.x == 0 && threadIdx.x == 0) {
+        p.ns->ticket = 0;
+        *reinterpret_cast<volatile int *>(&p.ns->gate) = NS_RUNNING;
+    }
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -416,8 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int num_m = (int)ceil_div(p.M, BM);
     const int num_tiles = p.sym ? num_m * (num_m + 1) / 2 : num_m * (int)ceil_div(p.N, BN);
-    const int total_kb = p.kblocks[0] + (p.nseg > 1 ? p.kblocks[1] : 0) +
-                         (p.nseg > 2 ? p.kblocks[2] : 0);
+    const int total_kb = F3 ? p.kblocks[0]
+                            : p.kblocks[0] + (p.nseg > 1 ? p.kblocks[1] : 0) +
+                                  (p.nseg > 2 ? p.kblocks[2] : 0);
     // split-K: work unit u = (split u / num_tiles, tile u % num_tiles); split s covers the
     // k-blocks [s * kchunk, (s + 1) * kchunk) of the concatenated segments
     const int ksplit = p.ksplit > 1 ? p.ksplit : 1;
@@ -459,7 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tile_origin<BN>(p, tile, num_m, m0, n0);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     int seg = 0, k = kb;
-                    while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                    if (!F3)
+                        while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
                     if (p.tri_k && k < (m0 > n0 ? m0 : n0) / BK) continue;
                     const int s = it % STAGES;
                     if (it >= STAGES &&
@@ -469,8 +605,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t *a_dst = smem + s * STAGE_BYTES;
                     mbar_expect_tx(&full_bar[s], STAGE_BYTES);
-                    tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
-                    tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0, &full_bar[s]);
+                    if constexpr (F3) {
+                        uint8_t *b_dst = a_dst + 2 * A_TILE_BYTES;
+                        tma_load_2d(a_dst, &maps.a[0], k * BK, m0, &full_bar[s]);
+                        tma_load_2d(a_dst + A_TILE_BYTES, &maps.a[1], k * BK, m0, &full_bar[s]);
+                        tma_load_2d(b_dst, &maps.b[0], k * BK, n0, &full_bar[s]);
+                        tma_load_2d(b_dst + B_TILE_BYTES, &maps.b[1], k * BK, n0, &full_bar[s]);
+                    } else {
+                        tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
+                        tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0,
+                                    &full_bar[s]);
+                    }
                     ++it;
                 }
             }
@@ -495,7 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (p.tri_k) {
                         int seg = 0, k = kb;
-                        while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                        if (!F3)
+                            while (seg < p.nseg - 1 && k >= p.kblocks[seg])
+                                k -= p.kblocks[seg++];
                         if (k < (m0 > n0 ? m0 : n0) / BK) continue;
                     }
                     const int s = it % STAGES;
@@ -505,11 +652,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint8_t *a_src = smem + s * STAGE_BYTES;
-                    const uint64_t adesc = smem_desc_sw128(a_src);
-                    const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
+                    if constexpr (F3) {
+                        const uint64_t ah = smem_desc_sw128(a_src);
+                        const uint64_t al = smem_desc_sw128(a_src + A_TILE_BYTES);
+                        const uint64_t bh = smem_desc_sw128(a_src + 2 * A_TILE_BYTES);
+                        const uint64_t bl = smem_desc_sw128(a_src + 2 * A_TILE_BYTES + B_TILE_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16(d, ah + 2 * k, bh + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) mma_bf16(d, al + 2 * k, bh + 2 * k, idesc, 1u);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) mma_bf16(d, ah + 2 * k, bl + 2 * k, idesc, 1u);
+                    } else {
+                        const uint64_t adesc = smem_desc_sw128(a_src);
+                        const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                     (first && k == 0) ? 0u : 1u);
+                    }
                     mma_commit(&empty_bar[s]);
                     first = false;
                     ++it;
@@ -549,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // split-K partial: the unit's raw 128 x 128 tile, reduced later
                         st16(p.out + ((int64_t)unit * BM + 32 * q + lane) * BM + c, v);
                     } else if (row < p.M && n0 + c < p.N) {
-                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum, acc_aux);
+                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum, acc_aux, fin);
                         if constexpr (EPI == EPI_SPLIT)
                             if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
                         if constexpr (EPI == EPI_GRAM)
@@ -567,6 +729,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     p.num[o] = (double)acc_sum;
                     p.den[o] = (double)acc_aux;
                 }
+            }
+            if constexpr (EPI == EPI_NS1 || EPI == EPI_NS2) {
+                if constexpr (EPI == EPI_NS1) {
+                    const double w = warp_sum((double)acc_sum);
+                    if (lane == 0) red[as][warp - 2] = dead ? __longlong_as_double(-1ll) : w;
+                    epilogue_bar();
+                }
+                if (warp == 2) ns_tile_done<EPI>(p, tile, num_tiles, lane, red[as], fin);
             }
             if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
                 if (p.part && (EPI == EPI_RECON || p.objective)) {
@@ -624,10 +794,11 @@ bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t col
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, bool F3>
 static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s) {
-    constexpr int smem = STAGES * (A_TILE_BYTES + BN * BK * 2) + 1024 + 256;  // + barriers
-    auto kern = gemm_kernel<BN, STAGES, EPI>;
+    constexpr int smem = STAGES * (F3 ? 2 : 1) * (A_TILE_BYTES + BN * BK * 2) + 1024 + 256;
+    static_assert(smem <= 227 * 1024, "shared memory of a GEMM stage ring");
+    auto kern = gemm_kernel<BN, STAGES, EPI, F3>;
     static std::atomic<uint64_t> configured{0};   // devices whose smem limit is set
     cudaError_t e = ensure_smem_limit((const void *)kern, smem, configured);
     if (e != cudaSuccess) return e;
@@ -644,10 +815,22 @@ static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s
 
 template <int EPI>
 static cudaError_t launch_bn(const Maps &maps, const EpiParams &p, int BN, cudaStream_t s) {
+    if (p.split3) {
+        if constexpr (EPI == EPI_RECON || EPI == EPI_SCALE || EPI == EPI_REFIT) {
+            return cudaErrorInvalidValue;
+        } else {
+            switch (BN) {
+                case 64: return launch_t<64, 4, EPI, true>(maps, p, s);
+                case 128: return launch_t<128, 3, EPI, true>(maps, p, s);
+                case 256: return launch_t<256, 2, EPI, true>(maps, p, s);
+                default: return cudaErrorInvalidValue;
+            }
+        }
+    }
     switch (BN) {
-        case 64: return launch_t<64, 8, EPI>(maps, p, s);
-        case 128: return launch_t<128, 6, EPI>(maps, p, s);
-        case 256: return launch_t<256, 4, EPI>(maps, p, s);
+        case 64: return launch_t<64, 8, EPI, false>(maps, p, s);
+        case 128: return launch_t<128, 6, EPI, false>(maps, p, s);
+        case 256: return launch_t<256, 4, EPI, false>(maps, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -662,6 +845,8 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_SPLIT: return launch_bn<EPI_SPLIT>(maps, p, BN, s);
         case EPI_SCALE: return launch_bn<EPI_SCALE>(maps, p, BN, s);
         case EPI_REFIT: return launch_bn<EPI_REFIT>(maps, p, BN, s);
+        case EPI_NS1: return launch_bn<EPI_NS1>(maps, p, BN, s);
+        case EPI_NS2: return launch_bn<EPI_NS2>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
 }

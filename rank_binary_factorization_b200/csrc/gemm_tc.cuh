@@ -1,7 +1,9 @@
 // tcgen05 / TMEM / TMA GEMM for sm_100a with fused LB-ADMM epilogues.
 //
 // D[M x N] = sum over K-segments s of A_s[M x K_s] . B_s[N x K_s]^T, all operands BF16
-// and K-major (row-major with K contiguous), accumulation FP32 in tensor memory.
+// and K-major (row-major with K contiguous), accumulation FP32 in tensor memory.  With
+// split3 the three products of split operands (hi.hi + lo.hi + hi.lo) share one stage of
+// four tiles per k-block, so each operand tile is loaded once.
 // Persistent: one CTA per SM walks 128 x BN output tiles round-robin.  Per CTA:
 //   warp 0     one elected thread issues TMA tile loads into a STAGES-deep ring
 //   warp 1     allocates TMEM (two accumulator stages of BN columns); one elected thread
@@ -14,6 +16,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "layout.h"
 
 namespace nq {
 namespace tc {
@@ -25,7 +28,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4,
-                 EPI_SCALE = 5, EPI_REFIT = 6 };
+                 EPI_SCALE = 5, EPI_REFIT = 6, EPI_NS1 = 7, EPI_NS2 = 8 };
 
 struct Maps {
     CUtensorMap a[3];
@@ -36,6 +39,9 @@ struct EpiParams {
     int M, N;
     int nseg;
     int kblocks[3];
+    int split3;         // split (hi + lo) operands in one pass over K: A_hi = maps.a[0],
+                        // A_lo = maps.a[1], B_hi = maps.b[0], B_lo = maps.b[1]; D = the sum of
+                        // hi.hi + lo.hi + hi.lo over kblocks[0] k-blocks
     int tri_k;          // operands zero for k < row index: start each tile's K at max(m0, n0)
     int sym;            // symmetric result (EPI_SPLIT / EPI_GRAM, BN == BM, M == N): lower-
                         // triangular tiles only, each off-diagonal tile also written mirrored
@@ -46,7 +52,13 @@ struct EpiParams {
                         // out + u * 128 * 128 (row-major, ld 128) for a later reduction.
                         // Every part must get at least one k-block.
     int *err;
-    // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0)
+    // Gate: when set, the whole launch returns at once if bit (*gate) of gate_skip is set
+    // (the word is read once by every thread before any other work)
+    const int *gate;
+    int gate_skip;
+    // EPI_GRAM: out[row*ldo + col] = acc + (row == col ? diag : 0); when Rhi is set, the
+    // same value also split into hi + lo BF16 (Rhi/Rlo, ld ldr); when ns is set, CTA 0
+    // opens the Newton-Schulz gate of the half step (ns->gate = NS_RUNNING)
     float *out;
     int64_t ldo;
     float diag;
@@ -85,6 +97,23 @@ struct EpiParams {
     int refit_trans;
     const float *sv;
     double *num, *den;
+    // Newton-Schulz step k (ns_step) towards G^-1 from X_k, in the form
+    // X_{k+1} = X_k (2I - G X_k) = X_k + E_k X_k with E_k = I - X_k G:
+    // EPI_NS1: acc = (X_k G)(row, col); E_k = delta - acc split into Rhi/Rlo; the tile's
+    //   sum of E_k entries squared goes to part[tile]; the CTA finishing the last tile
+    //   forms ||E_k||_F and moves ns->gate: NS_FINAL if k >= ns_min_final and it is
+    //   <= ns_tau; NS_FAIL if it is not finite, if k == ns_last without NS_FINAL, if it
+    //   grew above 1.5 x the previous step's during the BF16 steps (k < ns_min_final),
+    //   or did not fall below 0.9 x the previous step's after the first split step
+    //   (k > ns_min_final).
+    // EPI_NS2: acc = (E_k X_k)(row, col); X_{k+1} = (Ph + Pl) + acc split into hi + lo,
+    //   written to Rhi/Rlo, or to Fhi/Flo when the gate reads NS_FINAL (then the CTA
+    //   finishing the last tile sets NS_DONE).
+    NsState *ns;
+    int ns_step, ns_last, ns_min_final;
+    float ns_tau;
+    const __nv_bfloat16 *Ph, *Pl;   // X_k (hi, lo), ld ldr
+    __nv_bfloat16 *Fhi, *Flo;       // destination of the final iterate, ld ldr
 };
 
 // Host: encode a 2-D BF16 tensor map over rows x cols (row stride ld elements) with

@@ -781,7 +781,8 @@ cudaError_t svid(const float *S, int64_t rows, int32_t r, int64_t ldf, int K, in
 // result does not depend on the order in which the GEMM's CTAs finished.
 // =================================================================================
 __global__ void __launch_bounds__(256)
-    gram_reduce_kernel(const float *__restrict__ P, int T, int S, int r, float diag, float *G) {
+    gram_reduce_kernel(const float *__restrict__ P, int T, int S, int r, float diag, float *G,
+                       __nv_bfloat16 *Gh, __nv_bfloat16 *Gl, int64_t ldg) {
     __shared__ float tr[32][33];
     const int t = blockIdx.x;
     int a = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
@@ -797,20 +798,29 @@ __global__ void __launch_bounds__(256)
         for (int sp = 0; sp < S; ++sp) v += P[((int64_t)(sp * T + t) * 128 + li) * 128 + lj];
         const int gi = m0 + li, gj = n0 + lj;
         if (gi == gj) v += diag;
-        if (gi < r && gj < r) G[(int64_t)gi * r + gj] = v;
+        if (gi < r && gj < r) {
+            G[(int64_t)gi * r + gj] = v;
+            if (Gh) split_bf16(v, Gh + (int64_t)gi * ldg + gj, Gl + (int64_t)gi * ldg + gj);
+        }
         tr[k][tx] = v;
     }
     if (a != b) {
         __syncthreads();
         for (int k = ty; k < 32; k += 8) {
             const int gi = n0 + sj + k, gj = m0 + si + tx;   // mirror of tile entry (si+tx, sj+k)
-            if (gi < r && gj < r) G[(int64_t)gi * r + gj] = tr[tx][k];
+            if (gi < r && gj < r) {
+                G[(int64_t)gi * r + gj] = tr[tx][k];
+                if (Gh)
+                    split_bf16(tr[tx][k], Gh + (int64_t)gi * ldg + gj,
+                               Gl + (int64_t)gi * ldg + gj);
+            }
         }
     }
 }
 
-cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G, cudaStream_t s) {
-    gram_reduce_kernel<<<dim3((unsigned)T, 16), 256, 0, s>>>(P, T, S, r, diag, G);
+cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G,
+                        __nv_bfloat16 *Gh, __nv_bfloat16 *Gl, int64_t ldg, cudaStream_t s) {
+    gram_reduce_kernel<<<dim3((unsigned)T, 16), 256, 0, s>>>(P, T, S, r, diag, G, Gh, Gl, ldg);
     count_launch();
     return cudaGetLastError();
 }

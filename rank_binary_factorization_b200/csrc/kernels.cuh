@@ -48,10 +48,12 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 // G = L L^T for the SPD r x r matrix G (row stride r); writes (L^-1)^T as hi + lo bf16
 // [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: 2 (rp/64)^2 counters.
 // max_ctas > 0 limits the cooperative grid (at least 3 CTAs); 0: one CTA per SM.
+// gate: optional device word; the launch does nothing when bit (*gate) of gate_skip is
+// set at its start.
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *LiT_hi, __nv_bfloat16 *LiT_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
-                         cudaStream_t s);
+                         const int *gate, int gate_skip, cudaStream_t s);
 
 // ---- SVID -------------------------------------------------------------------------
 // K power steps on |S| (S rows x r, row stride ldf): a = t/||t||, b = A^T t / ||t||.
@@ -78,7 +80,9 @@ cudaError_t bin_expand(const uint32_t *Up, const uint32_t *Vp, const float *s2, 
 // ---- split-K Gram reduction ------------------------------------------------------
 // G (r x r) = sum_{s < S} P[s * T + t] (raw 128 x 128 lower-triangular tiles t < T) +
 // diag I, each off-diagonal tile also stored mirrored.
-cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G, cudaStream_t s);
+// Gh/Gl (optional, ld ldg): the same Gram split into hi + lo BF16.
+cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G,
+                        __nv_bfloat16 *Gh, __nv_bfloat16 *Gl, int64_t ldg, cudaStream_t s);
 
 // ---- objective --------------------------------------------------------------------
 // obj[slot] = (what_n2 - 2 sum(px) + <GU - cI, GV - cI>) / what_n2

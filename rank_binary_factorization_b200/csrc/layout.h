@@ -34,6 +34,23 @@ inline int gram_ksplit(int32_t r, int64_t K, int nseg, int sms) {
 }
 constexpr int64_t kMaxDim = 65536;
 
+// Newton-Schulz update of G^-1 (see NsState): at most kNsMaxSteps steps, the first
+// kNsBf16Steps of them with plain BF16 operands, the rest split (hi + lo).
+constexpr int kNsMaxSteps = 6;
+constexpr int kNsBf16Steps = 2;
+enum NsGate : int { NS_RUNNING = 0, NS_FINAL = 1, NS_DONE = 2, NS_FAIL = 3 };
+
+// State of the Newton-Schulz inverse update of one half step (8-byte words first: the
+// first 11 words are readable as a state field).
+struct NsState {
+    unsigned long long accepted;   // half steps whose inverse came from the update
+    unsigned long long fallbacks;  // attempts that fell back to the Cholesky factorisation
+    long long steps;               // steps of the last accepted update
+    double ef[kNsMaxSteps + 2];    // ||I - X_k G||_F of the last attempt, step by step
+    int gate;                      // NsGate of the running half step
+    unsigned int ticket;           // finished tiles of the running launch
+};
+
 // Scalars block at the start of every workspace.
 struct Scalars {
     double gamma;        // ||W~||_F / (2 sqrt r)
@@ -56,7 +73,8 @@ struct LbLayout {
     int nsv = 0;       // CTAs of an SVID pass (rows of its partial array)
     size_t scal = 0, what = 0, whatT = 0, whatL = 0, whatTL = 0, x[2] = {0, 0}, s[2] = {0, 0},
            a[2] = {0, 0}, b[2] = {0, 0}, xt[2] = {0, 0}, xtl[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
-           gih = 0, gil = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
+           gih[2] = {0, 0}, gil[2] = {0, 0}, gsh = 0, gsl = 0, nqh[2] = {0, 0}, nql[2] = {0, 0},
+           nth = 0, ntl = 0, nspart = 0, ns = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
            partb = 0, obj = 0, gpart = 0, total = 0;
     size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
 
@@ -100,8 +118,21 @@ struct LbLayout {
         rlo = take((size_t)maxrows * ldr * 2);
         chA = take((size_t)rp * rp * 4);
         chLi = take((size_t)rp * rp * 4);
-        gih = take((size_t)r * ldr * 2);
-        gil = take((size_t)r * ldr * 2);
+        // G^-1 of each side's solve (hi + lo), kept as the start of that side's next
+        // Newton-Schulz update; the Gram split into hi + lo; the update's iterates and its
+        // products X G
+        for (int sd = 0; sd < 2; ++sd) {
+            gih[sd] = take((size_t)r * ldr * 2);
+            gil[sd] = take((size_t)r * ldr * 2);
+            nqh[sd] = take((size_t)r * ldr * 2);
+            nql[sd] = take((size_t)r * ldr * 2);
+        }
+        gsh = take((size_t)r * ldr * 2);
+        gsl = take((size_t)r * ldr * 2);
+        nth = take((size_t)r * ldr * 2);
+        ntl = take((size_t)r * ldr * 2);
+        nspart = take((size_t)((r + 127) / 128) * ((r + 63) / 64) * 8);
+        ns = take(sizeof(NsState));
         lth = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 hi
         ltl = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 lo
         chF = take((size_t)2 * (rp / 64) * (rp / 64) * 4);  // Cholesky / inverse tile counters
