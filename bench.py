@@ -134,15 +134,15 @@ class ClockSampler:
                     reasons=sorted(reasons))
 
 
-def kernel_units(cls, m, n, r, K, T):
+def kernel_units(cls, m, n, r, K, T, ns_steps=4):
     """Algorithmic work of one launch scope of a kernel class: (amount, unit, bound).
 
     Per launch scope, averaged over the two sides where they differ.  "chol" counts the
     method's own work, one Cholesky factorisation (r^3 / 3); the triangular inverse the
     library also forms there is executed work beyond it.  "ginv" is the product
     L^-T L^-1 of two triangular factors (r^3 / 3).  "newton" (the Newton-Schulz update
-    of G^-1 that replaces the factorisation once G changes little) is credited with the
-    explicit inverse it replaces (r^3)."""
+    of G^-1 that replaces the factorisation once G changes little) counts its own two
+    r x r x r products per step."""
     if cls == "calib":
         return T * (m + n), "B", "hbm"   # per launch: mean of the two BF16 streams (T x n, T x m)
     if cls == "rhs":
@@ -156,10 +156,9 @@ def kernel_units(cls, m, n, r, K, T):
     if cls == "ginv":
         return float(r) ** 3 / 3.0, "FLOP", "tensor"         # L^-T L^-1
     if cls == "newton":
-        # the update stands in for forming G^-1 explicitly (Cholesky r^3/3, triangular
-        # inverse r^3/3, L^-T L^-1 r^3/3); its own steps execute 4 r^3 each (two r x r
-        # products), in BF16 or split BF16
-        return float(r) ** 3, "FLOP", "tensor"
+        # two r x r x r products (2 r^3 each) per step of the update, ns_steps steps (the
+        # last accepted update's count); the split passes of the residual are not counted
+        return 4.0 * float(r) ** 3 * max(ns_steps, 1), "FLOP", "tensor"
     if cls == "svid":
         # K reads of S (FP32).  Inside nq_lbadmm the SVID passes run on an auxiliary
         # stream beside the next RHS GEMM and solve, so this class's time is elapsed time
@@ -178,8 +177,21 @@ def ncu_traffic(cls, m, n, r, T):
     return None
 
 
-def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks):
-    u = kernel_units(cls, m, n, r, K, T)
+def inverse_update_steps(nq, ws, m, n, r):
+    """Steps of the last accepted Newton-Schulz update of G^-1 in workspace ``ws``."""
+    import ctypes
+    import torch
+    p, c, e, ld = ctypes.c_void_p(), ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int64()
+    nq.check("nq_lbadmm_state_field", nq.lib.nq_lbadmm_state_field(
+        m, n, r, nq._lib.FIELDS["INV_STATS"], ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+        ctypes.byref(p), ctypes.byref(c), ctypes.byref(e), ctypes.byref(ld)))
+    off = p.value - ws.data_ptr()
+    words = ws[off:off + c.value * e.value].view(torch.int64).cpu()
+    return int(words[2])
+
+
+def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks, ns_steps=4):
+    u = kernel_units(cls, m, n, r, K, T, ns_steps)
     if u is None or launches == 0 or ms <= 0:
         return None
     amount, unit, bound = u
@@ -387,7 +399,6 @@ def run_ours(args):
     clocks = ClockSampler(local_rank)
     barrier(device)
     torch.cuda.synchronize()
-    nq.nq_profile_enable(True)
     launches0 = nq.nq_launch_count()
     clocks.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -400,10 +411,23 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(device)
     launches = nq.nq_launch_count() - launches0
+    t = reduce_max(ev0.elapsed_time(ev1) / 1e3, device)
+
+    # the same steps again with the library's per-class CUDA event pairs on its launching
+    # streams (the kernel roofline entries); the event records between kernels cost time
+    # of their own, so the headline value above is taken without them
+    torch.cuda.synchronize()
+    nq.nq_profile_enable(True)
+    evp0, evp1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evp0.record(stream)
+    for _ in range(args.steps):
+        res = step()
+    evp1.record(stream)
+    evp1.synchronize()
+    torch.cuda.synchronize()
     prof = nq.nq_profile_get()
     nq.nq_profile_enable(False)
-    t_local = ev0.elapsed_time(ev1) / 1e3
-    t = reduce_max(t_local, device)
+    t_local = evp0.elapsed_time(evp1) / 1e3
 
     # end-to-end through the public API with pinned host buffers
     for _ in range(1):
@@ -424,8 +448,9 @@ def run_ours(args):
     peaks = read_peaks()
     step_ms = t / args.steps * 1e3
     entries = {}
+    ns_steps = inverse_update_steps(nq, lb_ws, m, n, r)
     for cls, (nl, ms) in prof.items():
-        e = roofline_entry(cls, nl, ms, m, n, r, K, T, peaks)
+        e = roofline_entry(cls, nl, ms, m, n, r, K, T, peaks, ns_steps)
         if e is not None:
             e["share_of_step"] = round(ms / (t_local * 1e3), 4)
             if cls == "svid":
@@ -459,6 +484,7 @@ def run_ours(args):
         calib_gbs=calib["achieved"] if calib else None,
         roofline=dominant,
         kernels=entries,
+        profiled_ms_per_step=round(t_local / args.steps * 1e3, 3),
         peaks_source=peaks["source"],
         gpu_launches=int(launches),
         clocks=clk,

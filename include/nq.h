@@ -159,8 +159,9 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  *   G^-1 = L^-T L^-1 (split-BF16 tensor-core GEMM).
  * NQ_INV_NEWTON: first a Newton-Schulz update of the inverse this side used in its
  *   previous half step, X_{k+1} = X_k + (I - X_k G) X_k (two r x r tensor-core GEMMs per
- *   step; the first two steps with BF16 operands, the later ones split BF16), at most 6
- *   steps; the iterate after the step whose ||I - X_k G||_F is <= 1e-2 is taken (so
+ *   step: the residual I - X_k G with BF16 operands in the first two steps and split BF16
+ *   in the later ones, the correction with BF16 operands), at most 6 steps; the iterate
+ *   after the step whose ||I - X_k G||_F is <= 1e-2 is taken (so
  *   ||I - X G||_2 <= 1e-4 up to rounding).  An update whose residual does not shrink,
  *   or that reaches no such step, is dropped and the Cholesky path runs instead, decided
  *   on the device (no synchronisation).
@@ -172,6 +173,22 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  */
 typedef enum { NQ_INV_AUTO = 0, NQ_INV_CHOLESKY = 1, NQ_INV_NEWTON = 2 } nq_inverse_mode;
 nq_status nq_set_inverse_mode(nq_inverse_mode mode);
+
+/*
+ * Scheduling settings of the LB-ADMM iterations (process-wide; none changes a result):
+ * NQ_TUNE_FACTOR_CTAS: CTAs given to forming G^-1 (factorisation or update) while the
+ *   RHS GEMM runs on the other SMs: -1 (default) half of the SMs up to r = 1536, else no
+ *   overlap; 0 no overlap; n >= 1: n CTAs (at least 3, at most all SMs but one).
+ * NQ_TUNE_NEWTON_BN: tile width of the update's GEMMs: 0 (default) the fewest waves x
+ *   width on the CTAs it gets, or 64, 128, 256.
+ * NQ_TUNE_SVID_BESIDE: 1 (default) the SVID passes of a side run on an auxiliary stream
+ *   beside the next half step's GEMMs; 0: right after the side's solve.
+ * Returns NQ_ERR_INVALID_ARG for an unknown key or value.
+ */
+typedef enum {
+    NQ_TUNE_FACTOR_CTAS = 0, NQ_TUNE_NEWTON_BN = 1, NQ_TUNE_SVID_BESIDE = 2, NQ_TUNE_COUNT = 3
+} nq_tuning;
+nq_status nq_set_tuning(nq_tuning key, int32_t value);
 
 /*
  * Full LB-ADMM initialisation of one layer.

@@ -24,7 +24,7 @@ __all__ = [
     "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "nq_ls_refit", "LBState", "NQError",
     "status_string", "lib",
     "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
-    "nq_set_inverse_mode",
+    "nq_set_inverse_mode", "nq_set_tuning",
 ]
 
 
@@ -177,6 +177,11 @@ def nq_set_inverse_mode(mode):
     code = {"auto": _lib.NQ_INV_AUTO, "cholesky": _lib.NQ_INV_CHOLESKY,
             "newton": _lib.NQ_INV_NEWTON}[mode]
     check("nq_set_inverse_mode", lib.nq_set_inverse_mode(code))
+
+
+def nq_set_tuning(key, value):
+    """Scheduling setting ("factor_ctas", "newton_bn", "svid_beside"; see nq_tuning)."""
+    check("nq_set_tuning", lib.nq_set_tuning(_lib.TUNING[key], int(value)))
 
 
 def nq_launch_count():

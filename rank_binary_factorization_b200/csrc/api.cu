@@ -5,6 +5,7 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
@@ -263,9 +264,10 @@ nq_status lb_open(Lb &lb, int64_t m, int64_t n, int32_t r, void *ws, size_t ws_b
 // symmetric, so only its lower-triangular 128 x 128 tiles are computed and mirrored.  In
 // the FP32-accurate mode the operand is split (hi + lo) and the Gram takes three passes.
 // With ``ns_prep`` the Gram is also written split (hi + lo BF16) for the Newton-Schulz
-// update, and the update's gate is opened.
+// update, and the update's gate is opened; with ``zero_chol`` it also zeroes the tile
+// counters of the factorisation that follows it.
 nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s,
-                  bool ns_prep = false) {
+                  bool ns_prep = false, bool zero_chol = false) {
     const LbLayout &L = lb.L;
     const int64_t K = L.rows(other), ld = L.ld_rows(other);
     const __nv_bfloat16 *xt = lb.p<__nv_bfloat16>(L.xt[other]);
@@ -297,6 +299,10 @@ nq_status lb_gram(const Lb &lb, int other, float diag, int prec, cudaStream_t s,
     ep.Rlo = gl;
     ep.ldr = L.ldr;
     ep.ns = ns_prep ? lb.p<NsState>(L.ns) : nullptr;
+    if (zero_chol) {   // tile counters of the factorisation that follows
+        ep.zero = lb.p<unsigned int>(L.chF);
+        ep.zero_words = (int)(2 * (L.rp / 64) * (L.rp / 64));
+    }
     // few tiles (small r): split K so that the (tile, part) units fill the SMs; the parts
     // are summed in a fixed order by gram_reduce
     const int S = gram_ksplit(L.r, K, 1, device_sm_count());
@@ -328,7 +334,8 @@ nq_status lb_svid(const Lb &lb, int side, int K, cudaStream_t s) {
 // (Schulz 1933; Ben-Israel 1965) iteration X_{k+1} = X_k (2I - G X_k), written as
 // X_{k+1} = X_k + E_k X_k with E_k = I - X_k G, converges quadratically (E_{k+1} = E_k^2)
 // whenever the spectral radius of E_0 is below 1.  Each step is two r x r tensor-core
-// GEMMs; the first kNsBf16Steps with plain BF16 operands, the rest split (hi + lo).  The
+// GEMMs: E_k = I - X_k G in plain BF16 for the first kNsBf16Steps steps and split
+// (hi + lo) after them, E_k X_k always in plain BF16 (a correction of size |E_k|).  The
 // device decides: a step whose ||E_k||_F falls to ns_tau makes the next iterate final
 // (written to the side's G^-1); a residual that does not shrink, or no final iterate
 // after kNsMaxSteps, falls back to the Cholesky path, which then runs (gated).
@@ -337,6 +344,9 @@ constexpr int kNsFirstIter = 3;      // iterations since prepare before the firs
 constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E||_2 <= 1e-4)
 
 std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
+
+// Performance settings of nq_set_tuning (none changes a result).
+std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}};
 
 // Iterations run on each workspace since its last prepare (host side; AUTO mode).
 std::mutex g_iter_mu;
@@ -374,7 +384,8 @@ nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
     NsState *ns = lb.p<NsState>(L.ns);
     const int r = L.r;
     const int ctas = max_ctas > 0 ? max_ctas : device_sm_count();
-    const int BN = pick_bn_square(r, ctas);
+    const int bn_set = g_tune[NQ_TUNE_NEWTON_BN].load(std::memory_order_relaxed);
+    const int BN = bn_set ? bn_set : pick_bn_square(r, ctas);
     const int kb = (int)ceil_div(r, tc::BK);
     const void *gh = lb.p<void>(L.gsh), *gl = lb.p<void>(L.gsl);
     const void *eh = lb.p<void>(L.nth), *el = lb.p<void>(L.ntl);
@@ -415,14 +426,16 @@ nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
             ep.Rlo = lb.p<__nv_bfloat16>(L.ntl);
             NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_NS1, BN, s));
         }
-        {   // X_{k+1} = X_k + E_k X_k: A = E_k, B = X_k (symmetric)
+        {   // X_{k+1} = X_k + E_k X_k: A = E_k, B = X_k (symmetric).  One BF16 pass: the
+            // correction's rounding (2^-8 |E_k| |X_k|) is removed by the next step, and in
+            // the final one |E_k| <= 1e-2 keeps it below the split products' floor
             tc::Maps maps;
             memset(&maps, 0, sizeof(maps));
-            const void *as[2] = {eh, el}, *bs[2] = {xh, xl};
-            for (int g = 0; g <= split; ++g)
-                if (!tc::make_map_bf16(&maps.a[g], as[g], r, r, L.ldr, tc::BM) ||
-                    !tc::make_map_bf16(&maps.b[g], bs[g], r, r, L.ldr, BN))
-                    return NQ_ERR_CUDA;
+            if (!tc::make_map_bf16(&maps.a[0], eh, r, r, L.ldr, tc::BM) ||
+                !tc::make_map_bf16(&maps.b[0], xh, r, r, L.ldr, BN))
+                return NQ_ERR_CUDA;
+            (void)el;
+            ep.split3 = 0;
             ep.part = nullptr;
             ep.Ph = static_cast<const __nv_bfloat16 *>(xh);
             ep.Pl = static_cast<const __nv_bfloat16 *>(xl);
@@ -455,13 +468,14 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
                         (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
                          iters_since_prepare(lb.ws) >= kNsFirstIter);
     NsState *ns = lb.p<NsState>(L.ns);
-    nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton);
+    nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton, true);
     if (st) return st;
     // The factorisation of G and the G^-1 GEMM depend only on the Gram; the RHS GEMM only
     // on the other side's operand and this side's dual state.  With overlap they run at
     // once: the factorisation on ``cc`` CTAs of a side stream, the RHS GEMM on the rest.
     const int sms = device_sm_count();
-    const int cc = chol_ctas(L.r, sms);
+    const int fc = g_tune[NQ_TUNE_FACTOR_CTAS].load(std::memory_order_relaxed);
+    const int cc = fc < 0 ? chol_ctas(L.r, sms) : (fc == 0 ? 0 : std::min(std::max(fc, 3), sms - 1));
     SideCtx *sc = nullptr;
     if (cc > 0 && (st = side_ctx(&sc))) return st;
     cudaStream_t fs = s;   // stream of the factorisation
@@ -479,7 +493,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
-                           &lb.sc->err, lb.sc->bar, cc, gate, gate_skip, fs));
+                           &lb.sc->err, lb.sc->bar, cc, gate, gate_skip, false, fs));
     }
     {
         ProfScope ps(NQ_K_GINV, fs);
@@ -646,6 +660,21 @@ nq_status lb_prepare(const Lb &lb, const void *W, int bf16, const float *d_in,
     return NQ_OK;
 }
 
+// After the iterations: the objective of the last one (it needs the Gram of the last V)
+// and the copy of the objectives not copied yet.
+nq_status lb_iterate_tail(const Lb &lb, float rho, float lambda, int iters, int prec,
+                          float *objective_h, cudaStream_t s) {
+    nq_status st = lb_gram(lb, 1, lambda + rho, prec, s);
+    if (st) return st;
+    if ((st = lb_objective(lb, lambda + rho, (iters - 1) % kObjRing, s))) return st;
+    if (objective_h) {
+        const int done = (iters - 1) / kObjRing * kObjRing;
+        NQ_CK(cudaMemcpyAsync(objective_h + done, lb.p<float>(lb.L.obj),
+                              (size_t)(iters - done) * 4, cudaMemcpyDeviceToHost, s));
+    }
+    return NQ_OK;
+}
+
 // The iterations.  The SVID of the side just solved is needed only by that side's next
 // RHS GEMM, one half step later, so it runs on the auxiliary stream beside the next half
 // step's RHS GEMM and solve; the last one runs on ``s`` before returning.
@@ -654,6 +683,19 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
     SideCtx *ov = nullptr;
     nq_status st = side_ctx(&ov);
     if (st) return st;
+    if (!g_tune[NQ_TUNE_SVID_BESIDE].load(std::memory_order_relaxed)) {
+        // every SVID right after its solve, on ``s``
+        for (int t = 0; t < iters; ++t) {
+            if ((st = lb_half_step(lb, 0, rho, lambda, K, prec, s))) return st;
+            if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
+            if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s))) return st;
+            add_iters(lb.ws, 1);
+            if (objective_h && t > 0 && (t % kObjRing) == 0)
+                NQ_CK(cudaMemcpyAsync(objective_h + (t - kObjRing), lb.p<float>(lb.L.obj),
+                                      (size_t)kObjRing * 4, cudaMemcpyDeviceToHost, s));
+        }
+        return lb_iterate_tail(lb, rho, lambda, iters, prec, objective_h, s);
+    }
     for (int t = 0; t < iters; ++t) {
         // U side: starts the SVID of V (solved by the previous half step, none at t = 0)
         st = lb_half_step(lb, 0, rho, lambda, K, prec, s, ov, t > 0 ? 1 : -1, t > 0);
@@ -673,16 +715,7 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
     // last SVID of V
     NQ_CK(cudaStreamWaitEvent(s, ov->svid_done[0], 0));
     if ((st = lb_svid(lb, 1, K, s))) return st;
-    // objective of the last iteration needs the Gram of the last V
-    st = lb_gram(lb, 1, lambda + rho, prec, s);
-    if (st) return st;
-    if ((st = lb_objective(lb, lambda + rho, (iters - 1) % kObjRing, s))) return st;
-    if (objective_h) {
-        const int done = (iters - 1) / kObjRing * kObjRing;
-        NQ_CK(cudaMemcpyAsync(objective_h + done, lb.p<float>(lb.L.obj),
-                              (size_t)(iters - done) * 4, cudaMemcpyDeviceToHost, s));
-    }
-    return NQ_OK;
+    return lb_iterate_tail(lb, rho, lambda, iters, prec, objective_h, s);
 }
 
 nq_status lb_finish(const Lb &lb, const void *W, int bf16, const float *d_in, const float *d_out,
@@ -823,6 +856,23 @@ nq_status nq_calib_precond(const void *acts, int64_t T_in, int64_t n, const void
         alpha_out[1] = h.alpha[1];
         if (h.err) return static_cast<nq_status>(h.err);
     }
+    return NQ_OK;
+}
+
+nq_status nq_set_tuning(nq_tuning key, int32_t value) {
+    switch (key) {
+        case NQ_TUNE_FACTOR_CTAS:
+            if (value < -1) return NQ_ERR_INVALID_ARG;
+            break;
+        case NQ_TUNE_NEWTON_BN:
+            if (value != 0 && value != 64 && value != 128 && value != 256) return NQ_ERR_INVALID_ARG;
+            break;
+        case NQ_TUNE_SVID_BESIDE:
+            if (value != 0 && value != 1) return NQ_ERR_INVALID_ARG;
+            break;
+        default: return NQ_ERR_INVALID_ARG;
+    }
+    g_tune[key].store(value, std::memory_order_relaxed);
     return NQ_OK;
 }
 

@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(256, 1) chol2_kernel(Chol2Args p) {
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *Gi_hi, __nv_bfloat16 *Gi_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
-                         const int *gate, int gate_skip, cudaStream_t s) {
+                         const int *gate, int gate_skip, bool zero_state, cudaStream_t s) {
     if (rp % TB != 0 || rp < r) return cudaErrorInvalidValue;
     constexpr int smem = (5 * TB * LDS + TB) * sizeof(float);
     // grid of the cooperative launch (one CTA per SM), per device
@@ -670,11 +670,13 @@ cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float 
         grids[dev].store(grid);
     }
     if (max_ctas > 0 && max_ctas < grid) grid = max_ctas < 3 ? 3 : max_ctas;
-    cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
-    if (e != cudaSuccess) return e;
     const int nb = (int)(rp / TB);
-    e = cudaMemsetAsync(flags, 0, (size_t)2 * nb * nb * sizeof(unsigned int), s);
-    if (e != cudaSuccess) return e;
+    if (zero_state) {
+        cudaError_t e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned int), s);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(flags, 0, (size_t)2 * nb * nb * sizeof(unsigned int), s);
+        if (e != cudaSuccess) return e;
+    }
     Chol2Args args{G, r, nb, rp, A, Li, Gi_hi, Gi_lo, ldr, flags, err, bar, gate, gate_skip};
     void *params[] = {&args};
     count_launch();

@@ -524,6 +524,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int STAGE_BYTES = (F3 ? 2 : 1) * (A_TILE_BYTES + B_TILE_BYTES);
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
+    // launched with programmatic stream serialization: everything below may read what the
+    // previous kernel of the stream wrote, so wait for its completion first; then let the
+    // next kernel's launch begin (it waits the same way before touching memory)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // gate: the whole launch is skipped on the gate values in gate_skip
     int gate_v = 0;
     if (p.gate) {
@@ -535,6 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.ns->ticket = 0;
         *reinterpret_cast<volatile int *>(&p.ns->gate) = NS_RUNNING;
     }
+    if (EPI == EPI_GRAM && p.zero)   // counters of a later kernel, zeroed here
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words;
+             i += gridDim.x * blockDim.x)
+            p.zero[i] = 0u;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -808,9 +817,20 @@ static cudaError_t launch_t(const Maps &maps, const EpiParams &p, cudaStream_t s
                                  : num_tiles(p.M, p.N, BN)) *
                           (p.ksplit > 1 ? p.ksplit : 1);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    kern<<<grid, kThreads, smem, s>>>(maps, p);
+    // programmatic dependent launch: the launch overlaps the tail of the previous kernel
+    // of the stream; the kernel waits for that kernel's completion before any memory access
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     count_launch();
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, kern, maps, p);
 }
 
 template <int EPI>

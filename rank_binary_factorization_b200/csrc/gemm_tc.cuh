@@ -110,6 +110,8 @@ struct EpiParams {
     //   written to Rhi/Rlo, or to Fhi/Flo when the gate reads NS_FINAL (then the CTA
     //   finishing the last tile sets NS_DONE).
     NsState *ns;
+    unsigned int *zero;   // EPI_GRAM: zero_words words zeroed before the tiles (counters
+    int zero_words;       // of the factorisation that follows on another stream)
     int ns_step, ns_last, ns_min_final;
     float ns_tau;
     const __nv_bfloat16 *Ph, *Pl;   // X_k (hi, lo), ld ldr

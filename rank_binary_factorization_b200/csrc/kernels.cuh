@@ -49,11 +49,12 @@ cudaError_t transpose_bf16(const __nv_bfloat16 *A, int64_t rows, int64_t cols, i
 // [r][ldr] (LiT_hi, LiT_lo).  A, Li: rp x rp FP32 scratch; flags: 2 (rp/64)^2 counters.
 // max_ctas > 0 limits the cooperative grid (at least 3 CTAs); 0: one CTA per SM.
 // gate: optional device word; the launch does nothing when bit (*gate) of gate_skip is
-// set at its start.
+// set at its start.  zero_state: zero the flags and the grid barrier first (else the
+// caller has zeroed the flags, and the barrier words are as a completed barrier left them).
 cudaError_t chol_inverse(const float *G, int32_t r, int64_t rp, float *A, float *Li,
                          __nv_bfloat16 *LiT_hi, __nv_bfloat16 *LiT_lo, int64_t ldr,
                          unsigned int *flags, int *err, unsigned int *bar, int max_ctas,
-                         const int *gate, int gate_skip, cudaStream_t s);
+                         const int *gate, int gate_skip, bool zero_state, cudaStream_t s);
 
 // ---- SVID -------------------------------------------------------------------------
 // K power steps on |S| (S rows x r, row stride ldf): a = t/||t||, b = A^T t / ||t||.

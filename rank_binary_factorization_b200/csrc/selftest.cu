@@ -85,7 +85,7 @@ extern "C" nq_status nq_selftest(int32_t kind, void *ws, size_t ws_bytes, nq_str
                          reinterpret_cast<__nv_bfloat16 *>(base + L.hi),
                          reinterpret_cast<__nv_bfloat16 *>(base + L.lo), kR,
                          reinterpret_cast<unsigned int *>(base + L.cnt), &sc->err, sc->bar,
-                         0, nullptr, 0, s) != cudaSuccess)
+                         0, nullptr, 0, true, s) != cudaSuccess)
             return NQ_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;

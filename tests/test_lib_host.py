@@ -157,3 +157,25 @@ def test_state_field_offsets_are_inside_the_workspace(m, n, r):
     seen.sort()
     for (s0, e0, n0), (s1, e1, n1) in zip(seen, seen[1:]):
         assert e0 <= s1, (n0, n1)     # fields do not overlap
+
+
+def test_inverse_mode_and_tuning_settings_are_checked():
+    nq = _lib()
+    L = nq.lib
+    INV = 1
+    for mode in (0, 1, 2):
+        assert L.nq_set_inverse_mode(mode) == 0
+    assert L.nq_set_inverse_mode(3) == INV and L.nq_set_inverse_mode(-1) == INV
+    T = nq._lib.TUNING
+    for key, good, bad in (("factor_ctas", (-1, 0, 3, 74, 1000), (-2,)),
+                           ("newton_bn", (0, 64, 128, 256), (32, 96, 512, -1)),
+                           ("svid_beside", (0, 1), (2, -1))):
+        for v in good:
+            assert L.nq_set_tuning(T[key], v) == 0, (key, v)
+        for v in bad:
+            assert L.nq_set_tuning(T[key], v) == INV, (key, v)
+    assert L.nq_set_tuning(3, 0) == INV
+    # back to the defaults
+    assert L.nq_set_inverse_mode(0) == 0
+    for key, v in (("factor_ctas", -1), ("newton_bn", 0), ("svid_beside", 1)):
+        assert L.nq_set_tuning(T[key], v) == 0
