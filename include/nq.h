@@ -166,8 +166,8 @@ size_t nq_lbadmm_workspace_size(int64_t m, int64_t n, int32_t r);
  *   or that reaches no such step, is dropped and the Cholesky path runs instead, decided
  *   on the device (no synchronisation).
  * NQ_INV_AUTO (default): NQ_INV_NEWTON for r >= 256 once the workspace has run 3
- *   iterations since its nq_lbadmm_prepare (the first iterations move G too far),
- *   NQ_INV_CHOLESKY otherwise.
+ *   iterations (4 above r = 1536) since its nq_lbadmm_prepare (the first iterations move
+ *   G too far), NQ_INV_CHOLESKY otherwise.
  * Process-wide; read when a half step is enqueued.  Returns NQ_ERR_INVALID_ARG for an
  * unknown mode.
  */
@@ -183,10 +183,14 @@ nq_status nq_set_inverse_mode(nq_inverse_mode mode);
  *   width on the CTAs it gets, or 64, 128, 256.
  * NQ_TUNE_SVID_BESIDE: 1 (default) the SVID passes of a side run on an auxiliary stream
  *   beside the next half step's GEMMs; 0: right after the side's solve.
+ * NQ_TUNE_NFAST: 1 (default) the RHS GEMM and the solve walk their output tiles column
+ *   tile fastest (the large row operand is read once while its few column tiles run
+ *   together); 0: row tile fastest.
  * Returns NQ_ERR_INVALID_ARG for an unknown key or value.
  */
 typedef enum {
-    NQ_TUNE_FACTOR_CTAS = 0, NQ_TUNE_NEWTON_BN = 1, NQ_TUNE_SVID_BESIDE = 2, NQ_TUNE_COUNT = 3
+    NQ_TUNE_FACTOR_CTAS = 0, NQ_TUNE_NEWTON_BN = 1, NQ_TUNE_SVID_BESIDE = 2, NQ_TUNE_NFAST = 3,
+    NQ_TUNE_COUNT = 4
 } nq_tuning;
 nq_status nq_set_tuning(nq_tuning key, int32_t value);
 

@@ -218,6 +218,7 @@ nq_status side_ctx(SideCtx **out) {
     if (dev < 0) return NQ_ERR_CUDA;
     SideCtx &c = ctx[dev];
     if (!c.side) {
+        // default priority: raising either stream above the caller's was measured slower
         NQ_CK(cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking));
         NQ_CK(cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking));
         for (cudaEvent_t *e : {&c.fork, &c.join, &c.pre_rhs, &c.svid_done[0], &c.svid_done[1]})
@@ -340,13 +341,15 @@ nq_status lb_svid(const Lb &lb, int side, int K, cudaStream_t s) {
 // (written to the side's G^-1); a residual that does not shrink, or no final iterate
 // after kNsMaxSteps, falls back to the Cholesky path, which then runs (gated).
 constexpr int32_t kNsMinRank = 256;  // below this the factorisation is as fast
-constexpr int kNsFirstIter = 3;      // iterations since prepare before the first attempt
+// iterations since prepare before the first attempt (3; 4 above r = 1536, where the
+// Grams of the fourth iteration still move too far)
+inline int ns_first_iter(int32_t r) { return r > 1536 ? 4 : 3; }
 constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E||_2 <= 1e-4)
 
 std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
 
 // Performance settings of nq_set_tuning (none changes a result).
-std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}};
+std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}};
 
 // Iterations run on each workspace since its last prepare (host side; AUTO mode).
 std::mutex g_iter_mu;
@@ -466,7 +469,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     const int mode = g_inverse_mode.load(std::memory_order_relaxed);
     const bool newton = mode == NQ_INV_NEWTON ||
                         (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
-                         iters_since_prepare(lb.ws) >= kNsFirstIter);
+                         iters_since_prepare(lb.ws) >= ns_first_iter(L.r));
     NsState *ns = lb.p<NsState>(L.ns);
     nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton, true);
     if (st) return st;
@@ -567,6 +570,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ep.Rlo = lb.p<__nv_bfloat16>(L.rlo);
         ep.ldr = L.ldr;
         ep.max_ctas = cc > 0 ? sms - cc : 0;
+        ep.nfast = g_tune[NQ_TUNE_NFAST].load(std::memory_order_relaxed);
         ProfScope ps(NQ_K_RHS, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RHS, BN, s));
     }
@@ -604,6 +608,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ep.ldxt = L.ld_rows(side);
         ep.objective = side == 1;
         ep.part = lb.p<double>(L.part);
+        ep.nfast = g_tune[NQ_TUNE_NFAST].load(std::memory_order_relaxed);
         ProfScope ps(NQ_K_SOLVE, s);
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BN, s));
     }
@@ -868,6 +873,7 @@ nq_status nq_set_tuning(nq_tuning key, int32_t value) {
             if (value != 0 && value != 64 && value != 128 && value != 256) return NQ_ERR_INVALID_ARG;
             break;
         case NQ_TUNE_SVID_BESIDE:
+        case NQ_TUNE_NFAST:
             if (value != 0 && value != 1) return NQ_ERR_INVALID_ARG;
             break;
         default: return NQ_ERR_INVALID_ARG;

@@ -493,8 +493,11 @@ __device__ __forceinline__ void ns_tile_done(const EpiParams &p, int tile, int n
     }
 }
 
-// Output tile -> (m0, n0).  Plain: m fastest.  Symmetric (BN == BM): the lower-triangular
-// tiles (tm >= tn) row by row, so tiles come in order of decreasing K range under tri_k.
+// Output tile -> (m0, n0).  Plain: m fastest (consecutive CTAs share the B tile), or n
+// fastest with nfast (they share the A tile: A is the large operand, read from HBM once
+// while its row block's few column tiles run at the same time).  Symmetric (BN == BM):
+// the lower-triangular tiles (tm >= tn) row by row, so tiles come in order of decreasing
+// K range under tri_k.
 template <int BN>
 __device__ __forceinline__ void tile_origin(const EpiParams &p, int tile, int num_m, int &m0,
                                             int &n0) {
@@ -504,6 +507,10 @@ __device__ __forceinline__ void tile_origin(const EpiParams &p, int tile, int nu
         while (a * (a + 1) / 2 > tile) --a;
         m0 = a * BM;
         n0 = (tile - a * (a + 1) / 2) * BN;
+    } else if (p.nfast) {
+        const int num_n = (p.N + BN - 1) / BN;
+        m0 = (tile / num_n) * BM;
+        n0 = (tile % num_n) * BN;
     } else {
         m0 = (tile % num_m) * BM;
         n0 = (tile / num_m) * BN;

@@ -45,6 +45,7 @@ struct EpiParams {
     int tri_k;          // operands zero for k < row index: start each tile's K at max(m0, n0)
     int sym;            // symmetric result (EPI_SPLIT / EPI_GRAM, BN == BM, M == N): lower-
                         // triangular tiles only, each off-diagonal tile also written mirrored
+    int nfast;          // tiles in n-fastest order (see tile_origin)
     int max_ctas;       // 0: one CTA per SM; else at most this many CTAs (SMs left free for
                         // kernels running beside this one on another stream)
     int ksplit;         // EPI_GRAM only: > 1 splits the K range into ksplit parts; unit u
