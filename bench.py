@@ -167,13 +167,16 @@ def kernel_units(cls, m, n, r, K, T, ns_steps=4):
     return None
 
 
-# DRAM bytes (read + write) per launch scope from an ncu capture of the current kernels
-# (calibration: `ncu --set full` of `bench.py --workload profile`, 65536 x 4096 BF16
-# streams; one read of the stream, so it scales with T x C).  Classes whose kernels
-# changed since their last capture report null.
+# DRAM bytes (read + write) per launch scope from ncu captures of the current kernels on
+# the profiling case (`bench.py --workload profile --iters 6`, the same 11008 x 4096 layer
+# at r = 1000 with 65536-token streams).  Calibration: one read of the stream, so it scales
+# with T x C.  The Newton-Schulz update: the sum over its GEMMs of one half step at
+# r = 1000, for that rank only.  Classes without a capture of their current kernels: null.
 def ncu_traffic(cls, m, n, r, T):
     if cls == "calib":
-        return 540.4e6 * (T * (m + n) / 2) / (65536 * 4096)
+        return 1.446e9 * (T * (m + n) / 2) / (65536 * 11008)
+    if cls == "newton" and r == 1000:
+        return 55.0e6
     return None
 
 

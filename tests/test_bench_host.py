@@ -46,13 +46,18 @@ def test_roofline_entry_fractions():
     c = bench.roofline_entry("calib", 2, 0.5, m, n, r, K, T, peaks)
     assert c["unit"] == "GB/s" and c["achieved"] == pytest.approx(T * 2 * n / 2.5e-4 / 1e9,
                                                                    rel=1e-3)
-    assert c["traffic"] == pytest.approx(540.4e6 * T * n / (65536 * 4096))
+    # the capture: 1.446 GB for one 65536 x 11008 BF16 stream (1.002 x its T x C x 2 bytes)
+    assert c["traffic"] == pytest.approx(1.446e9 * T * n / (65536 * 11008))
+    assert c["traffic"] == pytest.approx(T * n * 2, rel=0.01)
     assert bench.roofline_entry("rhs", 0, 1.0, m, n, r, K, T, peaks) is None
 
 
 def test_traffic_only_for_captured_kernels():
-    # only the calibration kernel's capture is current; it scales with the stream size
+    # the calibration capture scales with the stream size; the inverse update's holds for
+    # the rank it was taken at only
     assert bench.ncu_traffic("calib", 4096, 4096, 2032, 262144) > 0
+    assert bench.ncu_traffic("newton", 11008, 4096, 1000, 262144) == 55.0e6
+    assert bench.ncu_traffic("newton", 4096, 4096, 2032, 262144) is None
     assert bench.ncu_traffic("chol", 4096, 4096, 2032, 262144) is None
     assert bench.ncu_traffic("svid", 4096, 4096, 2032, 262144) is None
 
