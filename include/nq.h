@@ -186,11 +186,14 @@ nq_status nq_set_inverse_mode(nq_inverse_mode mode);
  * NQ_TUNE_NFAST: 1 (default) the RHS GEMM and the solve walk their output tiles column
  *   tile fastest (the large row operand is read once while its few column tiles run
  *   together); 0: row tile fastest.
+ * NQ_TUNE_RHS_BN, NQ_TUNE_SOLVE_BN: tile width of the RHS GEMM / of the solve: 0 (default:
+ *   RHS 256 for r > 128, solve 128 for 128 < r <= 1024 and 256 above; narrower for small
+ *   r), or 128, 256.
  * Returns NQ_ERR_INVALID_ARG for an unknown key or value.
  */
 typedef enum {
     NQ_TUNE_FACTOR_CTAS = 0, NQ_TUNE_NEWTON_BN = 1, NQ_TUNE_SVID_BESIDE = 2, NQ_TUNE_NFAST = 3,
-    NQ_TUNE_COUNT = 4
+    NQ_TUNE_RHS_BN = 4, NQ_TUNE_SOLVE_BN = 5, NQ_TUNE_COUNT = 6
 } nq_tuning;
 nq_status nq_set_tuning(nq_tuning key, int32_t value);
 

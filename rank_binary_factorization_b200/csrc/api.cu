@@ -209,7 +209,8 @@ nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s
 // the next half step's RHS GEMM and solve (see lb_iterate), with its events.
 struct SideCtx {
     cudaStream_t side = nullptr, aux = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr, pre_rhs = nullptr, svid_done[2] = {nullptr, nullptr};
+    cudaEvent_t fork = nullptr, join = nullptr, pre_rhs = nullptr, obj_done = nullptr,
+                svid_done[2] = {nullptr, nullptr};
 };
 
 nq_status side_ctx(SideCtx **out) {
@@ -221,7 +222,8 @@ nq_status side_ctx(SideCtx **out) {
         // default priority: raising either stream above the caller's was measured slower
         NQ_CK(cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking));
         NQ_CK(cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking));
-        for (cudaEvent_t *e : {&c.fork, &c.join, &c.pre_rhs, &c.svid_done[0], &c.svid_done[1]})
+        for (cudaEvent_t *e :
+             {&c.fork, &c.join, &c.pre_rhs, &c.obj_done, &c.svid_done[0], &c.svid_done[1]})
             NQ_CK(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     }
     *out = &c;
@@ -349,7 +351,19 @@ constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E|
 std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
 
 // Performance settings of nq_set_tuning (none changes a result).
-std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}};
+std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}, {0}, {0}};
+
+// Tile widths of the RHS GEMM and of the solve (the objective's partials follow the solve's).
+int rhs_bn(int32_t r) {
+    const int v = g_tune[NQ_TUNE_RHS_BN].load(std::memory_order_relaxed);
+    return v ? v : pick_bn(r);
+}
+int solve_bn(int32_t r) {
+    // 128-wide tiles up to r = 1024 (twice the tiles, so the heavy epilogue of one tile
+    // overlaps the next tile's MMAs on more CTAs; measured 1 % faster at r = 1000)
+    const int v = g_tune[NQ_TUNE_SOLVE_BN].load(std::memory_order_relaxed);
+    return v ? v : (r > 128 && r <= 1024 ? 128 : pick_bn(r));
+}
 
 // Iterations run on each workspace since its last prepare (host side; AUTO mode).
 std::mutex g_iter_mu;
@@ -459,13 +473,17 @@ nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
 // G^-1 is formed, beside its RHS GEMM and solve; ``wait_own`` makes the RHS GEMM wait for
 // the SVID of ``side`` started by the previous half step (the RHS and the solve read the
 // dual state a, b it writes).
+nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s);
+
 nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, int prec,
                        cudaStream_t s, SideCtx *ov = nullptr, int pending = -1,
-                       bool wait_own = false) {
+                       bool wait_own = false, int obj_slot = -1, bool wait_obj = false) {
     const LbLayout &L = lb.L;
+    // the Gram below overwrites the Gram of U that the previous objective reads
+    if (ov && wait_obj) NQ_CK(cudaStreamWaitEvent(s, ov->obj_done, 0));
     const int other = 1 - side;
     const int64_t rows = L.rows(side), Kd = L.rows(other);
-    const int BN = pick_bn(L.r);
+    const int BN = rhs_bn(L.r), BNs = solve_bn(L.r);
     const int mode = g_inverse_mode.load(std::memory_order_relaxed);
     const bool newton = mode == NQ_INV_NEWTON ||
                         (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
@@ -533,6 +551,10 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     if (ov && pending >= 0) {   // the previous half step's SVID, beside this RHS and solve
         NQ_CK(cudaEventRecord(ov->pre_rhs, s));
         NQ_CK(cudaStreamWaitEvent(ov->aux, ov->pre_rhs, 0));
+        if (obj_slot >= 0) {    // the previous iteration's objective: both Grams are formed
+            if ((st = lb_objective(lb, lambda + rho, obj_slot, ov->aux))) return st;
+            NQ_CK(cudaEventRecord(ov->obj_done, ov->aux));
+        }
         if ((st = lb_svid(lb, pending, K, ov->aux))) return st;
         NQ_CK(cudaEventRecord(ov->svid_done[pending], ov->aux));
     }
@@ -583,8 +605,8 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         const void *gh = lb.p<void>(L.gih[side]), *gl = lb.p<void>(L.gil[side]);
         if (!tc::make_map_bf16(&maps.a[0], rh, rows, L.r, L.ldr, tc::BM) ||
             !tc::make_map_bf16(&maps.a[1], rl, rows, L.r, L.ldr, tc::BM) ||
-            !tc::make_map_bf16(&maps.b[0], gh, L.r, L.r, L.ldr, BN) ||
-            !tc::make_map_bf16(&maps.b[1], gl, L.r, L.r, L.ldr, BN))
+            !tc::make_map_bf16(&maps.b[0], gh, L.r, L.r, L.ldr, BNs) ||
+            !tc::make_map_bf16(&maps.b[1], gl, L.r, L.r, L.ldr, BNs))
             return NQ_ERR_CUDA;
         tc::EpiParams ep;
         memset(&ep, 0, sizeof(ep));
@@ -610,7 +632,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         ep.part = lb.p<double>(L.part);
         ep.nfast = g_tune[NQ_TUNE_NFAST].load(std::memory_order_relaxed);
         ProfScope ps(NQ_K_SOLVE, s);
-        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BN, s));
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_SOLVE, BNs, s));
     }
     if (ov) return NQ_OK;
     return lb_svid(lb, side, K, s);
@@ -618,7 +640,7 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
 
 nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s) {
     const LbLayout &L = lb.L;
-    const int npx = (int)tc::num_tiles((int)L.n, L.r, pick_bn(L.r));
+    const int npx = (int)tc::num_tiles((int)L.n, L.r, solve_bn(L.r));
     ProfScope ps(NQ_K_OBJ, s);
     NQ_CK(objective(lb.p<float>(L.g[0]), lb.p<float>(L.g[1]), L.r, c, lb.p<double>(L.part), npx,
                     lb.p<double>(L.partg), lb.sc, lb.p<float>(L.obj) + slot, s));
@@ -682,7 +704,9 @@ nq_status lb_iterate_tail(const Lb &lb, float rho, float lambda, int iters, int 
 
 // The iterations.  The SVID of the side just solved is needed only by that side's next
 // RHS GEMM, one half step later, so it runs on the auxiliary stream beside the next half
-// step's RHS GEMM and solve; the last one runs on ``s`` before returning.
+// step's RHS GEMM and solve; the last one runs on ``s`` before returning.  The objective of
+// iteration t - 1 needs both Grams, the second formed at the start of iteration t: it runs
+// on the auxiliary stream too, before the next Gram of U overwrites the first.
 nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, int prec,
                      float *objective_h, cudaStream_t s) {
     SideCtx *ov = nullptr;
@@ -702,12 +726,15 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
         return lb_iterate_tail(lb, rho, lambda, iters, prec, objective_h, s);
     }
     for (int t = 0; t < iters; ++t) {
-        // U side: starts the SVID of V (solved by the previous half step, none at t = 0)
-        st = lb_half_step(lb, 0, rho, lambda, K, prec, s, ov, t > 0 ? 1 : -1, t > 0);
+        // U side: starts the objective of the previous iteration and the SVID of V (solved
+        // by the previous half step; none at t = 0) on the auxiliary stream
+        st = lb_half_step(lb, 0, rho, lambda, K, prec, s, ov, t > 0 ? 1 : -1, t > 0,
+                          t > 0 ? (t - 1) % kObjRing : -1);
         if (st) return st;
-        if (t > 0 && (st = lb_objective(lb, lambda + rho, (t - 1) % kObjRing, s))) return st;
-        // V side: starts the SVID of U, waits for its own from the previous iteration
-        if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s, ov, 0, t > 0))) return st;
+        // V side: starts the SVID of U, waits for its own from the previous iteration; its
+        // Gram waits for that objective
+        if ((st = lb_half_step(lb, 1, rho, lambda, K, prec, s, ov, 0, t > 0, -1, t > 0)))
+            return st;
         add_iters(lb.ws, 1);
         if (objective_h && t > 0 && (t % kObjRing) == 0) {
             // the ring holds the objectives of iterations t - kObjRing .. t - 1; the copy is
@@ -871,6 +898,10 @@ nq_status nq_set_tuning(nq_tuning key, int32_t value) {
             break;
         case NQ_TUNE_NEWTON_BN:
             if (value != 0 && value != 64 && value != 128 && value != 256) return NQ_ERR_INVALID_ARG;
+            break;
+        case NQ_TUNE_RHS_BN:
+        case NQ_TUNE_SOLVE_BN:
+            if (value != 0 && value != 128 && value != 256) return NQ_ERR_INVALID_ARG;
             break;
         case NQ_TUNE_SVID_BESIDE:
         case NQ_TUNE_NFAST:
