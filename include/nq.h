@@ -189,11 +189,16 @@ nq_status nq_set_inverse_mode(nq_inverse_mode mode);
  * NQ_TUNE_RHS_BN, NQ_TUNE_SOLVE_BN: tile width of the RHS GEMM / of the solve: 0 (default:
  *   RHS 256 for r > 128, solve 128 for 128 < r <= 1024 and 256 above; narrower for small
  *   r), or 128, 256.
+ * NQ_TUNE_NEWTON_FUSED: 0 (default) two launches per step of the Newton-Schulz update;
+ *   1: all its steps in one cooperative launch on 128 x 128 tiles (grid-wide barriers
+ *   between its GEMMs; the update itself is shorter, but its CTAs stay resident through
+ *   the barriers and the GEMMs and SVID passes beside it slow down by as much at r = 1000,
+ *   more at other ranks).  NQ_TUNE_NEWTON_BN applies to the two-launch form only.
  * Returns NQ_ERR_INVALID_ARG for an unknown key or value.
  */
 typedef enum {
     NQ_TUNE_FACTOR_CTAS = 0, NQ_TUNE_NEWTON_BN = 1, NQ_TUNE_SVID_BESIDE = 2, NQ_TUNE_NFAST = 3,
-    NQ_TUNE_RHS_BN = 4, NQ_TUNE_SOLVE_BN = 5, NQ_TUNE_COUNT = 6
+    NQ_TUNE_RHS_BN = 4, NQ_TUNE_SOLVE_BN = 5, NQ_TUNE_NEWTON_FUSED = 6, NQ_TUNE_COUNT = 7
 } nq_tuning;
 nq_status nq_set_tuning(nq_tuning key, int32_t value);
 

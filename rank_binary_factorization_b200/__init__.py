@@ -181,7 +181,7 @@ def nq_set_inverse_mode(mode):
 
 def nq_set_tuning(key, value):
     """Scheduling setting ("factor_ctas", "newton_bn", "svid_beside", "nfast", "rhs_bn",
-    "solve_bn"; see nq_tuning)."""
+    "solve_bn", "newton_fused"; see nq_tuning)."""
     check("nq_set_tuning", lib.nq_set_tuning(_lib.TUNING[key], int(value)))
 
 

@@ -28,7 +28,8 @@ NQ_PREC_BF16, NQ_PREC_FP32 = 0, 1
 FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9, WHAT_LO=10,
               INV_STATS=11, GINV_U=12, GINV_U_LO=13, GINV_V=14, GINV_V_LO=15)
 NQ_INV_AUTO, NQ_INV_CHOLESKY, NQ_INV_NEWTON = 0, 1, 2
-TUNING = dict(factor_ctas=0, newton_bn=1, svid_beside=2, nfast=3, rhs_bn=4, solve_bn=5)
+TUNING = dict(factor_ctas=0, newton_bn=1, svid_beside=2, nfast=3, rhs_bn=4, solve_bn=5,
+              newton_fused=6)
 
 # name -> (restype, argtypes); the list is the full set of exported entry points
 SIGNATURES = {

@@ -351,7 +351,7 @@ constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E|
 std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
 
 // Performance settings of nq_set_tuning (none changes a result).
-std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}, {0}, {0}};
+std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}, {0}, {0}, {0}};
 
 // Tile widths of the RHS GEMM and of the solve (the objective's partials follow the solve's).
 int rhs_bn(int32_t r) {
@@ -396,7 +396,45 @@ int pick_bn_square(int32_t r, int ctas) {
     return best;
 }
 
+// All steps in one cooperative launch (see tc::newton_kernel).
+nq_status lb_newton_fused(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    const int r = L.r;
+    tc::NsMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    tc::NsArgs a;
+    memset(&a, 0, sizeof(a));
+    const size_t xh[3] = {L.gih[side], L.nqh[0], L.nqh[1]};
+    const size_t xl[3] = {L.gil[side], L.nql[0], L.nql[1]};
+    for (int i = 0; i < 3; ++i) {
+        a.xh[i] = lb.p<__nv_bfloat16>(xh[i]);
+        a.xl[i] = lb.p<__nv_bfloat16>(xl[i]);
+        if (!tc::make_map_bf16(&maps.xh[i], a.xh[i], r, r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.xl[i], a.xl[i], r, r, L.ldr, tc::BM))
+            return NQ_ERR_CUDA;
+    }
+    a.eh = lb.p<__nv_bfloat16>(L.nth);
+    a.el = lb.p<__nv_bfloat16>(L.ntl);
+    if (!tc::make_map_bf16(&maps.gh, lb.p<void>(L.gsh), r, r, L.ldr, tc::BM) ||
+        !tc::make_map_bf16(&maps.gl, lb.p<void>(L.gsl), r, r, L.ldr, tc::BM) ||
+        !tc::make_map_bf16(&maps.eh, a.eh, r, r, L.ldr, tc::BM))
+        return NQ_ERR_CUDA;
+    a.r = r;
+    a.ldr = L.ldr;
+    a.nsteps = kNsMaxSteps;
+    a.bf16_steps = kNsBf16Steps;
+    a.tau = kNsTau;
+    a.err = &lb.sc->err;
+    a.ns = lb.p<NsState>(L.ns);
+    a.part = lb.p<double>(L.nspart);
+    ProfScope ps(NQ_K_NEWTON, s);
+    NQ_CK(tc::launch_newton(maps, a, max_ctas, s));
+    return NQ_OK;
+}
+
 nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
+    if (g_tune[NQ_TUNE_NEWTON_FUSED].load(std::memory_order_relaxed))
+        return lb_newton_fused(lb, side, max_ctas, s);
     const LbLayout &L = lb.L;
     NsState *ns = lb.p<NsState>(L.ns);
     const int r = L.r;
@@ -905,6 +943,7 @@ nq_status nq_set_tuning(nq_tuning key, int32_t value) {
             break;
         case NQ_TUNE_SVID_BESIDE:
         case NQ_TUNE_NFAST:
+        case NQ_TUNE_NEWTON_FUSED:
             if (value != 0 && value != 1) return NQ_ERR_INVALID_ARG;
             break;
         default: return NQ_ERR_INVALID_ARG;

@@ -545,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool fin = (EPI == EPI_NS2) && gate_v == NS_FINAL;
     if (EPI == EPI_GRAM && p.ns && blockIdx.x == 0 && threadIdx.x == 0) {
         p.ns->ticket = 0;
+        p.ns->grid_count = 0;
         *reinterpret_cast<volatile int *>(&p.ns->gate) = NS_RUNNING;
     }
     if (EPI == EPI_GRAM && p.zero)   // counters of a later kernel, zeroed here
@@ -779,6 +780,305 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------
+// Newton-Schulz update of G^-1 in one cooperative launch.  Phases 2k and 2k+1 are the two
+// GEMMs of step k (E_k = I - X_k G; X_{k+1} = X_k + E_k X_k) on 128 x 128 tiles; between
+// phases every CTA's epilogue stores are made visible (proxy fence, release) and the next
+// phase's loads wait on a grid-wide arrival count (bounded).  The gate decides at each
+// phase start, read once per CTA after the barrier: an E phase runs while the gate is
+// RUNNING; an X phase runs while RUNNING, and writes the final iterate to X buffer 0 when
+// it is FINAL.  The operand pipeline, the TMEM stages and their barriers carry across
+// phases; each stage holds four tiles (split phases use all four, BF16 phases two).
+// ---------------------------------------------------------------------------------
+constexpr int kNsBN = 128;
+constexpr int kNsStages = 3;
+
+__device__ __forceinline__ void ns_decide(const NsArgs &a, int k, int lane, int num_tiles) {
+    // called by the warp that finished the last E tile of phase 2k
+    NsState *ns = a.ns;
+    double t = 0.0;
+    for (int i = lane; i < num_tiles; i += 32) t += __ldcg(a.part + i);
+    t = warp_sum(t);
+    if (lane == 0) {
+        const double ef = t >= 0.0 ? sqrt(t) : -1.0;
+        ns->ef[k] = ef;
+        const double prev = k > 0 ? ns->ef[k - 1] : 0.0;
+        int g = NS_RUNNING;
+        if (!(ef >= 0.0 && ef < 1e30))
+            g = NS_FAIL;
+        else if (k >= a.bf16_steps && ef <= (double)a.tau)
+            g = NS_FINAL;
+        else if (k >= a.nsteps - 1 || (k > a.bf16_steps && ef > 0.9 * prev) ||
+                 (k > 0 && k < a.bf16_steps && ef > 1.5 * prev))
+            g = NS_FAIL;
+        if (g == NS_FAIL) ns->fallbacks += 1;
+        if (g == NS_FINAL) ns->steps = k + 1;
+        ns->ticket = 0;
+        __threadfence();
+        *reinterpret_cast<volatile int *>(&ns->gate) = g;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    newton_kernel(const __grid_constant__ NsMaps maps, const NsArgs a) {
+    constexpr int BN = kNsBN, STAGES = kNsStages;
+    constexpr int B_TILE_BYTES = BN * BK * 2;
+    constexpr int STAGE_BYTES = 2 * (A_TILE_BYTES + B_TILE_BYTES);
+    constexpr uint32_t TMEM_COLS = 2 * BN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *empty_bar = full_bar + STAGES;
+    uint64_t *tfull = empty_bar + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    __shared__ double red[2][kEpiWarps];
+    __shared__ int s_gate;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (int)ceil_div(a.r, BM);
+    const int num_tiles = num_m * (int)ceil_div(a.r, BN);
+    const int kbs = (int)ceil_div(a.r, BK);
+    const unsigned G = gridDim.x;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&tfull[s], 1);
+            mbar_init(&tempty[s], kEpiWarps);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    uint32_t it = 0;       // operand stages issued (producer) / consumed (MMA)
+    int lt = 0;            // tiles through the accumulator stages (MMA and epilogue)
+    bool ok = true;        // this thread's waits all completed
+    const int nphases = 2 * a.nsteps;
+    for (int ph = 0; ph < nphases; ++ph) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            // (after a wait ran out anywhere, later barriers are not waited for)
+            if (ph > 0 && *reinterpret_cast<volatile int *>(a.err) != NQ_ERR_TIMEOUT &&
+                !wait_geq(&a.ns->grid_count, (unsigned)ph * G, kGridSpinLimit))
+                raise_error(a.err, NQ_ERR_TIMEOUT);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            int g = *reinterpret_cast<volatile int *>(&a.ns->gate);
+            if (blockIdx.x == 0 && (ph & 1) == 0 && g == NS_FINAL) {
+                // the previous step's X phase wrote the final iterate: close the update
+                a.ns->accepted += 1;
+                *reinterpret_cast<volatile int *>(&a.ns->gate) = NS_DONE;
+            }
+            s_gate = g;
+        }
+        __syncthreads();
+        const int k = ph >> 1;
+        const bool eph = (ph & 1) == 0;   // E phase (else X phase)
+        const int g = s_gate;
+        const bool run = eph ? g == NS_RUNNING : (g == NS_RUNNING || g == NS_FINAL);
+        const bool fin = !eph && g == NS_FINAL;
+        const bool split = eph && k >= a.bf16_steps;
+        const int xi = k == 0 ? 0 : 1 + (k & 1);         // X_k
+        const int di = 1 + ((k + 1) & 1);                  // X_{k+1} when not final
+        // producer and MMA issuer stop after a wait that ran out; the epilogue warps walk
+        // every tile of a phase that runs (they meet at named barriers per tile)
+        if (run) {
+            if (warp == 0) {
+                if (lane == 0 && ok) {
+                    const CUtensorMap *ma = eph ? &maps.xh[xi] : &maps.eh;
+                    const CUtensorMap *mal = &maps.xl[xi];
+                    const CUtensorMap *mb = eph ? &maps.gh : &maps.xh[xi];
+                    const CUtensorMap *mbl = &maps.gl;
+                    const uint32_t bytes = split ? STAGE_BYTES : A_TILE_BYTES + B_TILE_BYTES;
+                    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += G) {
+                        const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+                        for (int kb = 0; kb < kbs; ++kb) {
+                            const int s = it % STAGES;
+                            if (it >= STAGES &&
+                                !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, a.err)) {
+                                ok = false;
+                                break;
+                            }
+                            uint8_t *a_dst = smem + s * STAGE_BYTES;
+                            uint8_t *b_dst = a_dst + 2 * A_TILE_BYTES;
+                            mbar_expect_tx(&full_bar[s], bytes);
+                            tma_load_2d(a_dst, ma, kb * BK, m0, &full_bar[s]);
+                            tma_load_2d(b_dst, mb, kb * BK, n0, &full_bar[s]);
+                            if (split) {
+                                tma_load_2d(a_dst + A_TILE_BYTES, mal, kb * BK, m0, &full_bar[s]);
+                                tma_load_2d(b_dst + B_TILE_BYTES, mbl, kb * BK, n0, &full_bar[s]);
+                            }
+                            ++it;
+                        }
+                    }
+                }
+            } else if (warp == 1) {
+                if (lane == 0 && ok) {
+                    constexpr uint32_t idesc = instr_desc_bf16(BM, BN);
+                    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += G, ++lt) {
+                        const int as = lt & 1;
+                        if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, a.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem + (uint32_t)(as * BN);
+                        for (int kb = 0; kb < kbs; ++kb) {
+                            const int s = it % STAGES;
+                            if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, a.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint8_t *src = smem + s * STAGE_BYTES;
+                            const uint64_t ah = smem_desc_sw128(src);
+                            const uint64_t bh = smem_desc_sw128(src + 2 * A_TILE_BYTES);
+#pragma unroll
+                            for (int q = 0; q < BK / 16; ++q)
+                                mma_bf16(d, ah + 2 * q, bh + 2 * q, idesc, (kb == 0 && q == 0) ? 0u : 1u);
+                            if (split) {
+                                const uint64_t al = smem_desc_sw128(src + A_TILE_BYTES);
+                                const uint64_t bl = smem_desc_sw128(src + 2 * A_TILE_BYTES + B_TILE_BYTES);
+#pragma unroll
+                                for (int q = 0; q < BK / 16; ++q) mma_bf16(d, al + 2 * q, bh + 2 * q, idesc, 1u);
+#pragma unroll
+                                for (int q = 0; q < BK / 16; ++q) mma_bf16(d, ah + 2 * q, bl + 2 * q, idesc, 1u);
+                            }
+                            mma_commit(&empty_bar[s]);
+                            ++it;
+                        }
+                        if (ok) mma_commit(&tfull[as]);
+                    }
+                }
+            } else {
+                const int qw = warp & 3;
+                __nv_bfloat16 *dh = fin ? a.xh[0] : a.xh[di];
+                __nv_bfloat16 *dl = fin ? a.xl[0] : a.xl[di];
+                const __nv_bfloat16 *ph_ = a.xh[xi], *pl_ = a.xl[xi];
+                for (int tile = blockIdx.x; tile < num_tiles; tile += G, ++lt) {
+                    const int as = lt & 1;
+                    const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+                    const int row = m0 + 32 * qw + lane;
+                    float acc_sum = 0.f;
+                    if (ok) {
+                        int w = 0;
+                        if (lane == 0) w = mbar_wait(&tfull[as], (lt >> 1) & 1, a.err) ? 1 : 0;
+                        w = __shfl_sync(0xffffffffu, w, 0);
+                        ok = w != 0;
+                    }
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t tbase = tmem + (uint32_t)(as * BN) + ((uint32_t)(32 * qw) << 16);
+#pragma unroll 1
+                        for (int c = 0; c < BN; c += 16) {
+                            float v[16];
+                            tmem_ld16(tbase + c, v);
+                            const int col0 = n0 + c;
+                            if (row < a.r && col0 < a.r) {
+                                const bool full = col0 + 16 <= a.r;
+                                const int64_t so = (int64_t)row * a.ldr + col0;
+                                float o[16];
+                                if (eph) {
+#pragma unroll
+                                    for (int j = 0; j < 16; ++j) {
+                                        o[j] = (row == col0 + j ? 1.f : 0.f) - v[j];
+                                        if (full || col0 + j < a.r) acc_sum += o[j] * o[j];
+                                    }
+                                    split_store(a.eh + so, a.el + so, full, a.r - col0, o);
+                                } else {
+                                    float xh[16], xl[16];
+                                    if (full) {
+                                        ld16_bf16(xh, ph_ + so);
+                                        ld16_bf16(xl, pl_ + so);
+                                    } else {
+#pragma unroll
+                                        for (int j = 0; j < 16; ++j) {
+                                            const bool in = col0 + j < a.r;
+                                            xh[j] = in ? __bfloat162float(ph_[so + j]) : 0.f;
+                                            xl[j] = in ? __bfloat162float(pl_[so + j]) : 0.f;
+                                        }
+                                    }
+#pragma unroll
+                                    for (int j = 0; j < 16; ++j) o[j] = (xh[j] + xl[j]) + v[j];
+                                    split_store(dh + so, dl + so, full, a.r - col0, o);
+                                }
+                            }
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[as]);
+                    }
+                    if (eph) {
+                        // the tile's sum of E^2; the warp finishing the last tile decides
+                        const double wsum = warp_sum((double)acc_sum);
+                        if (lane == 0) red[as][warp - 2] = ok ? wsum : __longlong_as_double(-1ll);
+                        epilogue_bar();
+                        if (warp == 2) {
+                            unsigned last = 0;
+                            if (lane == 0) {
+                                double t = 0.0;
+                                for (int e = 0; e < kEpiWarps; ++e) t += red[as][e];
+                                a.part[tile] = t;
+                                __threadfence();
+                                last = atomicAdd(&a.ns->ticket, 1u) == (unsigned)(num_tiles - 1) ? 1u : 0u;
+                            }
+                            last = __shfl_sync(0xffffffffu, last, 0);
+                            if (last) {
+                                __threadfence();
+                                ns_decide(a, k, lane, num_tiles);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        // arrival: this CTA's outputs of the phase are written (every phase, run or not)
+        if (warp >= 2) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            epilogue_bar();
+            if (warp == 2 && lane == 0) {
+                __threadfence();
+                atomicAdd(&a.ns->grid_count, 1u);
+            }
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        // an update accepted in the last step: close it once every CTA has arrived
+        if (*reinterpret_cast<volatile int *>(a.err) != NQ_ERR_TIMEOUT &&
+            !wait_geq(&a.ns->grid_count, (unsigned)nphases * G, kGridSpinLimit))
+            raise_error(a.err, NQ_ERR_TIMEOUT);
+        if (*reinterpret_cast<volatile int *>(&a.ns->gate) == NS_FINAL) {
+            a.ns->accepted += 1;
+            *reinterpret_cast<volatile int *>(&a.ns->gate) = NS_DONE;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -876,6 +1176,31 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_NS2: return launch_bn<EPI_NS2>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_newton(const NsMaps &maps, const NsArgs &a, int max_ctas, cudaStream_t s) {
+    constexpr int smem = kNsStages * 2 * (A_TILE_BYTES + kNsBN * BK * 2) + 1024 + 256;
+    static_assert(smem <= 227 * 1024, "shared memory of the update's stage ring");
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = ensure_smem_limit((const void *)newton_kernel, smem, configured);
+    if (e != cudaSuccess) return e;
+    int sms = device_sm_count();
+    if (max_ctas > 0 && max_ctas < sms) sms = max_ctas;
+    const int64_t tiles = ceil_div(a.r, BM) * ceil_div(a.r, kNsBN);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    // cooperative: the phases wait on one another across CTAs (one CTA per SM fits)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, newton_kernel, maps, a);
 }
 
 }  // namespace tc

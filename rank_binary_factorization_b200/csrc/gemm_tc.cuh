@@ -127,6 +127,27 @@ bool make_map_bf16(CUtensorMap *map, const void *base, int64_t rows, int64_t col
 // Host: launch one GEMM.  BN in {64, 128, 256}.
 cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, cudaStream_t s);
 
+// Newton-Schulz update of G^-1 (all steps) in one cooperative launch on 128 x 128 tiles.
+// X buffers (hi + lo BF16, r x r, ld ldr): 0 holds X_0 on entry and receives the accepted
+// iterate; 1 and 2 hold the iterates between steps.  E: the residual I - X_k G.
+struct NsMaps {
+    CUtensorMap xh[3], xl[3];   // box 64 x 128
+    CUtensorMap gh, gl;         // the Gram, split (box 64 x 128)
+    CUtensorMap eh;             // E hi (box 64 x 128)
+};
+struct NsArgs {
+    int r;
+    int64_t ldr;
+    int nsteps, bf16_steps;     // steps enqueued; the first bf16_steps residuals in BF16
+    float tau;                  // ||E_k||_F that makes X_{k+1} final
+    int *err;
+    NsState *ns;                // gate, ticket and grid_count reset by the Gram
+    double *part;               // per-tile partials of ||E_k||_F^2
+    __nv_bfloat16 *xh[3], *xl[3];
+    __nv_bfloat16 *eh, *el;
+};
+cudaError_t launch_newton(const NsMaps &maps, const NsArgs &a, int max_ctas, cudaStream_t s);
+
 // Host: number of output tiles of a launch (size of the per-tile partial array).
 inline int64_t num_tiles(int M, int N, int BN) { return ceil_div(M, BM) * ceil_div(N, BN); }
 

@@ -49,6 +49,8 @@ struct NsState {
     double ef[kNsMaxSteps + 2];    // ||I - X_k G||_F of the last attempt, step by step
     int gate;                      // NsGate of the running half step
     unsigned int ticket;           // finished tiles of the running launch
+    unsigned int grid_count;       // phases x CTAs arrived (one-launch update's grid barrier)
+    int pad;
 };
 
 // Scalars block at the start of every workspace.

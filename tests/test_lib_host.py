@@ -172,14 +172,15 @@ def test_inverse_mode_and_tuning_settings_are_checked():
                            ("svid_beside", (0, 1), (2, -1)),
                            ("nfast", (0, 1), (2, -1)),
                            ("rhs_bn", (0, 128, 256), (64, 1)),
-                           ("solve_bn", (0, 128, 256), (64, 1))):
+                           ("solve_bn", (0, 128, 256), (64, 1)),
+                           ("newton_fused", (0, 1), (2, -1))):
         for v in good:
             assert L.nq_set_tuning(T[key], v) == 0, (key, v)
         for v in bad:
             assert L.nq_set_tuning(T[key], v) == INV, (key, v)
-    assert L.nq_set_tuning(6, 0) == INV
+    assert L.nq_set_tuning(7, 0) == INV
     # back to the defaults
     assert L.nq_set_inverse_mode(0) == 0
     for key, v in (("factor_ctas", -1), ("newton_bn", 0), ("svid_beside", 1), ("nfast", 1),
-                   ("rhs_bn", 0), ("solve_bn", 0)):
+                   ("rhs_bn", 0), ("solve_bn", 0), ("newton_fused", 0)):
         assert L.nq_set_tuning(T[key], v) == 0
