@@ -608,34 +608,51 @@ __global__ void __launch_bounds__(256, 2)
     __shared__ float red[8][32 * NPL];
     __shared__ double sn[8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float bl[NPL], acc[NPL];
+    // b is read from shared memory (its registers go to the next row's prefetch)
+    float *sb = red[0];
+    for (int k = threadIdx.x; k < 32 * NPL; k += blockDim.x)
+        sb[k] = k < r ? (b_in ? b_in[k] : 1.f) : 0.f;
+    __syncthreads();
+    float acc[NPL];
 #pragma unroll
-    for (int u = 0; u < NPL; ++u) {
-        const int k = lane + 32 * u;
-        bl[u] = k < r ? (b_in ? b_in[k] : 1.f) : 0.f;
-        acc[u] = 0.f;
-    }
+    for (int u = 0; u < NPL; ++u) acc[u] = 0.f;
     double nacc = 0.0;
     const int64_t nw = (int64_t)gridDim.x * 8;
-    for (int64_t i = (int64_t)blockIdx.x * 8 + warp; i < rows; i += nw) {
+    // two rows in flight per warp: the next row's loads are issued before this row's sums
+    float cur[NPL], nxt[NPL];
+    int64_t i = (int64_t)blockIdx.x * 8 + warp;
+    if (i < rows) {
         const float *row = S + i * ldf;
-        float sv[NPL];
 #pragma unroll
         for (int u = 0; u < NPL; ++u) {
             const int k = lane + 32 * u;
-            sv[u] = k < r ? fabsf(__ldcg(row + k)) : 0.f;
+            cur[u] = k < r ? __ldcg(row + k) : 0.f;
+        }
+    }
+    for (; i < rows; i += nw) {
+        const int64_t in = i + nw;
+        if (in < rows) {
+            const float *row = S + in * ldf;
+#pragma unroll
+            for (int u = 0; u < NPL; ++u) {
+                const int k = lane + 32 * u;
+                nxt[u] = k < r ? __ldcg(row + k) : 0.f;
+            }
         }
         float t = 0.f;
 #pragma unroll
-        for (int u = 0; u < NPL; ++u) t = fmaf(sv[u], bl[u], t);
+        for (int u = 0; u < NPL; ++u) t = fmaf(fabsf(cur[u]), sb[lane + 32 * u], t);
         t = warp_sum(t);
 #pragma unroll
-        for (int u = 0; u < NPL; ++u) acc[u] = fmaf(sv[u], t, acc[u]);
+        for (int u = 0; u < NPL; ++u) acc[u] = fmaf(fabsf(cur[u]), t, acc[u]);
         if (lane == 0) {
             nacc += (double)t * (double)t;
             if (write_t) tvec[i] = t;
         }
+#pragma unroll
+        for (int u = 0; u < NPL; ++u) cur[u] = nxt[u];
     }
+    __syncthreads();   // every warp is done with sb (it aliases red[0])
 #pragma unroll
     for (int u = 0; u < NPL; ++u) red[warp][lane + 32 * u] = acc[u];
     if (lane == 0) sn[warp] = nacc;
@@ -653,15 +670,15 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-// b'_k = sum over CTAs of partb[.][k] / ||t||: CTA = 32 columns x 8 groups of partial rows;
-// each group walks every 8th partial row, then the 8 group sums are combined in a fixed
-// order (deterministic).  The last pass also writes a = t / ||t||.
-__global__ void __launch_bounds__(256)
+// b'_k = sum over CTAs of partb[.][k] / ||t||: CTA = 32 columns x 32 groups of partial
+// rows; each group walks every 32nd partial row, then the 32 group sums are combined in a
+// fixed order (deterministic).  The last pass also writes a = t / ||t||.
+__global__ void __launch_bounds__(1024)
     svid_reduce_kernel(const float *__restrict__ partb, const double *__restrict__ partn, int nblk,
                        int r, int64_t rows, int last, const float *__restrict__ tvec,
                        float *b_out, float *a_out) {
     __shared__ double s_inv;
-    __shared__ double sg[8][33];
+    __shared__ double sg[32][33];
     if (threadIdx.x < 32) {
         double n2 = 0.0;
         for (int k = threadIdx.x; k < nblk; k += 32) n2 += partn[k];
@@ -678,7 +695,7 @@ __global__ void __launch_bounds__(256)
         double w[4] = {0.0, 0.0, 0.0, 0.0};   // interleaved sums keep the loads in flight
         int k = grp, u = 0;
 #pragma unroll 4
-        for (; k < nblk; k += 8, u = (u + 1) & 3) w[u] += partb[(int64_t)k * r + col];
+        for (; k < nblk; k += 32, u = (u + 1) & 3) w[u] += partb[(int64_t)k * r + col];
         v = (w[0] + w[1]) + (w[2] + w[3]);
     }
     sg[grp][c] = v;
@@ -687,7 +704,7 @@ __global__ void __launch_bounds__(256)
     if (grp == 0 && col < r) {
         double t = 0.0;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) t += sg[g][c];
+        for (int g = 0; g < 32; ++g) t += sg[g][c];
         b_out[col] = (float)(t * inv);
     }
     if (last) {
@@ -731,7 +748,7 @@ static cudaError_t svid_passes(const float *S, int64_t rows, int32_t r, int64_t 
         svid_pass2_kernel<ROWS><<<(unsigned)grid, 256, smem, s>>>(S, rows, r, ldf, b_in, tvec,
                                                                  last ? 1 : 0, partb, partn);
         count_launch();
-        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 256, 0, s>>>(
+        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 1024, 0, s>>>(
             partb, partn, (int)grid, r, rows, last ? 1 : 0, tvec, b_out, a);
         count_launch();
     }
@@ -753,7 +770,7 @@ static cudaError_t svid_row_passes(const float *S, int64_t rows, int32_t r, int6
         svid_rows_kernel<NPL><<<(unsigned)grid, 256, 0, s>>>(S, rows, r, ldf, b_in, tvec,
                                                             last ? 1 : 0, partb, partn);
         count_launch();
-        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 256, 0, s>>>(
+        svid_reduce_kernel<<<(unsigned)ceil_div(r, 32), 1024, 0, s>>>(
             partb, partn, (int)grid, r, rows, last ? 1 : 0, tvec, b_out, a);
         count_launch();
     }
