@@ -531,28 +531,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int STAGE_BYTES = (F3 ? 2 : 1) * (A_TILE_BYTES + B_TILE_BYTES);
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
-    // launched with programmatic stream serialization: everything below may read what the
-    // previous kernel of the stream wrote, so wait for its completion first; then let the
-    // next kernel's launch begin (it waits the same way before touching memory)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // gate: the whole launch is skipped on the gate values in gate_skip
-    int gate_v = 0;
-    if (p.gate) {
-        gate_v = *reinterpret_cast<const volatile int *>(p.gate);
-        if ((unsigned)gate_v < 32u && ((p.gate_skip >> gate_v) & 1)) return;
-    }
-    const bool fin = (EPI == EPI_NS2) && gate_v == NS_FINAL;
-    if (EPI == EPI_GRAM && p.ns && blockIdx.x == 0 && threadIdx.x == 0) {
-        p.ns->ticket = 0;
-        p.ns->grid_count = 0;
-        *reinterpret_cast<volatile int *>(&p.ns->gate) = NS_RUNNING;
-    }
-    if (EPI == EPI_GRAM && p.zero)   // counters of a later kernel, zeroed here
-        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words;
-             i += gridDim.x * blockDim.x)
-            p.zero[i] = 0u;
-
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -586,6 +564,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tempty[s], kEpiWarps);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        const int nmaps = F3 ? 2 : p.nseg;
+        for (int g = 0; g < nmaps; ++g) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.a[g])) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.b[g])) : "memory");
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -598,172 +581,199 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // launched with programmatic stream serialization: the set-up above touches no global
+    // memory; everything below may read what the previous kernel of the stream wrote, so
+    // wait for its completion first, then let the next kernel's launch begin (it waits the
+    // same way).  No other GEMM CTA can share this SM (shared memory), so the TMEM
+    // allocation above does not wait on the previous kernel.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // gate: the whole launch is skipped on the gate values in gate_skip
+    int gate_v = 0;
+    bool skip = false;
+    if (p.gate) {
+        gate_v = *reinterpret_cast<const volatile int *>(p.gate);
+        skip = (unsigned)gate_v < 32u && ((p.gate_skip >> gate_v) & 1);
+    }
+    const bool fin = (EPI == EPI_NS2) && gate_v == NS_FINAL;
+    if (EPI == EPI_GRAM && p.ns && blockIdx.x == 0 && threadIdx.x == 0) {
+        p.ns->ticket = 0;
+        p.ns->grid_count = 0;
+        *reinterpret_cast<volatile int *>(&p.ns->gate) = NS_RUNNING;
+    }
+    if (EPI == EPI_GRAM && p.zero)   // counters of a later kernel, zeroed here
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words;
+             i += gridDim.x * blockDim.x)
+            p.zero[i] = 0u;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            // TMA producer
-            uint32_t it = 0;
-            bool ok = true;
-            for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
-                const int tile = unit % num_tiles, ks = unit / num_tiles;
-                const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
-                int m0, n0;
-                tile_origin<BN>(p, tile, num_m, m0, n0);
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    int seg = 0, k = kb;
-                    if (!F3)
-                        while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
-                    if (p.tri_k && k < (m0 > n0 ? m0 : n0) / BK) continue;
-                    const int s = it % STAGES;
-                    if (it >= STAGES &&
-                        !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, p.err)) {
-                        ok = false;
-                        break;
+    if (!skip) {
+
+        if (warp == 0) {
+            if (lane == 0) {
+                // TMA producer
+                uint32_t it = 0;
+                bool ok = true;
+                for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+                    const int tile = unit % num_tiles, ks = unit / num_tiles;
+                    const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
+                    int m0, n0;
+                    tile_origin<BN>(p, tile, num_m, m0, n0);
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        int seg = 0, k = kb;
+                        if (!F3)
+                            while (seg < p.nseg - 1 && k >= p.kblocks[seg]) k -= p.kblocks[seg++];
+                        if (p.tri_k && k < (m0 > n0 ? m0 : n0) / BK) continue;
+                        const int s = it % STAGES;
+                        if (it >= STAGES &&
+                            !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *a_dst = smem + s * STAGE_BYTES;
+                        mbar_expect_tx(&full_bar[s], STAGE_BYTES);
+                        if constexpr (F3) {
+                            uint8_t *b_dst = a_dst + 2 * A_TILE_BYTES;
+                            tma_load_2d(a_dst, &maps.a[0], k * BK, m0, &full_bar[s]);
+                            tma_load_2d(a_dst + A_TILE_BYTES, &maps.a[1], k * BK, m0, &full_bar[s]);
+                            tma_load_2d(b_dst, &maps.b[0], k * BK, n0, &full_bar[s]);
+                            tma_load_2d(b_dst + B_TILE_BYTES, &maps.b[1], k * BK, n0, &full_bar[s]);
+                        } else {
+                            tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
+                            tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0,
+                                        &full_bar[s]);
+                        }
+                        ++it;
                     }
-                    uint8_t *a_dst = smem + s * STAGE_BYTES;
-                    mbar_expect_tx(&full_bar[s], STAGE_BYTES);
-                    if constexpr (F3) {
-                        uint8_t *b_dst = a_dst + 2 * A_TILE_BYTES;
-                        tma_load_2d(a_dst, &maps.a[0], k * BK, m0, &full_bar[s]);
-                        tma_load_2d(a_dst + A_TILE_BYTES, &maps.a[1], k * BK, m0, &full_bar[s]);
-                        tma_load_2d(b_dst, &maps.b[0], k * BK, n0, &full_bar[s]);
-                        tma_load_2d(b_dst + B_TILE_BYTES, &maps.b[1], k * BK, n0, &full_bar[s]);
-                    } else {
-                        tma_load_2d(a_dst, &maps.a[seg], k * BK, m0, &full_bar[s]);
-                        tma_load_2d(a_dst + A_TILE_BYTES, &maps.b[seg], k * BK, n0,
-                                    &full_bar[s]);
-                    }
-                    ++it;
                 }
             }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // MMA issuer
-            constexpr uint32_t idesc = instr_desc_bf16(BM, BN);
-            uint32_t it = 0;
-            bool ok = true;
+        } else if (warp == 1) {
+            if (lane == 0) {
+                // MMA issuer
+                constexpr uint32_t idesc = instr_desc_bf16(BM, BN);
+                uint32_t it = 0;
+                bool ok = true;
+                int lt = 0;
+                for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x, ++lt) {
+                    const int tile = unit % num_tiles, ks = unit / num_tiles;
+                    const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
+                    const int as = lt & 1;
+                    int m0, n0;
+                    tile_origin<BN>(p, tile, num_m, m0, n0);
+                    if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + (uint32_t)(as * BN);
+                    bool first = true;
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (p.tri_k) {
+                            int seg = 0, k = kb;
+                            if (!F3)
+                                while (seg < p.nseg - 1 && k >= p.kblocks[seg])
+                                    k -= p.kblocks[seg++];
+                            if (k < (m0 > n0 ? m0 : n0) / BK) continue;
+                        }
+                        const int s = it % STAGES;
+                        if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint8_t *a_src = smem + s * STAGE_BYTES;
+                        if constexpr (F3) {
+                            const uint64_t ah = smem_desc_sw128(a_src);
+                            const uint64_t al = smem_desc_sw128(a_src + A_TILE_BYTES);
+                            const uint64_t bh = smem_desc_sw128(a_src + 2 * A_TILE_BYTES);
+                            const uint64_t bl = smem_desc_sw128(a_src + 2 * A_TILE_BYTES + B_TILE_BYTES);
+    #pragma unroll
+                            for (int k = 0; k < BK / 16; ++k)
+                                mma_bf16(d, ah + 2 * k, bh + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+    #pragma unroll
+                            for (int k = 0; k < BK / 16; ++k) mma_bf16(d, al + 2 * k, bh + 2 * k, idesc, 1u);
+    #pragma unroll
+                            for (int k = 0; k < BK / 16; ++k) mma_bf16(d, ah + 2 * k, bl + 2 * k, idesc, 1u);
+                        } else {
+                            const uint64_t adesc = smem_desc_sw128(a_src);
+                            const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
+    #pragma unroll
+                            for (int k = 0; k < BK / 16; ++k)
+                                mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                         (first && k == 0) ? 0u : 1u);
+                        }
+                        mma_commit(&empty_bar[s]);
+                        first = false;
+                        ++it;
+                    }
+                    if (ok) mma_commit(&tfull[as]);
+                }
+            }
+        } else {
+            // epilogue warps.  Every epilogue warp walks the same tiles and reaches the same
+            // named barriers, also after a timed-out wait (then it only skips the work).
+            const int q = warp & 3;
             int lt = 0;
-            for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x, ++lt) {
-                const int tile = unit % num_tiles, ks = unit / num_tiles;
-                const int kb0 = ks * kchunk, kb1 = min(total_kb, kb0 + kchunk);
+            bool dead = false;
+            for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++lt) {
+                const int tile = unit % num_tiles;
                 const int as = lt & 1;
                 int m0, n0;
                 tile_origin<BN>(p, tile, num_m, m0, n0);
-                if (lt >= 2 && !mbar_wait(&tempty[as], ((lt >> 1) - 1) & 1, p.err)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)(as * BN);
-                bool first = true;
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    if (p.tri_k) {
-                        int seg = 0, k = kb;
-                        if (!F3)
-                            while (seg < p.nseg - 1 && k >= p.kblocks[seg])
-                                k -= p.kblocks[seg++];
-                        if (k < (m0 > n0 ? m0 : n0) / BK) continue;
-                    }
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, p.err)) {
-                        ok = false;
-                        break;
-                    }
+                const int row = m0 + 32 * q + lane;
+                float acc_sum = 0.f, acc_aux = 0.f;
+                if (!dead) {
+                    // one lane waits; the outcome is broadcast so that the warp-collective
+                    // tcgen05.ld below is executed by all 32 lanes or by none
+                    int ok = 0;
+                    if (lane == 0) ok = mbar_wait(&tfull[as], (lt >> 1) & 1, p.err) ? 1 : 0;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    dead = !ok;
+                }
+                if (!dead) {
                     tc_fence_after();
-                    const uint8_t *a_src = smem + s * STAGE_BYTES;
-                    if constexpr (F3) {
-                        const uint64_t ah = smem_desc_sw128(a_src);
-                        const uint64_t al = smem_desc_sw128(a_src + A_TILE_BYTES);
-                        const uint64_t bh = smem_desc_sw128(a_src + 2 * A_TILE_BYTES);
-                        const uint64_t bl = smem_desc_sw128(a_src + 2 * A_TILE_BYTES + B_TILE_BYTES);
-#pragma unroll
-                        for (int k = 0; k < BK / 16; ++k)
-                            mma_bf16(d, ah + 2 * k, bh + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
-#pragma unroll
-                        for (int k = 0; k < BK / 16; ++k) mma_bf16(d, al + 2 * k, bh + 2 * k, idesc, 1u);
-#pragma unroll
-                        for (int k = 0; k < BK / 16; ++k) mma_bf16(d, ah + 2 * k, bl + 2 * k, idesc, 1u);
-                    } else {
-                        const uint64_t adesc = smem_desc_sw128(a_src);
-                        const uint64_t bdesc = smem_desc_sw128(a_src + A_TILE_BYTES);
-#pragma unroll
-                        for (int k = 0; k < BK / 16; ++k)
-                            mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc,
-                                     (first && k == 0) ? 0u : 1u);
+                    const uint32_t tbase = tmem + (uint32_t)(as * BN) + ((uint32_t)(32 * q) << 16);
+    #pragma unroll 1
+                    for (int c = 0; c < BN; c += 16) {
+                        float v[16];
+                        tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
+                        if (EPI == EPI_GRAM && ksplit > 1) {
+                            // split-K partial: the unit's raw 128 x 128 tile, reduced later
+                            st16(p.out + ((int64_t)unit * BM + 32 * q + lane) * BM + c, v);
+                        } else if (row < p.M && n0 + c < p.N) {
+                            epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum, acc_aux, fin);
+                            if constexpr (EPI == EPI_SPLIT)
+                                if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
+                            if constexpr (EPI == EPI_GRAM)
+                                if (p.sym && m0 != n0) gram_mirror(p, row, n0 + c, v);
+                        }
                     }
-                    mma_commit(&empty_bar[s]);
-                    first = false;
-                    ++it;
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[as]);
                 }
-                if (ok) mma_commit(&tfull[as]);
-            }
-        }
-    } else {
-        // epilogue warps.  Every epilogue warp walks the same tiles and reaches the same
-        // named barriers, also after a timed-out wait (then it only skips the work).
-        const int q = warp & 3;
-        int lt = 0;
-        bool dead = false;
-        for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++lt) {
-            const int tile = unit % num_tiles;
-            const int as = lt & 1;
-            int m0, n0;
-            tile_origin<BN>(p, tile, num_m, m0, n0);
-            const int row = m0 + 32 * q + lane;
-            float acc_sum = 0.f, acc_aux = 0.f;
-            if (!dead) {
-                // one lane waits; the outcome is broadcast so that the warp-collective
-                // tcgen05.ld below is executed by all 32 lanes or by none
-                int ok = 0;
-                if (lane == 0) ok = mbar_wait(&tfull[as], (lt >> 1) & 1, p.err) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                dead = !ok;
-            }
-            if (!dead) {
-                tc_fence_after();
-                const uint32_t tbase = tmem + (uint32_t)(as * BN) + ((uint32_t)(32 * q) << 16);
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(tbase + c, v);  // warp-collective: every lane takes part
-                    if (EPI == EPI_GRAM && ksplit > 1) {
-                        // split-K partial: the unit's raw 128 x 128 tile, reduced later
-                        st16(p.out + ((int64_t)unit * BM + 32 * q + lane) * BM + c, v);
-                    } else if (row < p.M && n0 + c < p.N) {
-                        epilogue_chunk<EPI>(p, row, n0 + c, v, acc_sum, acc_aux, fin);
-                        if constexpr (EPI == EPI_SPLIT)
-                            if (p.sym && m0 != n0) split_mirror(p, row, n0 + c, v);
-                        if constexpr (EPI == EPI_GRAM)
-                            if (p.sym && m0 != n0) gram_mirror(p, row, n0 + c, v);
+                if constexpr (EPI == EPI_REFIT) {
+                    // one thread owns (row, this tile's columns): its sums are the partials
+                    if (!dead && row < p.M) {
+                        const int64_t o = (int64_t)(n0 / BN) * p.M + row;
+                        p.num[o] = (double)acc_sum;
+                        p.den[o] = (double)acc_aux;
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[as]);
-            }
-            if constexpr (EPI == EPI_REFIT) {
-                // one thread owns (row, this tile's columns): its sums are the partials
-                if (!dead && row < p.M) {
-                    const int64_t o = (int64_t)(n0 / BN) * p.M + row;
-                    p.num[o] = (double)acc_sum;
-                    p.den[o] = (double)acc_aux;
+                if constexpr (EPI == EPI_NS1 || EPI == EPI_NS2) {
+                    if constexpr (EPI == EPI_NS1) {
+                        const double w = warp_sum((double)acc_sum);
+                        if (lane == 0) red[as][warp - 2] = dead ? __longlong_as_double(-1ll) : w;
+                        epilogue_bar();
+                    }
+                    if (warp == 2) ns_tile_done<EPI>(p, tile, num_tiles, lane, red[as], fin);
                 }
-            }
-            if constexpr (EPI == EPI_NS1 || EPI == EPI_NS2) {
-                if constexpr (EPI == EPI_NS1) {
-                    const double w = warp_sum((double)acc_sum);
-                    if (lane == 0) red[as][warp - 2] = dead ? __longlong_as_double(-1ll) : w;
-                    epilogue_bar();
-                }
-                if (warp == 2) ns_tile_done<EPI>(p, tile, num_tiles, lane, red[as], fin);
-            }
-            if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
-                if (p.part && (EPI == EPI_RECON || p.objective)) {
-                    const double w = warp_sum((double)acc_sum);
-                    if (lane == 0) red[as][warp - 2] = w;
-                    epilogue_bar();
-                    if (warp == 2 && lane == 0) {
-                        double t = 0.0;
-                        for (int e = 0; e < kEpiWarps; ++e) t += red[as][e];
-                        p.part[tile] = t;
+                if constexpr (EPI == EPI_SOLVE || EPI == EPI_RECON) {
+                    if (p.part && (EPI == EPI_RECON || p.objective)) {
+                        const double w = warp_sum((double)acc_sum);
+                        if (lane == 0) red[as][warp - 2] = w;
+                        epilogue_bar();
+                        if (warp == 2 && lane == 0) {
+                            double t = 0.0;
+                            for (int e = 0; e < kEpiWarps; ++e) t += red[as][e];
+                            p.part[tile] = t;
+                        }
                     }
                 }
             }

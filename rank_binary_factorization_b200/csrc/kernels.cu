@@ -605,7 +605,9 @@ __global__ void __launch_bounds__(256, 2)
     svid_rows_kernel(const float *__restrict__ S, int64_t rows, int r, int64_t ldf,
                      const float *__restrict__ b_in, float *tvec, int write_t, float *partb,
                      double *partn) {
-    __shared__ float red[8][32 * NPL];
+    // 16 KB of partial rows (the warps' column sums are combined in two rounds), so that a
+    // CTA fits on an SM beside a GEMM CTA of the half step it runs beside
+    __shared__ float red[4][32 * NPL];
     __shared__ double sn[8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // b is read from shared memory (its registers go to the next row's prefetch)
@@ -653,14 +655,21 @@ __global__ void __launch_bounds__(256, 2)
         for (int u = 0; u < NPL; ++u) cur[u] = nxt[u];
     }
     __syncthreads();   // every warp is done with sb (it aliases red[0])
+    if (warp >= 4) {
 #pragma unroll
-    for (int u = 0; u < NPL; ++u) red[warp][lane + 32 * u] = acc[u];
+        for (int u = 0; u < NPL; ++u) red[warp - 4][lane + 32 * u] = acc[u];
+    }
     if (lane == 0) sn[warp] = nacc;
+    __syncthreads();
+    if (warp < 4) {
+#pragma unroll
+        for (int u = 0; u < NPL; ++u) red[warp][lane + 32 * u] += acc[u];
+    }
     __syncthreads();
     for (int k = threadIdx.x; k < r; k += blockDim.x) {
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[w][k];
+        for (int w = 0; w < 4; ++w) v += red[w][k];
         partb[(int64_t)blockIdx.x * r + k] = v;
     }
     if (threadIdx.x == 0) {
