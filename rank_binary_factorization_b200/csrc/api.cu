@@ -208,7 +208,7 @@ nq_status enqueue_stats(const void *X, int64_t T, int64_t C, int bf16, double *s
 // The same context also holds the auxiliary stream of the SVID passes, which run beside
 // the next half step's RHS GEMM and solve (see lb_iterate), with its events.
 struct SideCtx {
-    cudaStream_t side = nullptr, aux = nullptr;
+    cudaStream_t side = nullptr, aux = nullptr, obj = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr, pre_rhs = nullptr, obj_done = nullptr,
                 svid_done[2] = {nullptr, nullptr};
 };
@@ -222,6 +222,7 @@ nq_status side_ctx(SideCtx **out) {
         // default priority: raising either stream above the caller's was measured slower
         NQ_CK(cudaStreamCreateWithFlags(&c.side, cudaStreamNonBlocking));
         NQ_CK(cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking));
+        NQ_CK(cudaStreamCreateWithFlags(&c.obj, cudaStreamNonBlocking));
         for (cudaEvent_t *e :
              {&c.fork, &c.join, &c.pre_rhs, &c.obj_done, &c.svid_done[0], &c.svid_done[1]})
             NQ_CK(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
@@ -590,8 +591,10 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         NQ_CK(cudaEventRecord(ov->pre_rhs, s));
         NQ_CK(cudaStreamWaitEvent(ov->aux, ov->pre_rhs, 0));
         if (obj_slot >= 0) {    // the previous iteration's objective: both Grams are formed
-            if ((st = lb_objective(lb, lambda + rho, obj_slot, ov->aux))) return st;
-            NQ_CK(cudaEventRecord(ov->obj_done, ov->aux));
+            // (its own stream: behind the SVID passes it could hold up the next Gram)
+            NQ_CK(cudaStreamWaitEvent(ov->obj, ov->pre_rhs, 0));
+            if ((st = lb_objective(lb, lambda + rho, obj_slot, ov->obj))) return st;
+            NQ_CK(cudaEventRecord(ov->obj_done, ov->obj));
         }
         if ((st = lb_svid(lb, pending, K, ov->aux))) return st;
         NQ_CK(cudaEventRecord(ov->svid_done[pending], ov->aux));
@@ -744,7 +747,8 @@ nq_status lb_iterate_tail(const Lb &lb, float rho, float lambda, int iters, int 
 // RHS GEMM, one half step later, so it runs on the auxiliary stream beside the next half
 // step's RHS GEMM and solve; the last one runs on ``s`` before returning.  The objective of
 // iteration t - 1 needs both Grams, the second formed at the start of iteration t: it runs
-// on the auxiliary stream too, before the next Gram of U overwrites the first.
+// on a stream of its own beside the U half step, before the next Gram of U overwrites the
+// first.
 nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, int prec,
                      float *objective_h, cudaStream_t s) {
     SideCtx *ov = nullptr;
@@ -781,9 +785,10 @@ nq_status lb_iterate(const Lb &lb, float rho, float lambda, int iters, int K, in
                                   (size_t)kObjRing * 4, cudaMemcpyDeviceToHost, s));
         }
     }
-    // join the auxiliary stream (the last SVID of U; the SVID scratch is shared), then the
-    // last SVID of V
+    // join the auxiliary stream (the last SVID of U; the SVID scratch is shared) and the
+    // objective stream, then the last SVID of V
     NQ_CK(cudaStreamWaitEvent(s, ov->svid_done[0], 0));
+    if (iters > 1) NQ_CK(cudaStreamWaitEvent(s, ov->obj_done, 0));
     if ((st = lb_svid(lb, 1, K, s))) return st;
     return lb_iterate_tail(lb, rho, lambda, iters, prec, objective_h, s);
 }
