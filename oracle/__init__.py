@@ -17,6 +17,7 @@ Modules
 ``lbadmm``   the Latent Binary ADMM iteration, magnitude balancing, scale
              extraction, sign packing and the reconstruction error.
 ``brute``    exhaustive sign-pattern search on tiny matrices (C, via ctypes).
+``gd``       the gradient-descent latent update (a solver variant) and LB-ADMM with it.
 
 Every function names the passage of the pages it follows.  Where the pages are
 silent the plainest reading is taken and stated in the function's docstring.
