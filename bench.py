@@ -214,6 +214,34 @@ def roofline_entry(cls, launches, ms, m, n, r, K, T, peaks, ns_steps=4):
                 share_of_step=None, peak_kind=peak_kind)
 
 
+def time_gd_variant(nq, W, acts, grads, calib_ws, lb_ws, r, iters, rho, lam, K, exact_err,
+                    stream, steps=8):
+    """The gradient-descent latent update in place of the exact solve (community blog page,
+    to-do section): one warm-up and one timed step of the same workload."""
+    import torch
+    nq.nq_set_latent_solver("gd", steps)
+    try:
+        def step():
+            d_in, d_out, _, _ = nq.nq_calib_precond(acts, grads, ws=calib_ws, sync=False)
+            return nq.nq_lbadmm(W, r, d_in, d_out, rho=rho, lam=lam, iters=iters, K=K, seed=0,
+                                ws=lb_ws)
+        step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        res = step()
+        e1.record(stream)
+        e1.synchronize()
+    finally:
+        nq.nq_set_latent_solver("exact")
+    ms = e0.elapsed_time(e1)
+    return {"gd": dict(steps_per_half_iteration=steps, ms_per_step=round(ms, 3),
+                       layer_iters_per_s=round(iters / (ms / 1e3), 3),
+                       rel_err=res["rel_err"], rel_err_exact=exact_err,
+                       note="inexact latent updates: a different trajectory from the exact "
+                            "LB-ADMM; one timed step")}
+
+
 def time_binary_matmul(nq, res, m, n, r, peaks, reps=10):
     """Device time of nq_binary_matmul on the packed result: batch 1 (packed-bit GEMV path)
     and batch 256 (tensor-core path, sign expansion included).  L2 is flushed before each
@@ -527,6 +555,9 @@ def run_ours(args):
         rel_err=res["rel_err"])
     if not args.no_binary:
         line["binary_matmul"] = time_binary_matmul(nq, res, m, n, r, peaks)
+    if not args.no_variants:
+        line["solver_variants"] = time_gd_variant(nq, W, acts, grads, calib_ws, lb_ws, r, iters,
+                                                  rho, lam, K, res["rel_err"], stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, info = oracle_sample(W_h, acts_h, grads_h, r, iters, T)
         info["value"] = round(v, 5)
@@ -548,6 +579,8 @@ def main():
     ap.add_argument("--iters", type=int, default=WORKLOAD["iters"])
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the timing of the gradient-descent latent-update variant")
     ap.add_argument("--no-binary", action="store_true",
                     help="skip the timing of nq_binary_matmul on the packed result")
     ap.add_argument("--workload", choices=["gate_proj", "q_proj", "profile", "q_proj_profile"],

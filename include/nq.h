@@ -175,6 +175,20 @@ typedef enum { NQ_INV_AUTO = 0, NQ_INV_CHOLESKY = 1, NQ_INV_NEWTON = 2 } nq_inve
 nq_status nq_set_inverse_mode(nq_inverse_mode mode);
 
 /*
+ * The latent update of each half step (a measured variant; community blog page, to-do
+ * section: a gradient-descent solver in place of the Cholesky solves).
+ * NQ_SOLVER_EXACT (default): X = R G^-1, the exact minimiser (G^-1 as nq_set_inverse_mode).
+ * NQ_SOLVER_GD: gd_steps (1..1000) gradient steps on the same objective from the side's
+ *   current latent, X <- X - eta (X G - R) with eta = 1 / max_i sum_j |G_ij|, each a
+ *   split-BF16 tensor-core GEMM X G whose epilogue takes the step.  An inexact update: the
+ *   iterates differ from the exact LB-ADMM's (equal as gd_steps grows).
+ * Process-wide; read when a half step is enqueued.  NQ_ERR_INVALID_ARG for an unknown
+ * solver or a step count out of range.
+ */
+typedef enum { NQ_SOLVER_EXACT = 0, NQ_SOLVER_GD = 1 } nq_latent_solver;
+nq_status nq_set_latent_solver(nq_latent_solver solver, int32_t gd_steps);
+
+/*
  * Scheduling settings of the LB-ADMM iterations (process-wide; none changes a result):
  * NQ_TUNE_FACTOR_CTAS: CTAs given to forming G^-1 (factorisation or update) while the
  *   RHS GEMM runs on the other SMs: -1 (default) half of the SMs up to r = 1536, else no
@@ -401,7 +415,8 @@ typedef enum {
     NQ_K_BINARY = 12,   /* binary GEMV/GEMM on the packed factors                    */
     NQ_K_REFIT = 13,    /* least-squares scale refit                                 */
     NQ_K_NEWTON = 14,   /* tcgen05 Newton-Schulz update of G^-1                      */
-    NQ_K_COUNT = 15
+    NQ_K_GD = 15,       /* gradient-descent latent update (solver variant)           */
+    NQ_K_COUNT = 16
 } nq_kernel_class;
 
 /* Number of kernel launches the library has issued in this process. */

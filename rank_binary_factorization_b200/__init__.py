@@ -24,7 +24,7 @@ __all__ = [
     "nq_recon_error", "nq_pack_signs", "nq_binary_matmul", "nq_ls_refit", "LBState", "NQError",
     "status_string", "lib",
     "nq_launch_count", "nq_profile_enable", "nq_profile_get", "nq_selftest",
-    "nq_set_inverse_mode", "nq_set_tuning",
+    "nq_set_inverse_mode", "nq_set_tuning", "nq_set_latent_solver",
 ]
 
 
@@ -177,6 +177,12 @@ def nq_set_inverse_mode(mode):
     code = {"auto": _lib.NQ_INV_AUTO, "cholesky": _lib.NQ_INV_CHOLESKY,
             "newton": _lib.NQ_INV_NEWTON}[mode]
     check("nq_set_inverse_mode", lib.nq_set_inverse_mode(code))
+
+
+def nq_set_latent_solver(solver="exact", gd_steps=8):
+    """Latent update of each half step: "exact" (default) or "gd" (gd_steps gradient steps)."""
+    code = {"exact": _lib.NQ_SOLVER_EXACT, "gd": _lib.NQ_SOLVER_GD}[solver]
+    check("nq_set_latent_solver", lib.nq_set_latent_solver(code, int(gd_steps)))
 
 
 def nq_set_tuning(key, value):

@@ -28,6 +28,7 @@ NQ_PREC_BF16, NQ_PREC_FP32 = 0, 1
 FIELDS = dict(U=0, V=1, SU=2, SV=3, AU=4, AV=5, BU=6, BV=7, WHAT=8, GAMMA=9, WHAT_LO=10,
               INV_STATS=11, GINV_U=12, GINV_U_LO=13, GINV_V=14, GINV_V_LO=15)
 NQ_INV_AUTO, NQ_INV_CHOLESKY, NQ_INV_NEWTON = 0, 1, 2
+NQ_SOLVER_EXACT, NQ_SOLVER_GD = 0, 1
 TUNING = dict(factor_ctas=0, newton_bn=1, svid_beside=2, nfast=3, rhs_bn=4, solve_bn=5,
               newton_fused=6)
 
@@ -45,6 +46,7 @@ SIGNATURES = {
     "nq_lbadmm_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
     "nq_set_inverse_mode": (c_i32, [c_i32]),
     "nq_set_tuning": (c_i32, [c_i32, c_i32]),
+    "nq_set_latent_solver": (c_i32, [c_i32, c_i32]),
     "nq_lbadmm": (c_i32, [c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_f32, c_f32, c_i32,
                           c_i32, c_u64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "nq_recon_workspace_size": (c_sz, [c_i64, c_i64, c_i32]),
@@ -78,7 +80,7 @@ SIGNATURES = {
 }
 NQ_SELFTEST_WAIT_TIMEOUT, NQ_SELFTEST_NOT_SPD = 0, 1
 KERNEL_CLASSES = ["calib", "calib_finalize", "prep", "gram", "chol", "rhs", "solve", "svid",
-                  "objective", "finish", "recon", "ginv", "binary", "refit", "newton"]
+                  "objective", "finish", "recon", "ginv", "binary", "refit", "newton", "gd"]
 
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(lib, _name)

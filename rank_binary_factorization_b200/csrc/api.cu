@@ -74,7 +74,7 @@ bool g_prof_on = false;
 const char *const kClassNames[NQ_K_COUNT] = {
     "nq.calib", "nq.calib_finalize", "nq.prep", "nq.gram", "nq.chol", "nq.rhs",
     "nq.solve", "nq.svid", "nq.objective", "nq.finish", "nq.recon", "nq.ginv", "nq.binary",
-    "nq.refit", "nq.newton"};
+    "nq.refit", "nq.newton", "nq.gd"};
 
 // Scope of one kernel class's launches: an NVTX range on the host timeline (seen by
 // profilers; inert otherwise) and, when recording is on, a CUDA event pair on the stream.
@@ -351,6 +351,10 @@ constexpr float kNsTau = 1e-2f;      // ||E_k||_F that makes X_{k+1} final (||E|
 
 std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
 
+// Latent update: the exact solve (default) or gradient-descent steps (nq_set_latent_solver).
+std::atomic<int> g_solver{NQ_SOLVER_EXACT};
+std::atomic<int> g_gd_steps{8};
+
 // Performance settings of nq_set_tuning (none changes a result).
 std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}, {0}, {0}, {0}};
 
@@ -514,6 +518,58 @@ nq_status lb_newton(const Lb &lb, int side, int max_ctas, cudaStream_t s) {
 // dual state a, b it writes).
 nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s);
 
+// Gradient-descent latent update (solver variant): X <- X - eta (X G - R), g_gd_steps steps
+// from the side's current latent, each one split-BF16 GEMM X G (K = r) whose epilogue
+// takes the step and writes the next operand; then the state update of the exact path's
+// solve epilogue (dual state, transposed operand copy, objective partials on the V side).
+nq_status lb_gd_steps(const Lb &lb, int side, float rho, int prec, cudaStream_t s) {
+    const LbLayout &L = lb.L;
+    const int other = 1 - side;
+    const int64_t rows = L.rows(side);
+    const int BN = solve_bn(L.r);
+    const int steps = g_gd_steps.load(std::memory_order_relaxed);
+    ProfScope ps(NQ_K_GD, s);
+    NQ_CK(split_rows(lb.p<float>(L.x[side]), rows, L.r, L.ldr, lb.p<__nv_bfloat16>(L.gdh[0]),
+                     lb.p<__nv_bfloat16>(L.gdl[0]), L.ldr, s));
+    for (int j = 0; j < steps; ++j) {
+        const int a = j & 1, w = 1 - a;
+        tc::Maps maps;
+        memset(&maps, 0, sizeof(maps));
+        if (!tc::make_map_bf16(&maps.a[0], lb.p<void>(L.gdh[a]), rows, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.a[1], lb.p<void>(L.gdl[a]), rows, L.r, L.ldr, tc::BM) ||
+            !tc::make_map_bf16(&maps.b[0], lb.p<void>(L.gsh), L.r, L.r, L.ldr, BN) ||
+            !tc::make_map_bf16(&maps.b[1], lb.p<void>(L.gsl), L.r, L.r, L.ldr, BN))
+            return NQ_ERR_CUDA;
+        tc::EpiParams ep;
+        memset(&ep, 0, sizeof(ep));
+        ep.M = (int)rows;
+        ep.N = L.r;
+        ep.nseg = 1;
+        ep.split3 = 1;
+        ep.kblocks[0] = (int)ceil_div(L.r, tc::BK);
+        ep.nfast = 1;
+        ep.err = &lb.sc->err;
+        ep.X = lb.p<float>(L.x[side]);
+        ep.ldf = L.ldr;
+        ep.Ph = lb.p<__nv_bfloat16>(L.rhi);
+        ep.Pl = lb.p<__nv_bfloat16>(L.rlo);
+        ep.ldr = L.ldr;
+        ep.Fhi = lb.p<__nv_bfloat16>(L.gdh[w]);
+        ep.Flo = lb.p<__nv_bfloat16>(L.gdl[w]);
+        ep.gd_max = lb.p<float>(L.gdmax);
+        NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_GD, BN, s));
+    }
+    const int npx = (int)tc::num_tiles((int)L.n, L.r, solve_bn(L.r));
+    NQ_CK(gd_finalize(lb.p<float>(L.x[side]), lb.p<float>(L.s[side]), lb.p<float>(L.a[side]),
+                      lb.p<float>(L.b[side]), rows, L.r, L.ldr, rho, lb.p<__nv_bfloat16>(L.rhi),
+                      lb.p<__nv_bfloat16>(L.rlo), L.ldr, lb.p<__nv_bfloat16>(L.xt[side]),
+                      prec == NQ_PREC_FP32 ? lb.p<__nv_bfloat16>(L.xtl[side]) : nullptr,
+                      L.ld_rows(side), side == 1, lb.p<double>(L.part),
+                      side == 1 ? npx : kRedBlocks, &lb.sc->err, s));
+    (void)other;
+    return NQ_OK;
+}
+
 nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, int prec,
                        cudaStream_t s, SideCtx *ov = nullptr, int pending = -1,
                        bool wait_own = false, int obj_slot = -1, bool wait_obj = false) {
@@ -523,19 +579,28 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     const int other = 1 - side;
     const int64_t rows = L.rows(side), Kd = L.rows(other);
     const int BN = rhs_bn(L.r), BNs = solve_bn(L.r);
+    const bool gd = g_solver.load(std::memory_order_relaxed) == NQ_SOLVER_GD;
     const int mode = g_inverse_mode.load(std::memory_order_relaxed);
-    const bool newton = mode == NQ_INV_NEWTON ||
-                        (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
-                         iters_since_prepare(lb.ws) >= ns_first_iter(L.r));
+    const bool newton = !gd && (mode == NQ_INV_NEWTON ||
+                                (mode == NQ_INV_AUTO && L.r >= kNsMinRank &&
+                                 iters_since_prepare(lb.ws) >= ns_first_iter(L.r)));
     NsState *ns = lb.p<NsState>(L.ns);
-    nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton, true);
+    // the update and the gradient steps take the Gram split into hi + lo as their operand
+    nq_status st = lb_gram(lb, other, lambda + rho, prec, s, newton || gd, !gd);
     if (st) return st;
+    if (gd) {   // step size 1 / max_i sum_j |G_ij|
+        ProfScope ps(NQ_K_GD, s);
+        NQ_CK(cudaMemsetAsync(lb.p<void>(L.gdmax), 0, sizeof(unsigned int), s));
+        NQ_CK(gd_rowabs_max(lb.p<float>(L.g[other]), L.r, lb.p<unsigned int>(L.gdmax), s));
+    }
     // The factorisation of G and the G^-1 GEMM depend only on the Gram; the RHS GEMM only
     // on the other side's operand and this side's dual state.  With overlap they run at
     // once: the factorisation on ``cc`` CTAs of a side stream, the RHS GEMM on the rest.
     const int sms = device_sm_count();
     const int fc = g_tune[NQ_TUNE_FACTOR_CTAS].load(std::memory_order_relaxed);
-    const int cc = fc < 0 ? chol_ctas(L.r, sms) : (fc == 0 ? 0 : std::min(std::max(fc, 3), sms - 1));
+    const int cc = gd ? 0
+                      : (fc < 0 ? chol_ctas(L.r, sms)
+                                : (fc == 0 ? 0 : std::min(std::max(fc, 3), sms - 1)));
     SideCtx *sc = nullptr;
     if (cc > 0 && (st = side_ctx(&sc))) return st;
     cudaStream_t fs = s;   // stream of the factorisation
@@ -548,14 +613,14 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
     // with the update, the factorisation and the G^-1 GEMM run only if it failed
     const int *gate = newton ? &ns->gate : nullptr;
     const int gate_skip = newton ? (1 << NS_DONE) : 0;
-    {
+    if (!gd) {
         ProfScope ps(NQ_K_CHOL, fs);
         NQ_CK(chol_inverse(lb.p<float>(L.g[other]), L.r, L.rp, lb.p<float>(L.chA),
                            lb.p<float>(L.chLi), lb.p<__nv_bfloat16>(L.lth),
                            lb.p<__nv_bfloat16>(L.ltl), L.ldr, lb.p<unsigned int>(L.chF),
                            &lb.sc->err, lb.sc->bar, cc, gate, gate_skip, false, fs));
     }
-    {
+    if (!gd) {
         ProfScope ps(NQ_K_GINV, fs);
         // G^-1 = Li^T Li = LiT LiT^T as three split-BF16 passes, written as hi + lo; G^-1 is
         // symmetric, so only its lower-triangular tiles are computed and mirrored
@@ -638,6 +703,11 @@ nq_status lb_half_step(const Lb &lb, int side, float rho, float lambda, int K, i
         NQ_CK(tc::launch_gemm(maps, ep, tc::EPI_RHS, BN, s));
     }
     if (cc > 0) NQ_CK(cudaStreamWaitEvent(s, sc->join, 0));
+    if (gd) {
+        if ((st = lb_gd_steps(lb, side, rho, prec, s))) return st;
+        if (ov) return NQ_OK;
+        return lb_svid(lb, side, K, s);
+    }
     // X = R G^-1 = [R_hi, R_lo, R_hi] [Gi_hi; Gi_hi; Gi_lo]; S <- X + L; Xt = bf16(X)^T
     {
         tc::Maps maps;
@@ -954,6 +1024,14 @@ nq_status nq_set_tuning(nq_tuning key, int32_t value) {
         default: return NQ_ERR_INVALID_ARG;
     }
     g_tune[key].store(value, std::memory_order_relaxed);
+    return NQ_OK;
+}
+
+nq_status nq_set_latent_solver(nq_latent_solver solver, int32_t gd_steps) {
+    if (solver != NQ_SOLVER_EXACT && solver != NQ_SOLVER_GD) return NQ_ERR_INVALID_ARG;
+    if (solver == NQ_SOLVER_GD && (gd_steps < 1 || gd_steps > 1000)) return NQ_ERR_INVALID_ARG;
+    if (solver == NQ_SOLVER_GD) g_gd_steps.store(gd_steps, std::memory_order_relaxed);
+    g_solver.store(solver, std::memory_order_relaxed);
     return NQ_OK;
 }
 

@@ -228,6 +228,37 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams &p, int row, int 
         }
         split_store(p.Rhi + so, p.Rlo + so, full, p.N - col0, e);
         acc_sum += part;
+    } else if constexpr (EPI == EPI_GD) {
+        const int64_t so = (int64_t)row * p.ldr + col0;
+        float *Xrow = p.X + (int64_t)row * p.ldf + col0;
+        const float eta = 1.f / *p.gd_max;
+        float rh[16], rl[16], x[16];
+        bool bad = false;
+        if (full) {
+            ld16_bf16(rh, p.Ph + so);
+            ld16_bf16(rl, p.Pl + so);
+            ld16(x, Xrow);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const bool in = col0 + j < p.N;
+                rh[j] = in ? __bfloat162float(p.Ph[so + j]) : 0.f;
+                rl[j] = in ? __bfloat162float(p.Pl[so + j]) : 0.f;
+                x[j] = in ? Xrow[j] : 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            x[j] = x[j] - eta * (v[j] - (rh[j] + rl[j]));
+            bad |= !isfinite(x[j]);
+        }
+        if (full) {
+            st16(Xrow, x);
+        } else {
+            for (int j = 0; j < 16 && col0 + j < p.N; ++j) Xrow[j] = x[j];
+        }
+        split_store(p.Fhi + so, p.Flo + so, full, p.N - col0, x);
+        if (bad) raise_error(p.err, NQ_ERR_NONFINITE);
     } else if constexpr (EPI == EPI_NS2) {
         const int64_t so = (int64_t)row * p.ldr + col0;
         float xh[16], xl[16], xn[16];
@@ -1184,6 +1215,7 @@ cudaError_t launch_gemm(const Maps &maps, const EpiParams &p, int epi, int BN, c
         case EPI_REFIT: return launch_bn<EPI_REFIT>(maps, p, BN, s);
         case EPI_NS1: return launch_bn<EPI_NS1>(maps, p, BN, s);
         case EPI_NS2: return launch_bn<EPI_NS2>(maps, p, BN, s);
+        case EPI_GD: return launch_bn<EPI_GD>(maps, p, BN, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -28,7 +28,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 enum Epi : int { EPI_GRAM = 0, EPI_RHS = 1, EPI_SOLVE = 2, EPI_RECON = 3, EPI_SPLIT = 4,
-                 EPI_SCALE = 5, EPI_REFIT = 6, EPI_NS1 = 7, EPI_NS2 = 8 };
+                 EPI_SCALE = 5, EPI_REFIT = 6, EPI_NS1 = 7, EPI_NS2 = 8, EPI_GD = 9 };
 
 struct Maps {
     CUtensorMap a[3];
@@ -110,6 +110,10 @@ struct EpiParams {
     // EPI_NS2: acc = (E_k X_k)(row, col); X_{k+1} = (Ph + Pl) + acc split into hi + lo,
     //   written to Rhi/Rlo, or to Fhi/Flo when the gate reads NS_FINAL (then the CTA
     //   finishing the last tile sets NS_DONE).
+    // EPI_GD (a gradient step of the latent update): acc = (X G)(row, col); with R = Ph + Pl
+    // (ld ldr) and eta = 1 / *gd_max: X[row][col] <- X - eta (acc - R) (X: FP32, ld ldf, in
+    // place) and its hi + lo split to Fhi/Flo (ld ldr), the next step's operand
+    const float *gd_max;
     NsState *ns;
     unsigned int *zero;   // EPI_GRAM: zero_words words zeroed before the tiles (counters
     int zero_words;       // of the factorisation that follows on another stream)

@@ -844,6 +844,102 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// =================================================================================
+// Gradient-descent latent update (solver variant): step size, operand split, and the
+// state update that the solve epilogue performs on the exact path.
+// =================================================================================
+__global__ void __launch_bounds__(256)
+    gd_rowabs_max_kernel(const float *__restrict__ G, int r, unsigned int *maxbits) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    if (row >= r) return;
+    float v = 0.f;
+    for (int j = lane; j < r; j += 32) v += fabsf(G[(int64_t)row * r + j]);
+    v = warp_sum(v);
+    if (lane == 0) atomicMax(maxbits, __float_as_uint(v));
+}
+
+cudaError_t gd_rowabs_max(const float *G, int32_t r, unsigned int *maxbits, cudaStream_t s) {
+    gd_rowabs_max_kernel<<<(unsigned)ceil_div(r, 8), 256, 0, s>>>(G, r, maxbits);
+    count_launch();
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    split_rows_kernel(const float *__restrict__ X, int64_t rows, int r, int64_t ldf,
+                      __nv_bfloat16 *Ph, __nv_bfloat16 *Pl, int64_t ldp) {
+    const int64_t total = rows * r;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / r;
+        const int k = (int)(e - i * r);
+        split_bf16(X[i * ldf + k], Ph + i * ldp + k, Pl + i * ldp + k);
+    }
+}
+
+cudaError_t split_rows(const float *X, int64_t rows, int32_t r, int64_t ldf,
+                       __nv_bfloat16 *Ph, __nv_bfloat16 *Pl, int64_t ldp, cudaStream_t s) {
+    split_rows_kernel<<<kRedBlocks, 256, 0, s>>>(X, rows, r, ldf, Ph, Pl, ldp);
+    count_launch();
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    gd_finalize_kernel(const float *__restrict__ X, float *S, const float *__restrict__ a,
+                       const float *__restrict__ b, int64_t rows, int r, int64_t ldf, float rho,
+                       const __nv_bfloat16 *__restrict__ Rhi, const __nv_bfloat16 *__restrict__ Rlo,
+                       int64_t ldr, __nv_bfloat16 *Xt, __nv_bfloat16 *XtL, int64_t ldxt,
+                       int objective, double *part, int *err) {
+    __shared__ double sh[256];
+    const int64_t total = rows * r;
+    double acc = 0.0;
+    bool bad = false;
+    // row-major walk: the reads of X, S and R and the store of S are coalesced, the
+    // transposed stores of the operand copy are not
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / r;
+        const int k = (int)(e - i * r);
+        const float x = X[i * ldf + k];
+        bad |= !isfinite(x);
+        const float so = S[i * ldf + k];
+        const float z = (so < 0.f ? -1.f : 1.f) * a[i] * b[k];
+        S[i * ldf + k] = x + so - z;
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        float xo = __bfloat162float(h);
+        Xt[(int64_t)k * ldxt + i] = h;
+        if (XtL) {
+            const __nv_bfloat16 l = __float2bfloat16_rn(x - xo);
+            XtL[(int64_t)k * ldxt + i] = l;
+            xo += __bfloat162float(l);
+        }
+        if (objective) {
+            const float rr = __bfloat162float(Rhi[i * ldr + k]) + __bfloat162float(Rlo[i * ldr + k]);
+            acc += (double)((rr - rho * (2.f * z - so)) * xo);
+        }
+    }
+    if (bad) raise_error(err, NQ_ERR_NONFINITE);
+    if (!objective) return;
+    sh[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) part[blockIdx.x] = sh[0];
+}
+
+cudaError_t gd_finalize(const float *X, float *S, const float *a, const float *b, int64_t rows,
+                        int32_t r, int64_t ldf, float rho, const __nv_bfloat16 *Rhi,
+                        const __nv_bfloat16 *Rlo, int64_t ldr, __nv_bfloat16 *Xt,
+                        __nv_bfloat16 *XtL, int64_t ldxt, int objective, double *part,
+                        int nparts, int *err, cudaStream_t s) {
+    gd_finalize_kernel<<<(unsigned)nparts, 256, 0, s>>>(X, S, a, b, rows, r, ldf, rho, Rhi, Rlo,
+                                                         ldr, Xt, XtL, ldxt, objective, part, err);
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t gram_reduce(const float *P, int T, int S, int r, float diag, float *G,
                         __nv_bfloat16 *Gh, __nv_bfloat16 *Gl, int64_t ldg, cudaStream_t s) {
     gram_reduce_kernel<<<dim3((unsigned)T, 16), 256, 0, s>>>(P, T, S, r, diag, G, Gh, Gl, ldg);

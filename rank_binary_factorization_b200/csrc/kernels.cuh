@@ -79,6 +79,23 @@ cudaError_t bin_expand(const uint32_t *Up, const uint32_t *Vp, const float *s2, 
                        cudaStream_t s);
 
 // ---- split-K Gram reduction ------------------------------------------------------
+// ---- gradient-descent latent update (solver variant) --------------------------------
+// *maxbits = bits of max_i sum_j |G_ij| (non-negative floats order as their bits; the word
+// must be zero before the launch).
+cudaError_t gd_rowabs_max(const float *G, int32_t r, unsigned int *maxbits, cudaStream_t s);
+// Ph/Pl[i][k] = hi / lo BF16 split of X[i][k] (rows x r, X stride ldf, P stride ldp).
+cudaError_t split_rows(const float *X, int64_t rows, int32_t r, int64_t ldf,
+                       __nv_bfloat16 *Ph, __nv_bfloat16 *Pl, int64_t ldp, cudaStream_t s);
+// The solve epilogue's state update for a latent X formed elsewhere: S <- X + S - sign(S) a b^T,
+// Xt[k][i] = bf16(X[i][k]) (+ XtL the low part when set), and, when ``objective`` is set,
+// nparts FP64 partial sums of (R - rho (2 Z - S_old)) . xo into part (xo: X as the operands
+// hold it, R = Rhi + Rlo).  A non-finite X raises NQ_ERR_NONFINITE.
+cudaError_t gd_finalize(const float *X, float *S, const float *a, const float *b, int64_t rows,
+                        int32_t r, int64_t ldf, float rho, const __nv_bfloat16 *Rhi,
+                        const __nv_bfloat16 *Rlo, int64_t ldr, __nv_bfloat16 *Xt,
+                        __nv_bfloat16 *XtL, int64_t ldxt, int objective, double *part,
+                        int nparts, int *err, cudaStream_t s);
+
 // G (r x r) = sum_{s < S} P[s * T + t] (raw 128 x 128 lower-triangular tiles t < T) +
 // diag I, each off-diagonal tile also stored mirrored.
 // Gh/Gl (optional, ld ldg): the same Gram split into hi + lo BF16.

@@ -76,7 +76,8 @@ struct LbLayout {
     size_t scal = 0, what = 0, whatT = 0, whatL = 0, whatTL = 0, x[2] = {0, 0}, s[2] = {0, 0},
            a[2] = {0, 0}, b[2] = {0, 0}, xt[2] = {0, 0}, xtl[2] = {0, 0}, rhi = 0, rlo = 0, g[2] = {0, 0}, chA = 0, chLi = 0,
            gih[2] = {0, 0}, gil[2] = {0, 0}, gsh = 0, gsl = 0, nqh[2] = {0, 0}, nql[2] = {0, 0},
-           nth = 0, ntl = 0, nspart = 0, ns = 0, lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
+           nth = 0, ntl = 0, nspart = 0, ns = 0, gdh[2] = {0, 0}, gdl[2] = {0, 0}, gdmax = 0,
+           lth = 0, ltl = 0, chF = 0, tvec = 0, bcur = 0, gk = 0, part = 0, partn = 0, partg = 0,
            partb = 0, obj = 0, gpart = 0, total = 0;
     size_t part_doubles = 0;   // capacity of ``part`` (doubles): one per GEMM tile
 
@@ -135,6 +136,13 @@ struct LbLayout {
         ntl = take((size_t)r * ldr * 2);
         nspart = take((size_t)((r + 127) / 128) * ((r + 63) / 64) * 8);
         ns = take(sizeof(NsState));
+        // gradient-descent variant: the latent split into hi + lo (two buffers, the GEMM of
+        // a step reads one and its epilogue writes the other) and the step size's bound
+        for (int sd = 0; sd < 2; ++sd) {
+            gdh[sd] = take((size_t)maxrows * ldr * 2);
+            gdl[sd] = take((size_t)maxrows * ldr * 2);
+        }
+        gdmax = take(sizeof(unsigned int));
         lth = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 hi
         ltl = take((size_t)r * ldr * 2);   // (L^-1)^T, bf16 lo
         chF = take((size_t)2 * (rp / 64) * (rp / 64) * 4);  // Cholesky / inverse tile counters

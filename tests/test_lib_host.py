@@ -184,3 +184,13 @@ def test_inverse_mode_and_tuning_settings_are_checked():
     for key, v in (("factor_ctas", -1), ("newton_bn", 0), ("svid_beside", 1), ("nfast", 1),
                    ("rhs_bn", 0), ("solve_bn", 0), ("newton_fused", 0)):
         assert L.nq_set_tuning(T[key], v) == 0
+
+
+def test_latent_solver_setting_is_checked():
+    nq = _lib()
+    L = nq.lib
+    INV = 1
+    assert L.nq_set_latent_solver(1, 8) == 0
+    assert L.nq_set_latent_solver(1, 0) == INV and L.nq_set_latent_solver(1, 1001) == INV
+    assert L.nq_set_latent_solver(2, 8) == INV and L.nq_set_latent_solver(-1, 8) == INV
+    assert L.nq_set_latent_solver(0, 0) == 0      # the step count only matters for GD
