@@ -189,7 +189,9 @@ typedef enum { NQ_SOLVER_EXACT = 0, NQ_SOLVER_GD = 1 } nq_latent_solver;
 nq_status nq_set_latent_solver(nq_latent_solver solver, int32_t gd_steps);
 
 /*
- * Scheduling settings of the LB-ADMM iterations (process-wide; none changes a result):
+ * Scheduling settings of the LB-ADMM iterations (process-wide; none changes what is
+ * computed, though a tile width can regroup the objective's partial sums and so its last
+ * bits):
  * NQ_TUNE_FACTOR_CTAS: CTAs given to forming G^-1 (factorisation or update) while the
  *   RHS GEMM runs on the other SMs: -1 (default) half of the SMs up to r = 1536, else no
  *   overlap; 0 no overlap; n >= 1: n CTAs (at least 3, at most all SMs but one).

@@ -355,7 +355,7 @@ std::atomic<int> g_inverse_mode{NQ_INV_AUTO};
 std::atomic<int> g_solver{NQ_SOLVER_EXACT};
 std::atomic<int> g_gd_steps{8};
 
-// Performance settings of nq_set_tuning (none changes a result).
+// Performance settings of nq_set_tuning (none changes what is computed).
 std::atomic<int> g_tune[NQ_TUNE_COUNT] = {{-1}, {0}, {1}, {1}, {0}, {0}, {0}};
 
 // Tile widths of the RHS GEMM and of the solve (the objective's partials follow the solve's).
