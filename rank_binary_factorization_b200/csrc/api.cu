@@ -380,6 +380,10 @@ long long iters_since_prepare(const void *ws) {
 }
 void add_iters(const void *ws, long long k) {
     std::lock_guard<std::mutex> g(g_iter_mu);
+    // bounded: a process that prepares very many distinct workspaces forgets the older
+    // counts (their next updates start a few iterations later; results do not change)
+    if (g_iter_count.size() >= 4096 && g_iter_count.find(ws) == g_iter_count.end())
+        g_iter_count.clear();
     if (k < 0)
         g_iter_count[ws] = 0;
     else
@@ -524,7 +528,6 @@ nq_status lb_objective(const Lb &lb, float c, int slot, cudaStream_t s);
 // solve epilogue (dual state, transposed operand copy, objective partials on the V side).
 nq_status lb_gd_steps(const Lb &lb, int side, float rho, int prec, cudaStream_t s) {
     const LbLayout &L = lb.L;
-    const int other = 1 - side;
     const int64_t rows = L.rows(side);
     const int BN = solve_bn(L.r);
     const int steps = g_gd_steps.load(std::memory_order_relaxed);
@@ -566,7 +569,6 @@ nq_status lb_gd_steps(const Lb &lb, int side, float rho, int prec, cudaStream_t 
                       prec == NQ_PREC_FP32 ? lb.p<__nv_bfloat16>(L.xtl[side]) : nullptr,
                       L.ld_rows(side), side == 1, lb.p<double>(L.part),
                       side == 1 ? npx : kRedBlocks, &lb.sc->err, s));
-    (void)other;
     return NQ_OK;
 }
 
