@@ -384,7 +384,9 @@ nq_status nq_lbadmm_state_field(int64_t m, int64_t n, int32_t r, nq_field f, voi
 
 /* Re-derive the BF16 operand copies (transposes of U and V, with their low parts at
  * NQ_PREC_FP32, and W^^T) after a caller has written NQ_FIELD_U / NQ_FIELD_V /
- * NQ_FIELD_WHAT (/ NQ_FIELD_WHAT_LO) directly. */
+ * NQ_FIELD_WHAT (/ NQ_FIELD_WHAT_LO) directly.  A warm start from a similar layer is
+ * nq_lbadmm_prepare, then the other layer's V written into NQ_FIELD_V, then this call,
+ * then nq_lbadmm_iterate. */
 nq_status nq_lbadmm_sync_operands(int64_t m, int64_t n, int32_t r, nq_precision prec, void *ws,
                                   size_t ws_bytes, nq_stream_t stream);
 
