@@ -194,3 +194,21 @@ def test_latent_solver_setting_is_checked():
     assert L.nq_set_latent_solver(1, 0) == INV and L.nq_set_latent_solver(1, 1001) == INV
     assert L.nq_set_latent_solver(2, 8) == INV and L.nq_set_latent_solver(-1, 8) == INV
     assert L.nq_set_latent_solver(0, 0) == 0      # the step count only matters for GD
+
+
+def _declared_arities():
+    src = open(os.path.join(ROOT, "include", "nq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(nq_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    from rank_binary_factorization_b200._lib import SIGNATURES
+    arity = _declared_arities()
+    assert set(arity) == set(SIGNATURES)
+    for name, (_, args) in SIGNATURES.items():
+        assert len(args) == arity[name], (name, len(args), arity[name])
