@@ -79,3 +79,10 @@ def test_peaks_measured_or_fallback(tmp_path, monkeypatch):
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(dict(hbm_gbs=1.0, bf16_tflops=2.0)))
     g = bench.read_peaks()
     assert g["source"] == "measured" and g["bf16_tflops_sustained"] == 2.0
+
+
+def test_update_units_count_its_own_products():
+    # two r x r x r products (2 r^3 each) per step of the Newton-Schulz update
+    amount, unit, bound = bench.kernel_units("newton", 11008, 4096, 1000, 4, 262144, ns_steps=4)
+    assert (unit, bound) == ("FLOP", "tensor") and amount == 4.0 * 1000 ** 3 * 4
+    assert bench.kernel_units("newton", 11008, 4096, 1000, 4, 262144, ns_steps=0)[0] == 4.0e9
